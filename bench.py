@@ -1,0 +1,423 @@
+#!/usr/bin/env python
+"""Benchmark of the VDA linear branch (prepare -> bidirectional scan -> readout).
+
+One step = one pass of the whole path over one synthetic batch of the chosen
+workload (default: the H3-like clip, B=1 H=24 d=128 T=40 U=1560 c=5 L=512, bf16
+storage, fp32 state), with inputs resident in HBM. Prints one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config h3] [--impl reference]
+
+N > 1 is launched with torch.distributed.run: every rank processes its own
+batch (independent problems, no data-path collective: weak scaling); the timed
+region is bracketed by barriers and the time is the max over ranks.
+`--impl reference` times the float64 CPU oracle on the host cores instead (rank
+0 only), one (batch, head) pair of the workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from frame_level_delta_b200.inputs import CONFIGS, make_inputs  # noqa: E402
+
+METRIC = "VDA bidir scan+readout tokens/s per head-layer; % of B200 bf16 tensor/HBM peak"
+UNIT = "head-tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def workload_desc(cfg) -> str:
+    extra = ", conv prep + RMSNorm/gate" if cfg.prep_conv else ""
+    return (f"{cfg.name}: B={cfg.B} H={cfg.H} d={cfg.d} T={cfg.T} U={cfg.U} ({cfg.grid_h}x{cfg.grid_w}) "
+            f"c={cfg.chunk} L={cfg.L} {cfg.dtype} storage, fp32 state{extra}")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------
+# Algorithmic bytes / flops per launch of each kernel (each input byte read
+# once, each output byte written once).
+# ----------------------------------------------------------------------------
+def kernel_bytes(name: str, cfg) -> float:
+    B, H, d, T, U, L, c = cfg.B, cfg.H, cfg.d, cfg.T, cfg.U, cfg.L, cfg.chunk
+    esz = 4 if cfg.dtype == "f32" else 2
+    F, NS, J = T - 2, T - 1, cfg.J
+    BH = B * H
+    dd4 = d * d * 4
+    if name in ("gram_tc", "gram_simt"):
+        return BH * ((F * U + L) * (2 * d * esz + 4) + 2 * NS * dd4)
+    if name == "solve_simt":
+        return BH * (4 * NS * dd4 + F * d * 4)
+    if name == "scan_simt":
+        fwd = max(0, c * (J - 2) - 1)
+        rev = max(0, (T - 2) - 2 * c + 1)
+        return BH * ((fwd + rev) * 2 * dd4 + 2 * dd4 + 2 * J * dd4)
+    if name in ("readout_tc", "readout_simt"):
+        gate = 1 if cfg.norm_gate else 0
+        return BH * (F * U * d * esz * (2 + gate) + 2 * J * dd4)
+    if name == "zero_anchors":
+        return BH * 2 * U * d * esz
+    if name == "prep_video":
+        return BH * (2 * T * U * d * esz + 2 * F * U * d * esz)
+    if name == "prep_text":
+        return BH * 4 * L * d * esz
+    return 0.0
+
+
+def path_bytes(cfg) -> float:
+    """Algorithmic bytes of one whole step: Q, K, V, beta read and O written once on
+    non-anchor frames, plus text, alpha, anchor zero-fill (and, with conv prep,
+    K and V of every frame plus the gate)."""
+    B, H, d, T, U, L = cfg.B, cfg.H, cfg.d, cfg.T, cfg.U, cfg.L
+    esz = 4 if cfg.dtype == "f32" else 2
+    F = T - 2
+    per_head = F * U * (4 * d * esz + 4) + L * (2 * d * esz + 4) + F * d * 4 + 2 * U * d * esz
+    if cfg.prep_conv:
+        per_head += 2 * 2 * U * d * esz + F * U * d * esz  # anchor-frame K, V for the conv; gate
+    return B * H * per_head
+
+
+def path_flops(cfg) -> float:
+    B, H, d, T, U, L, c = cfg.B, cfg.H, cfg.d, cfg.T, cfg.U, cfg.L, cfg.chunk
+    F, NS, J = T - 2, T - 1, cfg.J
+    gram = (F * U + L) * 4 * d * d
+    solve = NS * (d ** 3 + 2 * d ** 3)  # Cholesky + L^-1 + L^-T L^-1 (~d^3) and C = B P (2 d^3)
+    fwd = max(0, c * (J - 2) - 1)
+    rev = max(0, (T - 2) - 2 * c + 1)
+    scan = (fwd + rev) * 2 * d ** 3
+    readout = F * U * 2 * d * d
+    return B * H * (gram + solve + scan + readout)
+
+
+def source_digest(kernel: str):
+    files = {"gram_tc": "gram_tc.cu", "readout_tc": "readout_tc.cu"}
+    fn = files.get(kernel, "kernels_simt.cu")
+    p = os.path.join(ROOT, "frame_level_delta_b200", "csrc", fn)
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def traffic_for(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, only if the kernel's
+    source is unchanged since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        tab = json.load(f)
+    e = tab.get(workload, {}).get(kernel)
+    if not e or e.get("source_sha") != source_digest(kernel):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------
+# Clock sampling during the timed region (NVML, the library nvidia-smi uses).
+# ----------------------------------------------------------------------------
+REASON_BITS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+
+class ClockSampler:
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.ok = False
+        self.samples = []
+        self.reasons = 0
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            props = torch.cuda.get_device_properties(device_index)
+            h = None
+            uuid = getattr(props, "uuid", None)
+            if uuid is not None:
+                s = str(uuid)
+                for cand in (s if s.startswith("GPU-") else "GPU-" + s,):
+                    try:
+                        h = pynvml.nvmlDeviceGetHandleByUUID(cand)
+                    except Exception:
+                        h = None
+            if h is None:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+                idx = device_index
+                parts = [x for x in vis.split(",") if x.strip()]
+                if parts and parts[min(device_index, len(parts) - 1)].strip().isdigit():
+                    idx = int(parts[device_index].strip())
+                h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.h = h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report that, do not guess
+            self.err = repr(e)
+
+    def _sample(self):
+        nv = self.nv
+        sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.samples.append(sm)
+        self.reasons |= r
+
+    def _loop(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def start(self):
+        if not self.ok:
+            return
+        self._stop = threading.Event()
+        self._t = threading.Thread(target=self._loop, daemon=True)
+        self._t.start()
+
+    def stop(self):
+        if not self.ok:
+            return
+        self._stop.set()
+        self._t.join()
+        try:
+            self._sample()
+        except Exception:
+            pass
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": getattr(self, "err", "no samples")}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": [n for b, n in REASON_BITS.items() if self.reasons & b],
+                "samples": len(self.samples), "source": "nvml"}
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing (test infrastructure; bench.py's CPU-baseline leg)
+# ----------------------------------------------------------------------------
+def blas_threads() -> int:
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        for d in info:
+            if d.get("user_api") == "blas":
+                return int(d.get("num_threads"))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def time_oracle(cfg, inp, heads, budget_s=None):
+    from oracle.vda_oracle import vda_reference
+    done = 0
+    t0 = time.perf_counter()
+    for bh in heads:
+        vda_reference(inp, cfg, heads=[bh], keep=False)
+        done += 1
+        if budget_s is not None and time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return done, dt
+
+
+def cpu_baseline(cfg, inp, budget_s=10.0):
+    heads = [(b, h) for b in range(cfg.B) for h in range(cfg.H)]
+    done, dt = time_oracle(cfg, inp, heads, budget_s=budget_s)
+    value = done * cfg.T * cfg.U / dt
+    return {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"float64 numpy oracle over {done} of {len(heads)} (batch, head) pairs of the "
+                      f"workload ({cfg.T * cfg.U} tokens each), {dt:.2f} s, BLAS threads={blas_threads()}"}
+
+
+def run_reference(args, cfg, rank):
+    if rank != 0:
+        return 0
+    inp = make_inputs(cfg)
+    heads = [(b, h) for b in range(cfg.B) for h in range(cfg.H)]
+    for i in range(args.warmup):
+        time_oracle(cfg, inp, [heads[i % len(heads)]])
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        time_oracle(cfg, inp, [heads[i % len(heads)]])
+    dt = time.perf_counter() - t0
+    value = args.steps * cfg.T * cfg.U / dt
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": workload_desc(cfg), "step": "one (batch, head) pair of the workload"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"one (batch, head) pair per step, {cfg.T * cfg.U} tokens"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="h3", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="vda", choices=["vda", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work (0: skip)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = CONFIGS[args.config]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, cfg, rank)
+
+    from frame_level_delta_b200 import vda as V
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    # Each rank draws its own batch (independent problems).
+    inp_cpu = make_inputs(cfg, seed=cfg.seed + rank)
+    inp_host = {k: v.pin_memory() for k, v in inp_cpu.items()}
+    inp_dev = {k: v.to(dev, non_blocking=True) for k, v in inp_host.items()}
+    lib = V.VDA(cfg, device=dev)
+    O = lib.new_output()
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        lib.run(inp_dev, O)
+    torch.cuda.synchronize(dev)
+    if lib.poll_device_status() != 0:
+        raise RuntimeError("device status reported a timeout during warm-up")
+
+    # ---- device-timed region: inputs resident in HBM (each step's working set,
+    # ~1.5 GB at the H3-like clip, is larger than the 126 MB L2) -------------
+    lib.profile_enable(True)
+    n0 = lib.launch_count()
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        lib.run(inp_dev, O)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.stop()
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    launches = lib.launch_count() - n0
+    prof = lib.profile_read()
+    lib.profile_enable(False)
+    if lib.poll_device_status() != 0:
+        raise RuntimeError("device status reported a timeout in the timed region")
+    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+    units = world * cfg.head_tokens * args.steps
+    value = units / (ms_max / 1e3)
+
+    # ---- end to end through the public API: pinned host inputs -> device ->
+    # prepare/scan/readout -> O back to pinned host memory, every step --------
+    O_host = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in inp_host.values())
+    d2h = O.numel() * O.element_size()
+    ke = max(1, min(args.e2e_steps, args.steps))
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(ke):
+        for k, v in inp_host.items():
+            inp_dev[k].copy_(v, non_blocking=True)
+        lib.run(inp_dev, O)
+        O_host.copy_(O, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    t = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_value = world * cfg.head_tokens * ke / (float(t.item()) / 1e3)
+
+    # ---- roofline of the dominant kernel (live per-kernel CUDA events) -------
+    peaks, peak_src = load_peaks()
+    dom = max(prof.items(), key=lambda kv: kv[1][1])
+    dom_name, (dom_n, dom_ms) = dom
+    dom_avg_s = dom_ms / dom_n / 1e3
+    dom_bytes = kernel_bytes(dom_name, cfg)
+    achieved = dom_bytes / dom_avg_s / 1e9
+    peak = float(peaks["hbm_gbs"])
+    traffic = traffic_for(dom_name, cfg.name)
+    kernels = {k: {"launches": n, "avg_us": tot / n * 1e3, "share": tot / sum(x[1] for x in prof.values()),
+                   "algorithmic_GBps": kernel_bytes(k, cfg) / (tot / n / 1e3) / 1e9}
+               for k, (n, tot) in prof.items()}
+
+    if rank == 0:
+        step_s = ms_max / 1e3 / args.steps
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32",
+            "data": "synthetic",
+            "config": {"workload": workload_desc(cfg), "global_batch": cfg.B * world,
+                       "parallelism": f"dp{world} (independent batches, no collective)",
+                       "l2": "no flush: each step reads and writes > 1 GB, far above the 126 MB L2",
+                       "path": V.describe(lib.c),
+                       "stream": "one CUDA stream, kernels back to back"},
+            "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": peak,
+                         "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"hbm_gbs of {peak_src}",
+                         "algorithmic_bytes_per_launch": dom_bytes},
+            "path_roofline": {"algorithmic_bytes_per_step": path_bytes(cfg),
+                              "hbm_GBps": path_bytes(cfg) / step_s / 1e9,
+                              "hbm_frac": path_bytes(cfg) / step_s / 1e9 / peak,
+                              "tflops": path_flops(cfg) / step_s / 1e12,
+                              "tensor_frac_of_bf16_burst": path_flops(cfg) / step_s / 1e12 / float(peaks["bf16_tflops"])},
+            "kernels": kernels,
+            "gpu_launches": launches,
+            "clocks": clocks.summary(),
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": ke},
+        }
+        if world == 1 and args.cpu_budget > 0:
+            line["cpu_baseline"] = cpu_baseline(cfg, inp_cpu, budget_s=args.cpu_budget)
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

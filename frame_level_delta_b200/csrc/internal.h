@@ -1,0 +1,87 @@
+// Internal definitions shared by the host orchestration (vda_api.cu) and the
+// kernel translation units. Not part of the C ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/vda.h"
+
+namespace vda {
+
+// A strided view of token vectors: element (b, h, t, u, k) of a token tensor
+// lives at p + b*s_b + h*s_h + t*s_t + u*s_u + k (in elements).
+struct TokView {
+  const void* p;
+  long long s_b, s_h, s_t, s_u;
+};
+
+// Everything a kernel needs, passed by value.
+struct Problem {
+  int B, H, T, U, L, D, c, J, gh, gw;
+  int bf16;            // 1: token tensors are bf16, 0: fp32
+  unsigned flags;
+  float l2_eps, rms_eps;
+  // Video and text keys/values as read by the statistics kernel (raw inputs, or
+  // the prepared copies in the workspace under VDA_PREP_CONV).
+  TokView Kv, Vv, Kt, Vt;
+  const float* alpha;     // [B,H,T,D]
+  const float* beta;      // [B,H,T,U]
+  const float* beta_txt;  // [B,H,L]
+  const void* Q;          // [B,T*U,H,D]
+  // Workspace regions (fp32 unless noted).
+  uint32_t* status;
+  float* A;     // [B,H,T-1,D,D]
+  float* Bm;    // [B,H,T-1,D,D]
+  float* M;     // [B,H,T-1,D,D]
+  float* C;     // [B,H,T-1,D,D]; slot 0 = S_T
+  float* Sf;    // [B,H,J,D,D]
+  float* Sr;    // [B,H,J,D,D]
+  void* Kp;     // [B,H,T,U,D] storage dtype (prep)
+  void* Vp;
+  void* Ktp;    // [B,H,L,D]
+  void* Vtp;
+  unsigned long long spin_limit;  // iteration bound of every device-side wait
+};
+
+// Slot s of the statistics / solve arrays: 0 = text, t = frame t (1..T-2).
+inline __host__ __device__ long long slot_off(const Problem& p, int b, int h, int s) {
+  return (((long long)b * p.H + h) * (p.T - 1) + s) * (long long)p.D * p.D;
+}
+inline __host__ __device__ long long chunk_off(const Problem& p, int b, int h, int j) {
+  return (((long long)b * p.H + h) * p.J + j) * (long long)p.D * p.D;
+}
+
+// Kernel ids for launch accounting and profiling.
+enum KernelId {
+  K_PREP_VIDEO = 0,
+  K_PREP_TEXT,
+  K_GRAM_SIMT,
+  K_GRAM_TC,
+  K_SOLVE_SIMT,
+  K_SCAN_SIMT,
+  K_READOUT_SIMT,
+  K_READOUT_TC,
+  K_ZERO_ANCHORS,
+  K_NUM_KERNELS
+};
+const char* kernel_name(int id);
+
+// Launchers (return cudaGetLastError() after the launch).
+cudaError_t launch_prep_video(const Problem& p, const void* K, const void* V, const float* conv_w,
+                              cudaStream_t s);
+cudaError_t launch_prep_text(const Problem& p, const void* Kt, const void* Vt, cudaStream_t s);
+cudaError_t launch_gram_simt(const Problem& p, cudaStream_t s);
+cudaError_t launch_solve_simt(const Problem& p, cudaStream_t s);
+cudaError_t launch_scan_simt(const Problem& p, cudaStream_t s);
+cudaError_t launch_readout_simt(const Problem& p, const void* gate, void* O, cudaStream_t s);
+cudaError_t launch_zero_anchors(const Problem& p, void* O, cudaStream_t s);
+cudaError_t launch_selftest_wait(uint32_t* status, unsigned long long spins, cudaStream_t s);
+
+// Tensor-core (tcgen05) kernels, bf16 with D in {64, 128}.
+bool gram_tc_supported(const Problem& p);
+cudaError_t launch_gram_tc(const Problem& p, cudaStream_t s);
+bool readout_tc_supported(const Problem& p);
+cudaError_t launch_readout_tc(const Problem& p, const void* gate, void* O, cudaStream_t s);
+
+}  // namespace vda

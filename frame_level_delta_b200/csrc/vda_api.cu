@@ -1,0 +1,406 @@
+// Host side of the C ABI declared in include/vda.h: argument validation,
+// workspace carving, stage orchestration, launch accounting and per-kernel
+// event timing. Every call only enqueues work on the caller's stream.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "internal.h"
+
+namespace vda {
+
+const char* kernel_name(int id) {
+  static const char* names[K_NUM_KERNELS] = {
+      "prep_video", "prep_text", "gram_simt", "gram_tc", "solve_simt",
+      "scan_simt", "readout_simt", "readout_tc", "zero_anchors"};
+  return (id >= 0 && id < K_NUM_KERNELS) ? names[id] : "?";
+}
+
+}  // namespace vda
+
+using namespace vda;
+
+struct EventPair {
+  cudaEvent_t a, b;
+};
+
+struct vda_ctx {
+  vda_config cfg;
+  Problem p;
+  bool prepared = false, scanned = false;
+  std::string err;
+  uint64_t launches = 0;
+  bool prof = false;
+  std::vector<EventPair> pending[K_NUM_KERNELS];
+  std::vector<EventPair> pool;
+  int prof_launches[K_NUM_KERNELS] = {};
+  double prof_ms[K_NUM_KERNELS] = {};
+};
+
+namespace {
+
+constexpr size_t kRegionAlign = 1024;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int d_of(const vda_config& c) { return c.d_k; }
+int J_of(const vda_config& c) { return (c.T + c.chunk - 1) / c.chunk; }
+
+vda_status check_config(const vda_config* c, std::string* why) {
+  auto bad = [&](const char* m) {
+    if (why) *why = m;
+    return VDA_ERR_INVALID_ARG;
+  };
+  if (!c) return bad("config is NULL");
+  if (c->B < 1 || c->H < 1) return bad("B and H must be >= 1");
+  if (c->T < 3) return bad("T must be >= 3 (two anchors and one scanned frame)");
+  if (c->grid_h < 1 || c->grid_w < 1) return bad("grid_h and grid_w must be >= 1");
+  if ((long long)c->grid_h * c->grid_w != c->U) return bad("U must equal grid_h * grid_w");
+  if (c->L < 1) return bad("L (text tokens) must be >= 1");
+  if (c->chunk < 1) return bad("chunk must be >= 1");
+  if (c->dtype != VDA_F32 && c->dtype != VDA_BF16) return bad("dtype must be VDA_F32 or VDA_BF16");
+  if (!(c->l2_eps >= 0.f) || !(c->rms_eps >= 0.f)) return bad("eps must be >= 0");
+  if (c->flags & ~(VDA_PREP_CONV | VDA_READOUT_NORM_GATE | VDA_FORCE_SIMT)) return bad("unknown flag bits");
+  if (c->d_k != c->d_v) {
+    if (why) *why = "d_k != d_v is not supported";
+    return VDA_ERR_UNSUPPORTED;
+  }
+  const int d = c->d_k;
+  if (d != 16 && d != 32 && d != 64 && d != 128) {
+    if (why) *why = "d must be one of 16, 32, 64, 128";
+    return VDA_ERR_UNSUPPORTED;
+  }
+  if ((c->flags & VDA_PREP_CONV) && (size_t)c->grid_w * d * sizeof(float) > 200 * 1024) {
+    if (why) *why = "grid_w * d too large for the prep kernel's row buffer";
+    return VDA_ERR_UNSUPPORTED;
+  }
+  const long long tokens = (long long)c->B * c->T * c->U * c->H * d;
+  if (tokens >= (1LL << 40)) return bad("tensor too large");
+  return VDA_OK;
+}
+
+struct Layout {
+  size_t off[VDA_NUM_REGIONS];
+  size_t bytes[VDA_NUM_REGIONS];
+  size_t total;
+};
+
+Layout make_layout(const vda_config& c) {
+  Layout L{};
+  const size_t d = (size_t)d_of(c), BH = (size_t)c.B * c.H;
+  const size_t esz = c.dtype == VDA_BF16 ? 2 : 4;
+  const bool prep = (c.flags & VDA_PREP_CONV) != 0;
+  L.bytes[VDA_REGION_STATUS] = 256;
+  L.bytes[VDA_REGION_A] = BH * (c.T - 1) * d * d * 4;
+  L.bytes[VDA_REGION_B] = BH * (c.T - 1) * d * d * 4;
+  L.bytes[VDA_REGION_M] = BH * (c.T - 1) * d * d * 4;
+  L.bytes[VDA_REGION_C] = BH * (c.T - 1) * d * d * 4;
+  L.bytes[VDA_REGION_S_FWD] = BH * J_of(c) * d * d * 4;
+  L.bytes[VDA_REGION_S_REV] = BH * J_of(c) * d * d * 4;
+  L.bytes[VDA_REGION_K_PREP] = prep ? BH * c.T * (size_t)c.U * d * esz : 0;
+  L.bytes[VDA_REGION_V_PREP] = prep ? BH * c.T * (size_t)c.U * d * esz : 0;
+  L.bytes[VDA_REGION_KT_PREP] = prep ? BH * c.L * d * esz : 0;
+  L.bytes[VDA_REGION_VT_PREP] = prep ? BH * c.L * d * esz : 0;
+  size_t o = 0;
+  for (int r = 0; r < VDA_NUM_REGIONS; ++r) {
+    L.off[r] = o;
+    o = align_up(o + L.bytes[r], kRegionAlign);
+  }
+  L.total = o;
+  return L;
+}
+
+bool aligned16(const void* ptr) { return ((uintptr_t)ptr & 15) == 0; }
+
+vda_status fail(vda_ctx* ctx, vda_status s, const std::string& msg) {
+  if (ctx) ctx->err = msg;
+  return s;
+}
+
+vda_status cuda_fail(vda_ctx* ctx, cudaError_t e, const char* what) {
+  std::string m = std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")";
+  return fail(ctx, VDA_ERR_CUDA, m);
+}
+
+EventPair take_pair(vda_ctx* ctx) {
+  if (!ctx->pool.empty()) {
+    EventPair e = ctx->pool.back();
+    ctx->pool.pop_back();
+    return e;
+  }
+  EventPair e{};
+  cudaEventCreate(&e.a);
+  cudaEventCreate(&e.b);
+  return e;
+}
+
+// Fold finished timing pairs into the accumulators (synchronising on them).
+void drain_events(vda_ctx* ctx) {
+  for (int k = 0; k < K_NUM_KERNELS; ++k) {
+    for (EventPair& e : ctx->pending[k]) {
+      float ms = 0.f;
+      if (cudaEventSynchronize(e.b) == cudaSuccess && cudaEventElapsedTime(&ms, e.a, e.b) == cudaSuccess) {
+        ctx->prof_launches[k] += 1;
+        ctx->prof_ms[k] += ms;
+      }
+      ctx->pool.push_back(e);
+    }
+    ctx->pending[k].clear();
+  }
+}
+
+template <typename F>
+vda_status run_kernel(vda_ctx* ctx, int id, cudaStream_t s, F&& launch) {
+  EventPair ev{};
+  const bool prof = ctx->prof;
+  if (prof) {
+    if (ctx->pending[id].size() > 4096) drain_events(ctx);
+    ev = take_pair(ctx);
+    cudaEventRecord(ev.a, s);
+  }
+  cudaError_t e = launch();
+  if (e != cudaSuccess) return cuda_fail(ctx, e, kernel_name(id));
+  ctx->launches += 1;
+  if (prof) {
+    cudaEventRecord(ev.b, s);
+    ctx->pending[id].push_back(ev);
+  }
+  return VDA_OK;
+}
+
+bool use_simt_only(const vda_config& c) { return (c.flags & VDA_FORCE_SIMT) != 0; }
+
+}  // namespace
+
+extern "C" {
+
+const char* vda_status_string(vda_status s) {
+  switch (s) {
+    case VDA_OK: return "VDA_OK";
+    case VDA_ERR_INVALID_ARG: return "VDA_ERR_INVALID_ARG";
+    case VDA_ERR_UNSUPPORTED: return "VDA_ERR_UNSUPPORTED";
+    case VDA_ERR_ALIGNMENT: return "VDA_ERR_ALIGNMENT";
+    case VDA_ERR_WORKSPACE_TOO_SMALL: return "VDA_ERR_WORKSPACE_TOO_SMALL";
+    case VDA_ERR_CUDA: return "VDA_ERR_CUDA";
+    case VDA_ERR_TIMEOUT: return "VDA_ERR_TIMEOUT";
+    case VDA_ERR_STATE: return "VDA_ERR_STATE";
+  }
+  return "VDA_ERR_UNKNOWN";
+}
+
+vda_status vda_create(const vda_config* cfg, vda_ctx** out) {
+  if (!out) return VDA_ERR_INVALID_ARG;
+  *out = nullptr;
+  vda_status st = check_config(cfg, nullptr);
+  if (st != VDA_OK) return st;
+  vda_ctx* ctx = new (std::nothrow) vda_ctx();
+  if (!ctx) return VDA_ERR_INVALID_ARG;
+  ctx->cfg = *cfg;
+  *out = ctx;
+  return VDA_OK;
+}
+
+vda_status vda_destroy(vda_ctx* ctx) {
+  if (!ctx) return VDA_ERR_INVALID_ARG;
+  for (int k = 0; k < K_NUM_KERNELS; ++k)
+    for (EventPair& e : ctx->pending[k]) ctx->pool.push_back(e);
+  for (EventPair& e : ctx->pool) {
+    cudaEventDestroy(e.a);
+    cudaEventDestroy(e.b);
+  }
+  delete ctx;
+  return VDA_OK;
+}
+
+vda_status vda_workspace_size(const vda_config* cfg, size_t* bytes) {
+  if (!bytes) return VDA_ERR_INVALID_ARG;
+  vda_status st = check_config(cfg, nullptr);
+  if (st != VDA_OK) return st;
+  *bytes = make_layout(*cfg).total;
+  return VDA_OK;
+}
+
+vda_status vda_workspace_region(const vda_config* cfg, int region, size_t* offset, size_t* bytes) {
+  if (!offset || !bytes || region < 0 || region >= VDA_NUM_REGIONS) return VDA_ERR_INVALID_ARG;
+  vda_status st = check_config(cfg, nullptr);
+  if (st != VDA_OK) return st;
+  Layout L = make_layout(*cfg);
+  *offset = L.off[region];
+  *bytes = L.bytes[region];
+  return VDA_OK;
+}
+
+const char* vda_last_error(const vda_ctx* ctx) { return ctx ? ctx->err.c_str() : ""; }
+
+vda_status vda_describe(const vda_config* cfg, const char** text) {
+  if (!text) return VDA_ERR_INVALID_ARG;
+  vda_status st = check_config(cfg, nullptr);
+  if (st != VDA_OK) return st;
+  Problem p{};
+  p.D = cfg->d_k;
+  p.bf16 = cfg->dtype == VDA_BF16;
+  p.flags = cfg->flags;
+  const bool simt = use_simt_only(*cfg);
+  const bool g = !simt && gram_tc_supported(p), r = !simt && readout_tc_supported(p);
+  static const char* table[2][2] = {
+      {"gram=simt solve=simt scan=simt readout=simt", "gram=simt solve=simt scan=simt readout=tcgen05"},
+      {"gram=tcgen05 solve=simt scan=simt readout=simt", "gram=tcgen05 solve=simt scan=simt readout=tcgen05"}};
+  *text = table[g][r];
+  return VDA_OK;
+}
+
+vda_status vda_prepare(vda_ctx* ctx, const void* Q, const void* K, const void* V, const void* K_txt,
+                       const void* V_txt, const float* alpha, const float* beta, const float* beta_txt,
+                       const float* conv_w, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!ctx) return VDA_ERR_INVALID_ARG;
+  ctx->prepared = ctx->scanned = false;
+  const vda_config& c = ctx->cfg;
+  const bool prep = (c.flags & VDA_PREP_CONV) != 0;
+  if (!Q || !K || !V || !K_txt || !V_txt || !alpha || !beta || !beta_txt || !workspace)
+    return fail(ctx, VDA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (prep && !conv_w) return fail(ctx, VDA_ERR_INVALID_ARG, "conv_w is required with VDA_PREP_CONV");
+  const void* ptrs[] = {Q, K, V, K_txt, V_txt, alpha, beta, beta_txt};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return fail(ctx, VDA_ERR_ALIGNMENT, "token tensors, alpha and beta must be 16-byte aligned");
+  if (prep && !aligned16(conv_w)) return fail(ctx, VDA_ERR_ALIGNMENT, "conv_w must be 16-byte aligned");
+  if (((uintptr_t)workspace & 255) != 0) return fail(ctx, VDA_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  const Layout L = make_layout(c);
+  if (workspace_bytes < L.total) return fail(ctx, VDA_ERR_WORKSPACE_TOO_SMALL, "workspace smaller than vda_workspace_size()");
+
+  char* ws = static_cast<char*>(workspace);
+  Problem& p = ctx->p;
+  p = Problem{};
+  p.B = c.B; p.H = c.H; p.T = c.T; p.U = c.U; p.L = c.L; p.D = c.d_k; p.c = c.chunk; p.J = J_of(c);
+  p.gh = c.grid_h; p.gw = c.grid_w;
+  p.bf16 = c.dtype == VDA_BF16;
+  p.flags = c.flags;
+  p.l2_eps = c.l2_eps;
+  p.rms_eps = c.rms_eps;
+  p.alpha = alpha; p.beta = beta; p.beta_txt = beta_txt; p.Q = Q;
+  p.status = reinterpret_cast<uint32_t*>(ws + L.off[VDA_REGION_STATUS]);
+  p.A = reinterpret_cast<float*>(ws + L.off[VDA_REGION_A]);
+  p.Bm = reinterpret_cast<float*>(ws + L.off[VDA_REGION_B]);
+  p.M = reinterpret_cast<float*>(ws + L.off[VDA_REGION_M]);
+  p.C = reinterpret_cast<float*>(ws + L.off[VDA_REGION_C]);
+  p.Sf = reinterpret_cast<float*>(ws + L.off[VDA_REGION_S_FWD]);
+  p.Sr = reinterpret_cast<float*>(ws + L.off[VDA_REGION_S_REV]);
+  p.spin_limit = 1ull << 26;
+  const long long D = p.D, H = p.H, T = p.T, U = p.U, Lt = p.L;
+  if (prep) {
+    p.Kp = ws + L.off[VDA_REGION_K_PREP];
+    p.Vp = ws + L.off[VDA_REGION_V_PREP];
+    p.Ktp = ws + L.off[VDA_REGION_KT_PREP];
+    p.Vtp = ws + L.off[VDA_REGION_VT_PREP];
+    p.Kv = TokView{p.Kp, H * T * U * D, T * U * D, U * D, D};
+    p.Vv = TokView{p.Vp, H * T * U * D, T * U * D, U * D, D};
+    p.Kt = TokView{p.Ktp, H * Lt * D, Lt * D, 0, D};
+    p.Vt = TokView{p.Vtp, H * Lt * D, Lt * D, 0, D};
+  } else {
+    p.Kv = TokView{K, T * U * H * D, D, U * H * D, H * D};
+    p.Vv = TokView{V, T * U * H * D, D, U * H * D, H * D};
+    p.Kt = TokView{K_txt, Lt * H * D, D, 0, H * D};
+    p.Vt = TokView{V_txt, Lt * H * D, D, 0, H * D};
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(p.status, 0, 256, s);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "status reset");
+  vda_status st;
+  if (prep) {
+    st = run_kernel(ctx, K_PREP_VIDEO, s, [&] { return launch_prep_video(p, K, V, conv_w, s); });
+    if (st != VDA_OK) return st;
+    st = run_kernel(ctx, K_PREP_TEXT, s, [&] { return launch_prep_text(p, K_txt, V_txt, s); });
+    if (st != VDA_OK) return st;
+  }
+  if (!use_simt_only(c) && gram_tc_supported(p))
+    st = run_kernel(ctx, K_GRAM_TC, s, [&] { return launch_gram_tc(p, s); });
+  else
+    st = run_kernel(ctx, K_GRAM_SIMT, s, [&] { return launch_gram_simt(p, s); });
+  if (st != VDA_OK) return st;
+  st = run_kernel(ctx, K_SOLVE_SIMT, s, [&] { return launch_solve_simt(p, s); });
+  if (st != VDA_OK) return st;
+  ctx->prepared = true;
+  return VDA_OK;
+}
+
+vda_status vda_scan_bidir(vda_ctx* ctx, void* stream) {
+  if (!ctx) return VDA_ERR_INVALID_ARG;
+  if (!ctx->prepared) return fail(ctx, VDA_ERR_STATE, "vda_scan_bidir before a successful vda_prepare");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  vda_status st = run_kernel(ctx, K_SCAN_SIMT, s, [&] { return launch_scan_simt(ctx->p, s); });
+  if (st != VDA_OK) return st;
+  ctx->scanned = true;
+  return VDA_OK;
+}
+
+vda_status vda_readout(vda_ctx* ctx, const void* gate, void* O, void* stream) {
+  if (!ctx) return VDA_ERR_INVALID_ARG;
+  if (!ctx->scanned) return fail(ctx, VDA_ERR_STATE, "vda_readout before a successful vda_scan_bidir");
+  if (!O) return fail(ctx, VDA_ERR_INVALID_ARG, "O is NULL");
+  if ((ctx->cfg.flags & VDA_READOUT_NORM_GATE) && !gate)
+    return fail(ctx, VDA_ERR_INVALID_ARG, "gate is required with VDA_READOUT_NORM_GATE");
+  if (!aligned16(O) || (gate && !aligned16(gate))) return fail(ctx, VDA_ERR_ALIGNMENT, "O and gate must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const Problem& p = ctx->p;
+  vda_status st = run_kernel(ctx, K_ZERO_ANCHORS, s, [&] { return launch_zero_anchors(p, O, s); });
+  if (st != VDA_OK) return st;
+  if (!use_simt_only(ctx->cfg) && readout_tc_supported(p))
+    st = run_kernel(ctx, K_READOUT_TC, s, [&] { return launch_readout_tc(p, gate, O, s); });
+  else
+    st = run_kernel(ctx, K_READOUT_SIMT, s, [&] { return launch_readout_simt(p, gate, O, s); });
+  return st;
+}
+
+vda_status vda_poll_device_status(vda_ctx* ctx, void* stream) {
+  if (!ctx) return VDA_ERR_INVALID_ARG;
+  if (!ctx->p.status) return fail(ctx, VDA_ERR_STATE, "no workspace bound yet");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, ctx->p.status, sizeof(word), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "status read");
+  if (word != 0) {
+    e = cudaMemsetAsync(ctx->p.status, 0, sizeof(word), s);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "status clear");
+    return fail(ctx, VDA_ERR_TIMEOUT, "a bounded device-side wait gave up");
+  }
+  return VDA_OK;
+}
+
+vda_status vda_profile_enable(vda_ctx* ctx, int enable) {
+  if (!ctx) return VDA_ERR_INVALID_ARG;
+  drain_events(ctx);
+  for (int k = 0; k < K_NUM_KERNELS; ++k) {
+    ctx->prof_launches[k] = 0;
+    ctx->prof_ms[k] = 0.0;
+  }
+  ctx->prof = enable != 0;
+  return VDA_OK;
+}
+
+int vda_num_kernels(void) { return K_NUM_KERNELS; }
+
+vda_status vda_profile_read(vda_ctx* ctx, int kernel, const char** name, int* launches, double* total_ms) {
+  if (!ctx || kernel < 0 || kernel >= K_NUM_KERNELS) return VDA_ERR_INVALID_ARG;
+  drain_events(ctx);
+  if (name) *name = kernel_name(kernel);
+  if (launches) *launches = ctx->prof_launches[kernel];
+  if (total_ms) *total_ms = ctx->prof_ms[kernel];
+  return VDA_OK;
+}
+
+vda_status vda_launch_count(const vda_ctx* ctx, uint64_t* launches) {
+  if (!ctx || !launches) return VDA_ERR_INVALID_ARG;
+  *launches = ctx->launches;
+  return VDA_OK;
+}
+
+vda_status vda_selftest_bounded_wait(uint32_t* status_dev, uint64_t spins, void* stream) {
+  if (!status_dev || !aligned16(status_dev)) return VDA_ERR_INVALID_ARG;
+  cudaError_t e = launch_selftest_wait(status_dev, spins, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VDA_OK : VDA_ERR_CUDA;
+}
+
+}  // extern "C"

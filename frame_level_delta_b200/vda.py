@@ -1,0 +1,235 @@
+"""Thin ctypes binding of libvda.so (the C ABI in include/vda.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels. PyTorch supplies device memory and streams. Loading fails loudly if the
+library has not been built; there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+import torch
+
+from .inputs import VDAConfig
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libvda.so")
+
+VDA_OK = 0
+STATUS_NAMES = {0: "VDA_OK", 1: "VDA_ERR_INVALID_ARG", 2: "VDA_ERR_UNSUPPORTED", 3: "VDA_ERR_ALIGNMENT",
+                4: "VDA_ERR_WORKSPACE_TOO_SMALL", 5: "VDA_ERR_CUDA", 6: "VDA_ERR_TIMEOUT", 7: "VDA_ERR_STATE"}
+VDA_F32, VDA_BF16 = 0, 1
+VDA_PREP_CONV = 0x1
+VDA_READOUT_NORM_GATE = 0x2
+VDA_FORCE_SIMT = 0x100
+REGIONS = {"status": 0, "A": 1, "B": 2, "M": 3, "C": 4, "S_fwd": 5, "S_rev": 6,
+           "K_prep": 7, "V_prep": 8, "Kt_prep": 9, "Vt_prep": 10}
+
+# Exported symbols, in the order include/vda.h declares them.
+EXPORTS = ["vda_create", "vda_destroy", "vda_workspace_size", "vda_prepare", "vda_scan_bidir",
+           "vda_readout", "vda_poll_device_status", "vda_workspace_region", "vda_status_string",
+           "vda_last_error", "vda_profile_enable", "vda_num_kernels", "vda_profile_read",
+           "vda_launch_count", "vda_describe", "vda_selftest_bounded_wait"]
+
+
+class VDAError(RuntimeError):
+    def __init__(self, status: int, msg: str = ""):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+class vda_config(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("T", ctypes.c_int), ("U", ctypes.c_int),
+                ("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int), ("L", ctypes.c_int),
+                ("d_k", ctypes.c_int), ("d_v", ctypes.c_int), ("chunk", ctypes.c_int),
+                ("dtype", ctypes.c_int), ("flags", ctypes.c_uint), ("l2_eps", ctypes.c_float),
+                ("rms_eps", ctypes.c_float)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libvda.so once; raise if it is missing (no fallback path exists)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing: build it with "
+                               "`python -m frame_level_delta_b200.build` (no CPU fallback exists)")
+        L = ctypes.CDLL(_LIB_PATH)
+        vp, sz, i, st = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_int
+        cfgp = ctypes.POINTER(vda_config)
+        L.vda_create.argtypes = [cfgp, ctypes.POINTER(vp)]
+        L.vda_destroy.argtypes = [vp]
+        L.vda_workspace_size.argtypes = [cfgp, ctypes.POINTER(sz)]
+        L.vda_prepare.argtypes = [vp] + [vp] * 9 + [vp, sz, vp]
+        L.vda_scan_bidir.argtypes = [vp, vp]
+        L.vda_readout.argtypes = [vp, vp, vp, vp]
+        L.vda_poll_device_status.argtypes = [vp, vp]
+        L.vda_workspace_region.argtypes = [cfgp, i, ctypes.POINTER(sz), ctypes.POINTER(sz)]
+        L.vda_status_string.argtypes = [st]
+        L.vda_status_string.restype = ctypes.c_char_p
+        L.vda_last_error.argtypes = [vp]
+        L.vda_last_error.restype = ctypes.c_char_p
+        L.vda_profile_enable.argtypes = [vp, i]
+        L.vda_num_kernels.argtypes = []
+        L.vda_profile_read.argtypes = [vp, i, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(i),
+                                       ctypes.POINTER(ctypes.c_double)]
+        L.vda_launch_count.argtypes = [vp, ctypes.POINTER(ctypes.c_uint64)]
+        L.vda_describe.argtypes = [cfgp, ctypes.POINTER(ctypes.c_char_p)]
+        L.vda_selftest_bounded_wait.argtypes = [vp, ctypes.c_uint64, vp]
+        for name in EXPORTS:
+            if name not in ("vda_status_string", "vda_last_error"):
+                getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def make_config(cfg: VDAConfig, force_simt: bool = False, l2_eps: float = 1e-6,
+                rms_eps: float = 1e-6) -> vda_config:
+    flags = (VDA_PREP_CONV if cfg.prep_conv else 0) | (VDA_READOUT_NORM_GATE if cfg.norm_gate else 0)
+    if force_simt:
+        flags |= VDA_FORCE_SIMT
+    return vda_config(B=cfg.B, H=cfg.H, T=cfg.T, U=cfg.U, grid_h=cfg.grid_h, grid_w=cfg.grid_w, L=cfg.L,
+                      d_k=cfg.d, d_v=cfg.d, chunk=cfg.chunk,
+                      dtype=VDA_F32 if cfg.dtype == "f32" else VDA_BF16, flags=flags,
+                      l2_eps=l2_eps, rms_eps=rms_eps)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def workspace_size(c: vda_config) -> int:
+    n = ctypes.c_size_t(0)
+    st = lib().vda_workspace_size(ctypes.byref(c), ctypes.byref(n))
+    if st != VDA_OK:
+        raise VDAError(st, "vda_workspace_size")
+    return n.value
+
+
+def workspace_region(c: vda_config, name: str):
+    off, nb = ctypes.c_size_t(0), ctypes.c_size_t(0)
+    st = lib().vda_workspace_region(ctypes.byref(c), REGIONS[name], ctypes.byref(off), ctypes.byref(nb))
+    if st != VDA_OK:
+        raise VDAError(st, "vda_workspace_region")
+    return off.value, nb.value
+
+
+def describe(c: vda_config) -> str:
+    t = ctypes.c_char_p()
+    st = lib().vda_describe(ctypes.byref(c), ctypes.byref(t))
+    if st != VDA_OK:
+        raise VDAError(st, "vda_describe")
+    return t.value.decode()
+
+
+class VDA:
+    """One context of the library: prepare -> scan_bidir -> readout on a stream."""
+
+    def __init__(self, cfg: VDAConfig, force_simt: bool = False, device="cuda"):
+        self.cfg = cfg
+        self.c = make_config(cfg, force_simt=force_simt)
+        self._ctx = ctypes.c_void_p()
+        st = lib().vda_create(ctypes.byref(self.c), ctypes.byref(self._ctx))
+        if st != VDA_OK:
+            raise VDAError(st, "vda_create")
+        self.ws_bytes = workspace_size(self.c)
+        self.device = torch.device(device)
+        self.workspace: Optional[torch.Tensor] = None
+        self._keep = None
+
+    def __del__(self):
+        if getattr(self, "_ctx", None) and self._ctx.value and _lib is not None:
+            _lib.vda_destroy(self._ctx)
+            self._ctx = ctypes.c_void_p()
+
+    def _check(self, st: int, what: str):
+        if st != VDA_OK:
+            raise VDAError(st, f"{what}: {lib().vda_last_error(self._ctx).decode()}")
+
+    def ensure_workspace(self) -> torch.Tensor:
+        if self.workspace is None:
+            self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
+        return self.workspace
+
+    def prepare(self, inp: Dict[str, torch.Tensor], stream=None):
+        ws = self.ensure_workspace()
+        self._keep = inp  # inputs must outlive the readout
+        st = lib().vda_prepare(self._ctx, _ptr(inp["Q"]), _ptr(inp["K"]), _ptr(inp["V"]), _ptr(inp["K_txt"]),
+                               _ptr(inp["V_txt"]), _ptr(inp["alpha"]), _ptr(inp["beta"]), _ptr(inp["beta_txt"]),
+                               _ptr(inp.get("conv_w")), _ptr(ws), ws.numel(), _stream_handle(stream))
+        self._check(st, "vda_prepare")
+
+    def scan_bidir(self, stream=None):
+        self._check(lib().vda_scan_bidir(self._ctx, _stream_handle(stream)), "vda_scan_bidir")
+
+    def readout(self, O: torch.Tensor, gate: Optional[torch.Tensor] = None, stream=None):
+        self._check(lib().vda_readout(self._ctx, _ptr(gate), _ptr(O), _stream_handle(stream)), "vda_readout")
+
+    def new_output(self) -> torch.Tensor:
+        cfg = self.cfg
+        dt = torch.float32 if cfg.dtype == "f32" else torch.bfloat16
+        return torch.empty(cfg.B, cfg.T * cfg.U, cfg.H, cfg.d, dtype=dt, device=self.device)
+
+    def run(self, inp: Dict[str, torch.Tensor], O: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """One pass of the whole path: prepare, bidirectional scan, readout."""
+        if O is None:
+            O = self.new_output()
+        self.prepare(inp, stream)
+        self.scan_bidir(stream)
+        self.readout(O, inp.get("gate"), stream)
+        return O
+
+    def poll_device_status(self, stream=None) -> int:
+        return lib().vda_poll_device_status(self._ctx, _stream_handle(stream))
+
+    def region(self, name: str) -> torch.Tensor:
+        """A view of one workspace region (float32 unless it is a prepared token copy)."""
+        off, nb = workspace_region(self.c, name)
+        raw = self.ensure_workspace()[off:off + nb]
+        cfg = self.cfg
+        D, BH = cfg.d, cfg.B * cfg.H
+        if name in ("A", "B", "M", "C"):
+            return raw.view(torch.float32).view(cfg.B, cfg.H, cfg.T - 1, D, D)
+        if name in ("S_fwd", "S_rev"):
+            return raw.view(torch.float32).view(cfg.B, cfg.H, cfg.J, D, D)
+        if name == "status":
+            return raw.view(torch.int32)
+        dt = torch.float32 if cfg.dtype == "f32" else torch.bfloat16
+        if name in ("K_prep", "V_prep"):
+            return raw.view(dt).view(cfg.B, cfg.H, cfg.T, cfg.U, D)
+        return raw.view(dt).view(cfg.B, cfg.H, cfg.L, D)
+
+    # -- profiling ---------------------------------------------------------------
+    def profile_enable(self, on: bool = True):
+        self._check(lib().vda_profile_enable(self._ctx, int(on)), "vda_profile_enable")
+
+    def profile_read(self) -> Dict[str, tuple]:
+        out = {}
+        for k in range(lib().vda_num_kernels()):
+            name, n, ms = ctypes.c_char_p(), ctypes.c_int(0), ctypes.c_double(0)
+            self._check(lib().vda_profile_read(self._ctx, k, ctypes.byref(name), ctypes.byref(n),
+                                               ctypes.byref(ms)), "vda_profile_read")
+            if n.value:
+                out[name.value.decode()] = (n.value, ms.value)
+        return out
+
+    def launch_count(self) -> int:
+        n = ctypes.c_uint64(0)
+        self._check(lib().vda_launch_count(self._ctx, ctypes.byref(n)), "vda_launch_count")
+        return n.value
+
+
+def selftest_bounded_wait(status: torch.Tensor, spins: int, stream=None) -> int:
+    return lib().vda_selftest_bounded_wait(_ptr(status), spins, _stream_handle(stream))
+
+
+def to_device(inp: Dict[str, torch.Tensor], device="cuda") -> Dict[str, torch.Tensor]:
+    return {k: v.to(device, non_blocking=True) for k, v in inp.items()}

@@ -1,0 +1,208 @@
+/*
+ * vda.h -- C ABI of libvda.so: Video Delta Attention (VDA), the linear branch
+ * of Video DeltaNet, as a bidirectional frame-level delta scan with a windowed
+ * readout, for NVIDIA B200 (sm_100a).
+ *
+ * Method (Video DeltaNet summary, onedev.kr/papers/80):
+ *  - section "how to use": per frame t, with keys K_t [U x d_k], values V_t
+ *    [U x d_v], write strengths beta_t [U] and decay alpha_t [d_k],
+ *      A_t = K_t^T Diag(beta_t) K_t,   B_t = V_t^T Diag(beta_t) K_t,
+ *      S_t = (S_{t-1} Diag(alpha_t) + B_t)(I + A_t)^-1
+ *    i.e. the minimiser of 1/2|S - Sbar|_F^2 + 1/2 sum_u beta_u |S k_u - v_u|^2,
+ *    with M_t = Diag(alpha_t)(I + A_t)^-1 (non-expansive) and the injection
+ *    C_t = B_t (I + A_t)^-1, so S_t = S_{t-1} M_t + C_t;
+ *  - section "how it works": a forward state summarises the frames before a
+ *    query chunk's softmax window (chunks j-1..j+1), a reverse state the frames
+ *    after it; both start at S_T/2 where S_T summarises the text tokens; the
+ *    query reads o = S-> q + S<- q;
+ *  - section "assumptions and limits": the boundary anchors (frames 0 and T-1)
+ *    are excluded from the linear state;
+ *  - section "how it differs": separable short conv (depthwise 5x5 spatial and
+ *    5-tap temporal) then SiLU on K and V, L2 norm on Q and K; RMS norm and a
+ *    sigmoid output gate on the linear readout.
+ *
+ * Readings fixed by this library where the pages are silent: S is d_v x d_k and
+ * o = S q; S_T = B_txt (I + A_txt)^-1 (the frame solve from S = 0 over the text
+ * tokens); the reverse scan uses the same M_t, C_t; chunk j = floor(t / c); the
+ * forward readout state of chunk j is the state after frame c(j-1)-1 (S_T/2 when
+ * that is < 1) and the reverse one the state after frame c(j+2) (S_T/2 when that
+ * is > T-2); anchor frames read out exactly zero.
+ *
+ * Conventions shared by every call:
+ *  - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *    never allocates or frees device memory; its only device memory is the
+ *    caller's workspace.
+ *  - Every call only enqueues work on the caller's CUDA stream (passed as
+ *    void*, a cudaStream_t; NULL is the legacy default stream) and never
+ *    synchronises, except vda_poll_device_status.
+ *  - Every call returns a vda_status and never aborts or prints. Argument errors
+ *    are detected before any launch and leave device memory untouched.
+ *  - Input pointers given to vda_prepare must stay valid until the matching
+ *    vda_readout has completed on the stream.
+ *  - A context is not thread-safe; use one per host thread.
+ */
+#ifndef VDA_H_
+#define VDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum vda_status {
+  VDA_OK = 0,
+  VDA_ERR_INVALID_ARG = 1,          /* null pointer, bad shape, inconsistent sizes */
+  VDA_ERR_UNSUPPORTED = 2,          /* valid but not implemented (e.g. d not in {16,32,64,128}) */
+  VDA_ERR_ALIGNMENT = 3,            /* a pointer is not 16-byte aligned (256 for the workspace) */
+  VDA_ERR_WORKSPACE_TOO_SMALL = 4,  /* workspace_bytes < vda_workspace_size() */
+  VDA_ERR_CUDA = 5,                 /* a CUDA runtime/driver call or a launch failed */
+  VDA_ERR_TIMEOUT = 6,              /* a bounded device-side wait gave up (see vda_poll_device_status) */
+  VDA_ERR_STATE = 7                 /* calls out of order (scan before prepare, ...) */
+} vda_status;
+
+typedef enum vda_dtype {
+  VDA_F32 = 0,  /* Q, K, V, K_txt, V_txt, gate and O stored as float32 */
+  VDA_BF16 = 1  /* ... stored as bfloat16; state, statistics and solves are always float32 */
+} vda_dtype;
+
+/* vda_config.flags */
+#define VDA_PREP_CONV 0x1u         /* video K, V: depthwise 5x5 spatial + centred 5-tap temporal
+                                      cross-correlation (zero padding, no bias) then SiLU; text K, V:
+                                      SiLU; then K, K_txt and Q divided by sqrt(|x|^2 + l2_eps) */
+#define VDA_READOUT_NORM_GATE 0x2u /* o <- o / sqrt(mean(o^2) + rms_eps) * sigmoid(gate) */
+#define VDA_FORCE_SIMT 0x100u      /* run the generic CUDA-core kernels even where a tensor-core
+                                      kernel exists (diagnostics and cross-checks) */
+
+typedef struct vda_config {
+  int B;        /* batch */
+  int H;        /* heads */
+  int T;        /* latent frames, >= 3 */
+  int U;        /* tokens per frame, == grid_h * grid_w */
+  int grid_h;   /* latent grid rows (row-major token order u = y * grid_w + x) */
+  int grid_w;   /* latent grid columns */
+  int L;        /* text tokens, >= 1 */
+  int d_k;      /* key channels; must equal d_v; one of 16, 32, 64, 128 */
+  int d_v;      /* value channels */
+  int chunk;    /* c: latent frames per chunk; chunk j holds frames c*j .. c*j+c-1 */
+  int dtype;    /* vda_dtype of the token tensors */
+  unsigned flags;
+  float l2_eps;  /* default 1e-6 */
+  float rms_eps; /* default 1e-6 */
+} vda_config;
+
+typedef struct vda_ctx vda_ctx; /* opaque host object; owns no device memory */
+
+/* Validate cfg and create a context. Host-only; touches no GPU. */
+vda_status vda_create(const vda_config* cfg, vda_ctx** out);
+vda_status vda_destroy(vda_ctx* ctx);
+
+/* Bytes of device workspace the caller must provide to vda_prepare. Host-only. */
+vda_status vda_workspace_size(const vda_config* cfg, size_t* bytes);
+
+/*
+ * Stage 1: feature prep (VDA_PREP_CONV only), frame statistics A_t, B_t for the
+ * text slot and frames 1..T-2, and the frame solve (Cholesky of I + A_t) giving
+ * M_t, C_t and S_T. Layouts (row-major, innermost last):
+ *   Q, K, V       [B, T*U, H, d]   token-major with heads interleaved; token
+ *                                  index t*U + u for frame t, grid position u
+ *   K_txt, V_txt  [B, L, H, d]
+ *   alpha         [B, H, T, d_k]   float32 in [0, 1] (entries of anchor frames unused)
+ *   beta          [B, H, T, U]     float32 >= 0
+ *   beta_txt      [B, H, L]        float32 >= 0
+ *   conv_w        float32, 60*H*d values: K-spatial [H*d,5,5], K-temporal [H*d,5],
+ *                 V-spatial [H*d,5,5], V-temporal [H*d,5] concatenated (channel
+ *                 h*d + k filters channel k of head h); required with
+ *                 VDA_PREP_CONV, ignored (may be NULL) otherwise.
+ *   workspace     >= vda_workspace_size(cfg) bytes, 256-byte aligned.
+ * All token tensors use the storage type cfg.dtype; all pointers 16-byte aligned.
+ */
+vda_status vda_prepare(vda_ctx* ctx, const void* Q, const void* K, const void* V,
+                       const void* K_txt, const void* V_txt, const float* alpha,
+                       const float* beta, const float* beta_txt, const float* conv_w,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Stage 2: the bidirectional scan. Forward F(0) = S_T/2, F(t) = F(t-1) M_t + C_t
+ * for t = 1 ..; reverse R(T-1) = S_T/2, R(t) = R(t+1) M_t + C_t for t = T-2 ..
+ * down. Writes, for every chunk j, its forward and reverse readout states into
+ * the workspace. VDA_ERR_STATE unless vda_prepare succeeded on this context.
+ */
+vda_status vda_scan_bidir(vda_ctx* ctx, void* stream);
+
+/*
+ * Stage 3: the readout. For every token of non-anchor frame t in chunk j:
+ * o = (S->_j + S<-_j) q (q divided by sqrt(|q|^2 + l2_eps) under
+ * VDA_PREP_CONV), then RMSNorm and the sigmoid gate under VDA_READOUT_NORM_GATE.
+ * Tokens of anchor frames 0 and T-1 are written as zeros.
+ *   gate  [B, T*U, H, d_v] storage dtype; required with VDA_READOUT_NORM_GATE.
+ *   O     [B, T*U, H, d_v] storage dtype; fully overwritten.
+ * VDA_ERR_STATE unless vda_scan_bidir succeeded after the last vda_prepare.
+ */
+vda_status vda_readout(vda_ctx* ctx, const void* gate, void* O, void* stream);
+
+/*
+ * Synchronise `stream`, read the device status word in the workspace, clear it
+ * and return VDA_ERR_TIMEOUT if a bounded device-side wait gave up since the last
+ * poll, VDA_OK otherwise (VDA_ERR_STATE before any vda_prepare).
+ */
+vda_status vda_poll_device_status(vda_ctx* ctx, void* stream);
+
+/* Regions of the workspace, for staged parity checks and debugging. */
+typedef enum vda_region {
+  VDA_REGION_STATUS = 0, /* uint32 device status word (+ padding) */
+  VDA_REGION_A = 1,      /* float32 [B, H, T-1, d_k, d_k]; slot 0 = text, slot t = frame t */
+  VDA_REGION_B = 2,      /* float32 [B, H, T-1, d_v, d_k]; same slots */
+  VDA_REGION_M = 3,      /* float32 [B, H, T-1, d_k, d_k]; slot t = M_t (slot 0 unused) */
+  VDA_REGION_C = 4,      /* float32 [B, H, T-1, d_v, d_k]; slot 0 = S_T, slot t = C_t */
+  VDA_REGION_S_FWD = 5,  /* float32 [B, H, J, d_v, d_k]; forward readout state of chunk j */
+  VDA_REGION_S_REV = 6,  /* float32 [B, H, J, d_v, d_k]; reverse readout state of chunk j */
+  VDA_REGION_K_PREP = 7, /* storage dtype [B, H, T, U, d]; prepared K (VDA_PREP_CONV only) */
+  VDA_REGION_V_PREP = 8, /* storage dtype [B, H, T, U, d]; prepared V (VDA_PREP_CONV only) */
+  VDA_REGION_KT_PREP = 9,  /* storage dtype [B, H, L, d]; prepared K_txt (VDA_PREP_CONV only) */
+  VDA_REGION_VT_PREP = 10, /* storage dtype [B, H, L, d]; prepared V_txt (VDA_PREP_CONV only) */
+  VDA_NUM_REGIONS = 11
+} vda_region;
+
+/* Byte offset and size of a region inside the workspace (size 0 if unused). Host-only. */
+vda_status vda_workspace_region(const vda_config* cfg, int region, size_t* offset, size_t* bytes);
+
+/* Static text for a status code. */
+const char* vda_status_string(vda_status s);
+
+/* Text of the last error recorded on this context ("" if none). */
+const char* vda_last_error(const vda_ctx* ctx);
+
+/*
+ * Per-kernel timing with CUDA events recorded on the launching stream around
+ * every kernel this context launches. Enabling resets the accumulators.
+ * vda_profile_read synchronises the recorded events, returns the number of
+ * launches and their summed duration (ms) for kernel id `kernel`, and the
+ * kernel's name through *name (static storage). Ids run 0 .. vda_num_kernels()-1.
+ */
+vda_status vda_profile_enable(vda_ctx* ctx, int enable);
+int vda_num_kernels(void);
+vda_status vda_profile_read(vda_ctx* ctx, int kernel, const char** name, int* launches,
+                            double* total_ms);
+
+/* Number of kernels this context has launched since it was created. */
+vda_status vda_launch_count(const vda_ctx* ctx, uint64_t* launches);
+
+/* Which implementation each stage uses for cfg: writes a static string such as
+ * "gram=tcgen05 solve=simt scan=simt readout=tcgen05". Host-only. */
+vda_status vda_describe(const vda_config* cfg, const char** text);
+
+/*
+ * Failure-detection self test: launch one kernel that waits, with an iteration
+ * limit `spins`, on a device flag that nothing sets, then writes
+ * VDA_ERR_TIMEOUT into the uint32 at `status_dev` (device pointer) and returns.
+ * Lets a test check that a bounded wait gives up and reports without faulting.
+ */
+vda_status vda_selftest_bounded_wait(uint32_t* status_dev, uint64_t spins, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VDA_H_ */

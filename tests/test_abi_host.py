@@ -1,0 +1,132 @@
+"""Host-side checks of the C ABI: the library loads and exports every symbol the
+header declares, and argument errors come back as status codes before any launch.
+No test here needs a GPU; no test passes pointers that could reach a kernel."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from frame_level_delta_b200 import vda as V
+from frame_level_delta_b200.inputs import CONFIGS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    with open(os.path.join(ROOT, "include", "vda.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:[\w\s\*]+?)\b(vda_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_matches_binding_list():
+    assert _declared_symbols() == sorted(V.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    L = V.lib()
+    for name in _declared_symbols():
+        assert hasattr(L, name), name
+
+
+def _cfg(**kw):
+    c = V.make_config(CONFIGS["small"])
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+def _create(c):
+    ctx = ctypes.c_void_p()
+    st = V.lib().vda_create(ctypes.byref(c), ctypes.byref(ctx))
+    return st, ctx
+
+
+@pytest.mark.parametrize("field,value,want", [
+    ("T", 2, 1), ("U", 255, 1), ("L", 0, 1), ("chunk", 0, 1), ("B", 0, 1), ("dtype", 7, 1),
+    ("d_k", 48, 2), ("d_v", 32, 2), ("flags", 0x80, 1),
+])
+def test_create_rejects_bad_configs(field, value, want):
+    c = _cfg(**{field: value})
+    if field == "d_k":
+        c.d_v = value
+    st, ctx = _create(c)
+    assert st == want and not ctx.value
+    n = ctypes.c_size_t(0)
+    assert V.lib().vda_workspace_size(ctypes.byref(c), ctypes.byref(n)) == want
+
+
+def test_workspace_regions_are_disjoint_and_aligned():
+    for name in ("tiny", "small", "h3", "long", "hires"):
+        c = V.make_config(CONFIGS[name])
+        total = V.workspace_size(c)
+        spans = []
+        for r in V.REGIONS:
+            off, nb = V.workspace_region(c, r)
+            assert off % 1024 == 0
+            assert off + nb <= total
+            if nb:
+                spans.append((off, off + nb))
+        spans.sort()
+        for (a0, a1), (b0, b1) in zip(spans, spans[1:]):
+            assert a1 <= b0
+        cfg = CONFIGS[name]
+        D = cfg.d
+        assert V.workspace_region(c, "A")[1] == cfg.B * cfg.H * (cfg.T - 1) * D * D * 4
+        assert V.workspace_region(c, "S_fwd")[1] == cfg.B * cfg.H * cfg.J * D * D * 4
+        assert (V.workspace_region(c, "K_prep")[1] > 0) == cfg.prep_conv
+
+
+def test_calls_out_of_order_and_bad_pointers_are_rejected_before_launch():
+    c = _cfg()
+    st, ctx = _create(c)
+    assert st == 0
+    L = V.lib()
+    try:
+        assert L.vda_scan_bidir(ctx, None) == 7
+        assert L.vda_readout(ctx, None, ctypes.c_void_p(0x10000), None) == 7
+        assert L.vda_poll_device_status(ctx, None) == 7
+        good = [ctypes.c_void_p(0x100000 * (i + 1)) for i in range(9)]
+        ws = ctypes.c_void_p(0x7000000)
+        big = V.workspace_size(c)
+        # NULL input
+        args = list(good)
+        args[2] = None
+        assert L.vda_prepare(ctx, *args, ws, big, None) == 1
+        # misaligned token tensor
+        args = list(good)
+        args[1] = ctypes.c_void_p(0x100008)
+        assert L.vda_prepare(ctx, *args, ws, big, None) == 3
+        # misaligned workspace
+        assert L.vda_prepare(ctx, *good, ctypes.c_void_p(0x7000080), big, None) == 3
+        # workspace too small
+        assert L.vda_prepare(ctx, *good, ws, big - 1, None) == 4
+        assert b"workspace" in L.vda_last_error(ctx)
+        # still not prepared
+        assert L.vda_scan_bidir(ctx, None) == 7
+    finally:
+        assert L.vda_destroy(ctx) == 0
+
+
+def test_conv_and_gate_requirements():
+    c = V.make_config(CONFIGS["hires"])
+    st, ctx = _create(c)
+    assert st == 0
+    L = V.lib()
+    try:
+        good = [ctypes.c_void_p(0x100000 * (i + 1)) for i in range(8)]
+        # conv_w is required with the conv flag
+        assert L.vda_prepare(ctx, *good, None, ctypes.c_void_p(0x7000000), V.workspace_size(c), None) == 1
+    finally:
+        L.vda_destroy(ctx)
+
+
+def test_status_strings_and_describe():
+    L = V.lib()
+    for code, name in V.STATUS_NAMES.items():
+        assert L.vda_status_string(code).decode() == name
+    assert L.vda_num_kernels() >= 8
+    text = V.describe(V.make_config(CONFIGS["tiny"]))
+    assert "gram=" in text and "readout=" in text
+    assert "tcgen05" not in text  # fp32 storage always takes the CUDA-core path
+    assert "tcgen05" not in V.describe(V.make_config(CONFIGS["h3"], force_simt=True))
