@@ -1,9 +1,321 @@
-// Frame statistics on tcgen05 tensor cores (bf16 operands, fp32 accumulation in TMEM).
+// Frame statistics on tcgen05 tensor cores: for every (b, h, slot)
+//   A = K^T Diag(beta) K   (d_k x d_k),   B = V^T Diag(beta) K   (d_v x d_k),
+// slot 0 over the text tokens, slot t over the U tokens of frame t (Video
+// DeltaNet summary, onedev.kr/papers/80, section "how to use": the key
+// correlation and value-key write statistics of a frame).
+//
+// Both products contract over tokens, the slow axis of a [tokens x d] tile, so
+// both tcgen05 operands are MN-major: TMA brings K and V token tiles (64 tokens
+// x 64 channels per box, 128-byte swizzle, zero fill past the frame's last token)
+// into shared memory, four warps form beta*K in place of a third buffer (bf16,
+// round to nearest), and one thread issues tcgen05.mma with fp32 accumulation
+// in TMEM. Warp roles: 0 = TMA producer, 1 = TMEM owner + MMA issuer,
+// 2..5 = beta scaling, then the TMEM -> global epilogue.
+//
+// d = 128: two M=128 N=128 MMAs per 16-token step (K-part -> TMEM columns
+// 0..127, V-part -> 128..255). d = 64: one M=128 N=64 MMA whose A operand is
+// [K | V] stacked along M (rows 0..63 give A, rows 64..127 give B).
+#include <cuda_bf16.h>
+
 #include "internal.h"
+#include "sm100.cuh"
+#include "tmap.h"
 
 namespace vda {
 
-bool gram_tc_supported(const Problem& p) { return false; }
-cudaError_t launch_gram_tc(const Problem& p, cudaStream_t s) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr int kTileU = 64;                    // tokens per pipeline stage
+constexpr int kBoxBytes = kTileU * 128;       // one box: 64 tokens x 64 bf16
+constexpr int kThreads = 192;
+
+template <int D>
+struct GramCfg {
+  static constexpr int kBoxes = D / 64;                     // boxes per operand tile
+  static constexpr int kStageBytes = 3 * kBoxes * kBoxBytes;  // K, V, beta*K
+  static constexpr int kStages = D == 128 ? 4 : 8;
+  static constexpr int kTmemCols = D == 128 ? 256 : 64;
+  static constexpr uint32_t kIdesc =
+      D == 128 ? sm100::idesc_bf16_f32(128, 128, true, true) : sm100::idesc_bf16_f32(128, 64, true, true);
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+struct GramArgs {
+  int B, H, T, U, L;
+  int layout;  // 0: token-major [B, tokens, H, d]; 1: frame-major [B, H, frames, tokens, d]
+  const float* beta;
+  const float* beta_txt;
+  float* A;
+  float* Bm;
+  uint32_t* status;
+  unsigned long long wait_ns;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    gram_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
+                   const __grid_constant__ CUtensorMap mKt, const __grid_constant__ CUtensorMap mVt,
+                   const GramArgs a) {
+  using C = GramCfg<D>;
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* bkf = full + C::kStages;
+  uint64_t* empty = bkf + C::kStages;
+  uint64_t* accb = empty + C::kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accb + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* issued_slot = reinterpret_cast<int*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int slot = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const bool text = slot == 0;
+  const int n = text ? a.L : a.U;
+  const int ntiles = (n + kTileU - 1) / kTileU;
+  const CUtensorMap* mk = text ? &mKt : &mK;
+  const CUtensorMap* mv = text ? &mVt : &mV;
+  const int tc = text ? 0 : slot;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&bkf[s], 4);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accb, 1);
+    *abort_flag = 0;
+    *issued_slot = 0;
+    fence_mbar_init();
+    prefetch_tmap(mk);
+    prefetch_tmap(mv);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer
+    if (lane == 0) {
+      int it = 0;
+      for (; it < ntiles; ++it) {
+        const int s = it % C::kStages;
+        const uint32_t ph = (it / C::kStages) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, a.status, a.wait_ns)) break;
+        uint8_t* st = smem + s * C::kStageBytes;
+        mbar_arrive_expect_tx(&full[s], 2 * C::kBoxes * kBoxBytes);
+        const int u0 = it * kTileU;
+#pragma unroll
+        for (int box = 0; box < C::kBoxes; ++box) {
+          const int d0 = box * 64;
+          if (a.layout == 0) {
+            tma_load_5d(st + box * kBoxBytes, mk, &full[s], d0, h, u0, tc, b);
+            tma_load_5d(st + (C::kBoxes + box) * kBoxBytes, mv, &full[s], d0, h, u0, tc, b);
+          } else {
+            tma_load_5d(st + box * kBoxBytes, mk, &full[s], d0, u0, tc, h, b);
+            tma_load_5d(st + (C::kBoxes + box) * kBoxBytes, mv, &full[s], d0, u0, tc, h, b);
+          }
+        }
+      }
+      *issued_slot = it;
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      uint32_t acc = 0;
+      for (int it = 0; it < ntiles; ++it) {
+        const int s = it % C::kStages;
+        const uint32_t ph = (it / C::kStages) & 1;
+        if (!mbar_wait(&full[s], ph, abort_flag, a.status, a.wait_ns)) break;
+        if (!mbar_wait(&bkf[s], ph, abort_flag, a.status, a.wait_ns)) break;
+        tc_fence_after();
+        const uint32_t base = smem_u32(smem + s * C::kStageBytes);
+#pragma unroll
+        for (int k = 0; k < kTileU / 16; ++k) {
+          const uint32_t koff = k * 16 * 128;  // 16 token rows of 128 bytes
+          if constexpr (D == 128) {
+            const uint64_t dK = smem_desc_sw128(base + koff, kBoxBytes, 1024);
+            const uint64_t dV = smem_desc_sw128(base + 2 * kBoxBytes + koff, kBoxBytes, 1024);
+            const uint64_t dB = smem_desc_sw128(base + 4 * kBoxBytes + koff, kBoxBytes, 1024);
+            mma_f16(tmem, dK, dB, C::kIdesc, acc);
+            mma_f16(tmem + 128, dV, dB, C::kIdesc, acc);
+          } else {
+            const uint64_t dKV = smem_desc_sw128(base + koff, kBoxBytes, 1024);  // K box then V box
+            const uint64_t dB = smem_desc_sw128(base + 2 * kBoxBytes + koff, kBoxBytes, 1024);
+            mma_f16(tmem, dKV, dB, C::kIdesc, acc);
+          }
+          acc = 1;
+        }
+        mma_commit(&empty[s]);
+      }
+      mma_commit(accb);  // completes once every MMA issued above has finished
+    }
+  } else {
+    // ---------------- beta scaling (warps 2..5), then the epilogue
+    const int tid = threadIdx.x - 64;  // 0..127
+    const float* beta = text ? a.beta_txt + ((long long)b * a.H + h) * a.L
+                             : a.beta + (((long long)b * a.H + h) * a.T + slot) * (long long)a.U;
+    int row, box, c0, c1;
+    if constexpr (D == 128) {
+      box = tid / 64;
+      row = tid % 64;
+      c0 = 0;
+      c1 = 8;
+    } else {
+      box = 0;
+      row = tid / 2;
+      c0 = (tid % 2) * 4;
+      c1 = c0 + 4;
+    }
+    bool ok = true;
+    for (int it = 0; it < ntiles; ++it) {
+      const int s = it % C::kStages;
+      const uint32_t ph = (it / C::kStages) & 1;
+      if (!mbar_wait(&full[s], ph, abort_flag, a.status, a.wait_ns)) {
+        ok = false;
+        break;
+      }
+      uint8_t* st = smem + s * C::kStageBytes;
+      const int u = it * kTileU + row;
+      const float bb = u < n ? __ldg(beta + u) : 0.f;
+      const uint8_t* src = st + box * kBoxBytes + row * 128;
+      uint8_t* dst = st + (2 * C::kBoxes + box) * kBoxBytes + row * 128;
+      for (int c = c0; c < c1; ++c) {
+        const int pc = c ^ (row & 7);  // any chunk order works; this one avoids bank conflicts
+        uint4 v = *reinterpret_cast<const uint4*>(src + pc * 16);
+        __nv_bfloat162* e = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float2 f = __bfloat1622float2(e[q]);
+          e[q] = __floats2bfloat162_rn(f.x * bb, f.y * bb);
+        }
+        *reinterpret_cast<uint4*>(dst + pc * 16) = v;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bkf[s]);
+    }
+    if (ok && mbar_wait(accb, 0, abort_flag, a.status, a.wait_ns)) {
+      tc_fence_after();
+      const int q = warp % 4;  // this warp may read TMEM lanes 32q .. 32q+31
+      const int r = q * 32 + lane;
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16);
+      const long long off = (((long long)b * a.H + h) * (a.T - 1) + slot) * (long long)D * D;
+      if constexpr (D == 128) {
+#pragma unroll 1
+        for (int c = 0; c < 16; ++c) {
+          uint32_t v[16];
+          tmem_ld16(taddr + c * 16, v);
+          tmem_ld_wait();
+          float* dst = (c < 8 ? a.A : a.Bm) + off + (long long)r * D + (c % 8) * 16;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            reinterpret_cast<float4*>(dst)[j] =
+                make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                            __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+        }
+      } else {
+        float* rowp = (r < 64 ? a.A + off + (long long)r * 64 : a.Bm + off + (long long)(r - 64) * 64);
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[16];
+          tmem_ld16(taddr + c * 16, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            reinterpret_cast<float4*>(rowp + c * 16)[j] =
+                make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                            __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+        }
+      }
+    }
+  }
+
+  // ---------------- teardown: nothing may be in flight when TMEM and smem go away
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) {
+    // Wait (bounded) for the last TMA load issued into each stage.
+    const int issued = *issued_slot;
+    for (int s = 0; s < C::kStages; ++s) {
+      int last = -1;
+      for (int it = s; it < issued; it += C::kStages) last = it;
+      if (last >= 0) mbar_wait(&full[s], (last / C::kStages) & 1, nullptr, a.status, a.wait_ns);
+    }
+  }
+  if (warp == 1) {
+    if (lane == 0) mbar_wait(accb, 0, nullptr, a.status, a.wait_ns);  // all MMAs retired
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+cudaError_t encode_maps(const Problem& p, CUtensorMap* mK, CUtensorMap* mV, CUtensorMap* mKt, CUtensorMap* mVt,
+                        int* layout) {
+  const uint64_t D = p.D, H = p.H, T = p.T, U = p.U, L = p.L, B = p.B;
+  const bool prep = (p.flags & VDA_PREP_CONV) != 0;
+  *layout = prep ? 1 : 0;
+  cudaError_t e;
+  if (!prep) {
+    // [B, T*U, H, D]: dims (d, h, u, t, b)
+    uint64_t dv[5] = {D, H, U, T, B};
+    uint64_t sv[4] = {D * 2, H * D * 2, U * H * D * 2, T * U * H * D * 2};
+    uint32_t box[5] = {64, 1, (uint32_t)kTileU, 1, 1};
+    if ((e = make_tmap_bf16(mK, p.Kv.p, 5, dv, sv, box)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16(mV, p.Vv.p, 5, dv, sv, box)) != cudaSuccess) return e;
+    // [B, L, H, D]: dims (d, h, u, 1, b)
+    uint64_t dt[5] = {D, H, L, 1, B};
+    uint64_t st[4] = {D * 2, H * D * 2, L * H * D * 2, L * H * D * 2};
+    if ((e = make_tmap_bf16(mKt, p.Kt.p, 5, dt, st, box)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16(mVt, p.Vt.p, 5, dt, st, box)) != cudaSuccess) return e;
+  } else {
+    // [B, H, T, U, D]: dims (d, u, t, h, b)
+    uint64_t dv[5] = {D, U, T, H, B};
+    uint64_t sv[4] = {D * 2, U * D * 2, T * U * D * 2, H * T * U * D * 2};
+    uint32_t box[5] = {64, (uint32_t)kTileU, 1, 1, 1};
+    if ((e = make_tmap_bf16(mK, p.Kv.p, 5, dv, sv, box)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16(mV, p.Vv.p, 5, dv, sv, box)) != cudaSuccess) return e;
+    // [B, H, L, D]: dims (d, u, 1, h, b)
+    uint64_t dt[5] = {D, L, 1, H, B};
+    uint64_t st[4] = {D * 2, L * D * 2, L * D * 2, H * L * D * 2};
+    if ((e = make_tmap_bf16(mKt, p.Kt.p, 5, dt, st, box)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16(mVt, p.Vt.p, 5, dt, st, box)) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+template <int D>
+cudaError_t launch_d(const Problem& p, cudaStream_t s) {
+  using C = GramCfg<D>;
+  CUtensorMap mK, mV, mKt, mVt;
+  GramArgs a{p.B, p.H, p.T, p.U, p.L, 0, p.beta, p.beta_txt, p.A, p.Bm, p.status, p.spin_limit};
+  cudaError_t e = encode_maps(p, &mK, &mV, &mKt, &mVt, &a.layout);
+  if (e != cudaSuccess) return e;
+  static bool attr_set = false;
+  if (!attr_set) {
+    e = cudaFuncSetAttribute(gram_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  dim3 grid(p.T - 1, p.H, p.B);
+  gram_tc_kernel<D><<<grid, kThreads, C::kSmemBytes, s>>>(mK, mV, mKt, mVt, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool gram_tc_supported(const Problem& p) { return p.bf16 && (p.D == 64 || p.D == 128); }
+
+cudaError_t launch_gram_tc(const Problem& p, cudaStream_t s) {
+  if (p.D == 128) return launch_d<128>(p, s);
+  if (p.D == 64) return launch_d<64>(p, s);
+  return cudaErrorNotSupported;
+}
 
 }  // namespace vda

@@ -41,7 +41,7 @@ struct Problem {
   void* Vp;
   void* Ktp;    // [B,H,L,D]
   void* Vtp;
-  unsigned long long spin_limit;  // iteration bound of every device-side wait
+  unsigned long long spin_limit;  // wall-time bound (ns) of every device-side wait
 };
 
 // Slot s of the statistics / solve arrays: 0 = text, t = frame t (1..T-2).

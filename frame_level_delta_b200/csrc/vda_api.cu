@@ -287,7 +287,7 @@ vda_status vda_prepare(vda_ctx* ctx, const void* Q, const void* K, const void* V
   p.C = reinterpret_cast<float*>(ws + L.off[VDA_REGION_C]);
   p.Sf = reinterpret_cast<float*>(ws + L.off[VDA_REGION_S_FWD]);
   p.Sr = reinterpret_cast<float*>(ws + L.off[VDA_REGION_S_REV]);
-  p.spin_limit = 1ull << 26;
+  p.spin_limit = 2000000000ull;  // 2 s of wall time per device-side wait
   const long long D = p.D, H = p.H, T = p.T, U = p.U, Lt = p.L;
   if (prep) {
     p.Kp = ws + L.off[VDA_REGION_K_PREP];
