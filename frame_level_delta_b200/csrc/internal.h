@@ -41,6 +41,7 @@ struct Problem {
   void* Vp;
   void* Ktp;    // [B,H,L,D]
   void* Vtp;
+  void* Msplit;  // [B,H,T-1] x 2 bf16 d*d images of M_t (hi, lo) for the tensor-core scan
   unsigned long long spin_limit;  // wall-time bound (ns) of every device-side wait
 };
 
@@ -63,6 +64,8 @@ enum KernelId {
   K_READOUT_SIMT,
   K_READOUT_TC,
   K_ZERO_ANCHORS,
+  K_SOLVE_TC,
+  K_SCAN_TC,
   K_NUM_KERNELS
 };
 const char* kernel_name(int id);
@@ -82,6 +85,10 @@ cudaError_t launch_selftest_wait(uint32_t* status, unsigned long long spins, cud
 bool gram_tc_supported(const Problem& p);
 cudaError_t launch_gram_tc(const Problem& p, cudaStream_t s);
 bool readout_tc_supported(const Problem& p);
+bool solve_tc_supported(const Problem& p);
+cudaError_t launch_solve_tc(const Problem& p, cudaStream_t s);
+bool scan_tc_supported(const Problem& p);
+cudaError_t launch_scan_tc(const Problem& p, cudaStream_t s);
 cudaError_t launch_readout_tc(const Problem& p, const void* gate, void* O, cudaStream_t s);
 
 }  // namespace vda

@@ -1,0 +1,260 @@
+// Bidirectional scan on tcgen05 tensor cores (Video DeltaNet summary,
+// onedev.kr/papers/80, section "how it works": a forward and a reverse state,
+// both started at S_T/2; section "how to use": S_t = S_{t-1} M_t + C_t).
+//
+// One CTA per (b, h, direction) runs the recurrence frame by frame:
+//   S <- S M_t + C_t,  S = Sh + Sl, M_t = Mh + Ml (bf16 parts, ~2^-16 relative),
+//   S M_t ~= Sh Mh + Sh Ml + Sl Mh  (24 MMAs of 128x128x16, fp32 in TMEM).
+// The fp32 state is rebuilt every step from TMEM plus C_t in the epilogue
+// (one thread per row), which also writes the readout states of the chunks
+// that need this frame's state and re-splits S into the K-major operand image
+// for the next step. M_t's hi/lo images, written by the solve in the operand
+// layout, arrive by one bulk copy per frame, double-buffered; C_t rows are
+// prefetched into registers while the MMAs run.
+// Warp roles: 0 = bulk-copy producer, 1 = TMEM owner + MMA issuer, 2..5 = epilogue.
+#include <cuda_bf16.h>
+
+#include "internal.h"
+#include "sm100.cuh"
+
+namespace vda {
+
+namespace {
+
+constexpr int D = 128;
+constexpr int kThreads = 192;
+constexpr int kImg = D * D * 2;           // one bf16 operand image
+constexpr int kMBuf = 2 * kImg;           // hi + lo images of one M_t
+constexpr int kSOff = 2 * kMBuf;          // S image (hi + lo) after two M buffers
+constexpr int kBarOff = kSOff + 2 * kImg;
+constexpr int kSmemBytes = kBarOff + 128 + 1024;
+constexpr uint32_t kIdesc = sm100::idesc_bf16_f32(128, 128, false, true);  // A (S) K-major, B (M) MN-major
+
+struct ScanArgs {
+  int B, H, T, c, J;
+  const float* C;     // [B,H,T-1,D,D]; slot 0 = S_T
+  const uint8_t* Mi;  // [B,H,T-1] x (hi, lo) operand images
+  float* Sf;
+  float* Sr;
+  uint32_t* status;
+  unsigned long long wait_ns;
+};
+
+__device__ __forceinline__ uint32_t img_off(int row, int col) {
+  const int atom = col >> 6, cc = col & 63;
+  return (uint32_t)(atom * D * 128 + row * 128 + ((((cc >> 3) ^ (row & 7))) << 4) + (cc & 7) * 2);
+}
+
+__device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&hi);
+  __nv_bfloat162* l = reinterpret_cast<__nv_bfloat162*>(&lo);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * q], x[2 * q + 1]);
+    const float2 hf = __bfloat1622float2(hh);
+    h[q] = hh;
+    l[q] = __floats2bfloat162_rn(x[2 * q] - hf.x, x[2 * q + 1] - hf.y);
+  }
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          sm100::smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(sm100::smem_u32(bar))
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) {
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sM = smem;           // [2][hi, lo]
+  uint8_t* sS = smem + kSOff;   // [hi, lo]
+  uint64_t* mfull = reinterpret_cast<uint64_t*>(smem + kBarOff);
+  uint64_t* mempty = mfull + 2;
+  uint64_t* tfull = mempty + 2;
+  uint64_t* sready = tfull + 1;
+  uint64_t* drain = sready + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int bh = blockIdx.x, dir = blockIdx.y;
+  const int c = a.c, T = a.T, J = a.J;
+  const int f_first = dir == 0 ? 1 : T - 2;
+  const int f_last = dir == 0 ? c * (J - 2) - 1 : 2 * c;
+  const int nsteps = max(0, dir == 0 ? f_last - f_first + 1 : f_first - f_last + 1);
+  const long long slots = (long long)bh * (T - 1);
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&mfull[s], 1);
+      mbar_init(&mempty[s], 1);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(sready, 4);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  int issued = 0;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int st = 0; st < nsteps; ++st) {
+        const int s = st & 1;
+        if (!mbar_wait(&mempty[s], ((st >> 1) & 1) ^ 1, abort_flag, a.status, a.wait_ns)) break;
+        const int f = dir == 0 ? f_first + st : f_first - st;
+        mbar_arrive_expect_tx(&mfull[s], kMBuf);
+        const uint8_t* src = a.Mi + (slots + f) * (long long)kMBuf;
+        bulk_load(sM + s * kMBuf, src, kImg, &mfull[s]);
+        bulk_load(sM + s * kMBuf + kImg, src + kImg, kImg, &mfull[s]);
+        issued = st + 1;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      for (int st = 0; st < nsteps; ++st) {
+        const int s = st & 1;
+        if (!mbar_wait(sready, st & 1, abort_flag, a.status, a.wait_ns)) break;
+        if (!mbar_wait(&mfull[s], (st >> 1) & 1, abort_flag, a.status, a.wait_ns)) break;
+        tc_fence_after();
+        const uint32_t sh = smem_u32(sS), sl = sh + kImg;
+        const uint32_t mh = smem_u32(sM + s * kMBuf), ml = mh + kImg;
+        const uint32_t as[3] = {sh, sh, sl}, bs[3] = {mh, ml, mh};
+#pragma unroll
+        for (int t = 0; t < 3; ++t)
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t da = smem_desc_sw128(as[t] + (kk / 4) * (D * 128) + (kk % 4) * 32, 16, 1024);
+            const uint64_t db = smem_desc_sw128(bs[t] + kk * 2048, D * 128, 1024);
+            mma_f16(tmem, da, db, kIdesc, (t == 0 && kk == 0) ? 0u : 1u);
+          }
+        mma_commit(&mempty[s]);
+        mma_commit(tfull);
+      }
+      mma_commit(drain);
+    }
+  } else {
+    const int q = warp % 4;
+    const int i = q * 32 + lane;  // state row == TMEM lane
+    float* out = dir == 0 ? a.Sf : a.Sr;
+    auto store_row = [&](int j, const float* x, int col0, int n) {
+      float4* d4 = reinterpret_cast<float4*>(out + ((long long)bh * J + j) * D * D + (long long)i * D + col0);
+      for (int t = 0; t < n / 4; ++t) d4[t] = make_float4(x[4 * t], x[4 * t + 1], x[4 * t + 2], x[4 * t + 3]);
+    };
+    // Initial state S_T / 2: readout states of the chunks that see no frame of
+    // this direction, and the first operand image.
+    {
+      const float* st0 = a.C + slots * (long long)D * D + (long long)i * D;
+#pragma unroll 1
+      for (int c16 = 0; c16 < D / 16; ++c16) {
+        float x[16];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float4 v = reinterpret_cast<const float4*>(st0 + c16 * 16)[t];
+          x[4 * t] = 0.5f * v.x; x[4 * t + 1] = 0.5f * v.y; x[4 * t + 2] = 0.5f * v.z; x[4 * t + 3] = 0.5f * v.w;
+        }
+        for (int j = 0; j < J; ++j)
+          if (dir == 0 ? (c * (j - 1) - 1 <= 0) : (c * (j + 2) >= T - 1)) store_row(j, x, c16 * 16, 16);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint4 hi, lo;
+          split8(x + 8 * hh, hi, lo);
+          const uint32_t o = img_off(i, c16 * 16 + 8 * hh);
+          *reinterpret_cast<uint4*>(sS + o) = hi;
+          *reinterpret_cast<uint4*>(sS + kImg + o) = lo;
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sready);
+    }
+    for (int st = 0; st < nsteps; ++st) {
+      const int f = dir == 0 ? f_first + st : f_first - st;
+      // Prefetch C_f row i while the MMAs run.
+      float crow[D];
+      const float4* csrc = reinterpret_cast<const float4*>(a.C + (slots + f) * (long long)D * D + (long long)i * D);
+#pragma unroll
+      for (int t = 0; t < D / 4; ++t) {
+        const float4 v = csrc[t];
+        crow[4 * t] = v.x; crow[4 * t + 1] = v.y; crow[4 * t + 2] = v.z; crow[4 * t + 3] = v.w;
+      }
+      if (!mbar_wait(tfull, st & 1, abort_flag, a.status, a.wait_ns)) break;
+      tc_fence_after();
+      int jout = -1;
+      if (dir == 0) {
+        if ((f + 1) % c == 0 && (f + 1) / c + 1 < J) jout = (f + 1) / c + 1;
+      } else {
+        if (f % c == 0 && f / c - 2 >= 0) jout = f / c - 2;
+      }
+#pragma unroll
+      for (int c16 = 0; c16 < D / 16; ++c16) {
+        uint32_t v[16];
+        tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + c16 * 16, v);
+        tmem_ld_wait();
+        float x[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) x[t] = __uint_as_float(v[t]) + crow[c16 * 16 + t];
+        if (jout >= 0) store_row(jout, x, c16 * 16, 16);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint4 hi, lo;
+          split8(x + 8 * hh, hi, lo);
+          const uint32_t o = img_off(i, c16 * 16 + 8 * hh);
+          *reinterpret_cast<uint4*>(sS + o) = hi;
+          *reinterpret_cast<uint4*>(sS + kImg + o) = lo;
+        }
+      }
+      tc_fence_before();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sready);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag && threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      int last = -1;
+      for (int st = s; st < issued; st += 2) last = st;
+      if (last >= 0) mbar_wait(&mfull[s], (last >> 1) & 1, nullptr, a.status, a.wait_ns);
+    }
+  }
+  if (warp == 1) {
+    if (lane == 0) mbar_wait(drain, 0, nullptr, a.status, a.wait_ns);
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+}  // namespace
+
+bool scan_tc_supported(const Problem& p) { return solve_tc_supported(p); }
+
+cudaError_t launch_scan_tc(const Problem& p, cudaStream_t s) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  ScanArgs a{p.B, p.H, p.T, p.c, p.J, p.C, static_cast<const uint8_t*>(p.Msplit), p.Sf, p.Sr, p.status,
+             p.spin_limit};
+  dim3 grid(p.B * p.H, 2);
+  scan_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace vda

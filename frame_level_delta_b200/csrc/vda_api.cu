@@ -15,7 +15,7 @@ namespace vda {
 const char* kernel_name(int id) {
   static const char* names[K_NUM_KERNELS] = {
       "prep_video", "prep_text", "gram_simt", "gram_tc", "solve_simt",
-      "scan_simt", "readout_simt", "readout_tc", "zero_anchors"};
+      "scan_simt", "readout_simt", "readout_tc", "zero_anchors", "solve_tc", "scan_tc"};
   return (id >= 0 && id < K_NUM_KERNELS) ? names[id] : "?";
 }
 
@@ -104,6 +104,7 @@ Layout make_layout(const vda_config& c) {
   L.bytes[VDA_REGION_V_PREP] = prep ? BH * c.T * (size_t)c.U * d * esz : 0;
   L.bytes[VDA_REGION_KT_PREP] = prep ? BH * c.L * d * esz : 0;
   L.bytes[VDA_REGION_VT_PREP] = prep ? BH * c.L * d * esz : 0;
+  L.bytes[VDA_REGION_M_SPLIT] = BH * (c.T - 1) * 2 * d * d * 2;
   size_t o = 0;
   for (int r = 0; r < VDA_NUM_REGIONS; ++r) {
     L.off[r] = o;
@@ -245,10 +246,12 @@ vda_status vda_describe(const vda_config* cfg, const char** text) {
   p.flags = cfg->flags;
   const bool simt = use_simt_only(*cfg);
   const bool g = !simt && gram_tc_supported(p), r = !simt && readout_tc_supported(p);
-  static const char* table[2][2] = {
-      {"gram=simt solve=simt scan=simt readout=simt", "gram=simt solve=simt scan=simt readout=tcgen05"},
-      {"gram=tcgen05 solve=simt scan=simt readout=simt", "gram=tcgen05 solve=simt scan=simt readout=tcgen05"}};
-  *text = table[g][r];
+  const bool v = !simt && solve_tc_supported(p), n = !simt && scan_tc_supported(p);
+  static char table[2][2][2][2][80];
+  char* t = table[g][v][n][r];
+  std::snprintf(t, 80, "gram=%s solve=%s scan=%s readout=%s", g ? "tcgen05" : "simt", v ? "tcgen05" : "simt",
+                n ? "tcgen05" : "simt", r ? "tcgen05" : "simt");
+  *text = t;
   return VDA_OK;
 }
 
@@ -287,6 +290,7 @@ vda_status vda_prepare(vda_ctx* ctx, const void* Q, const void* K, const void* V
   p.C = reinterpret_cast<float*>(ws + L.off[VDA_REGION_C]);
   p.Sf = reinterpret_cast<float*>(ws + L.off[VDA_REGION_S_FWD]);
   p.Sr = reinterpret_cast<float*>(ws + L.off[VDA_REGION_S_REV]);
+  p.Msplit = ws + L.off[VDA_REGION_M_SPLIT];
   p.spin_limit = 2000000000ull;  // 2 s of wall time per device-side wait
   const long long D = p.D, H = p.H, T = p.T, U = p.U, Lt = p.L;
   if (prep) {
@@ -319,7 +323,10 @@ vda_status vda_prepare(vda_ctx* ctx, const void* Q, const void* K, const void* V
   else
     st = run_kernel(ctx, K_GRAM_SIMT, s, [&] { return launch_gram_simt(p, s); });
   if (st != VDA_OK) return st;
-  st = run_kernel(ctx, K_SOLVE_SIMT, s, [&] { return launch_solve_simt(p, s); });
+  if (!use_simt_only(c) && solve_tc_supported(p))
+    st = run_kernel(ctx, K_SOLVE_TC, s, [&] { return launch_solve_tc(p, s); });
+  else
+    st = run_kernel(ctx, K_SOLVE_SIMT, s, [&] { return launch_solve_simt(p, s); });
   if (st != VDA_OK) return st;
   ctx->prepared = true;
   return VDA_OK;
@@ -329,7 +336,11 @@ vda_status vda_scan_bidir(vda_ctx* ctx, void* stream) {
   if (!ctx) return VDA_ERR_INVALID_ARG;
   if (!ctx->prepared) return fail(ctx, VDA_ERR_STATE, "vda_scan_bidir before a successful vda_prepare");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  vda_status st = run_kernel(ctx, K_SCAN_SIMT, s, [&] { return launch_scan_simt(ctx->p, s); });
+  vda_status st;
+  if (!use_simt_only(ctx->cfg) && scan_tc_supported(ctx->p))
+    st = run_kernel(ctx, K_SCAN_TC, s, [&] { return launch_scan_tc(ctx->p, s); });
+  else
+    st = run_kernel(ctx, K_SCAN_SIMT, s, [&] { return launch_scan_simt(ctx->p, s); });
   if (st != VDA_OK) return st;
   ctx->scanned = true;
   return VDA_OK;

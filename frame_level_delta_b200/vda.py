@@ -24,7 +24,7 @@ VDA_PREP_CONV = 0x1
 VDA_READOUT_NORM_GATE = 0x2
 VDA_FORCE_SIMT = 0x100
 REGIONS = {"status": 0, "A": 1, "B": 2, "M": 3, "C": 4, "S_fwd": 5, "S_rev": 6,
-           "K_prep": 7, "V_prep": 8, "Kt_prep": 9, "Vt_prep": 10}
+           "K_prep": 7, "V_prep": 8, "Kt_prep": 9, "Vt_prep": 10, "M_split": 11}
 
 # Exported symbols, in the order include/vda.h declares them.
 EXPORTS = ["vda_create", "vda_destroy", "vda_workspace_size", "vda_prepare", "vda_scan_bidir",

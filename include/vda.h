@@ -162,7 +162,10 @@ typedef enum vda_region {
   VDA_REGION_V_PREP = 8, /* storage dtype [B, H, T, U, d]; prepared V (VDA_PREP_CONV only) */
   VDA_REGION_KT_PREP = 9,  /* storage dtype [B, H, L, d]; prepared K_txt (VDA_PREP_CONV only) */
   VDA_REGION_VT_PREP = 10, /* storage dtype [B, H, L, d]; prepared V_txt (VDA_PREP_CONV only) */
-  VDA_NUM_REGIONS = 11
+  VDA_REGION_M_SPLIT = 11, /* bf16 [B, H, T-1, 2, d*d]: M_t as hi + lo parts (M = hi + lo to ~2^-16),
+                              each in the swizzled shared-memory operand layout of the tensor-core
+                              scan (used when that scan runs, unused otherwise) */
+  VDA_NUM_REGIONS = 12
 } vda_region;
 
 /* Byte offset and size of a region inside the workspace (size 0 if unused). Host-only. */
