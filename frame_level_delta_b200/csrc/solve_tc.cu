@@ -2,19 +2,20 @@
 // S_t (I + A_t) = Sbar_t + B_t, transition M_t = Diag(alpha_t)(I + A_t)^-1, with
 // the inverse taken in the d_k x d_k key space; the injection is C_t = B_t (I + A_t)^-1).
 //
-// Per (b, h, slot), d = 128, one CTA of 256 threads:
-//   1. X = I + A in shared memory (fp32), blocked right-looking Cholesky X = L L^T
-//      (16-wide panels: one warp factors the diagonal block, one thread per row
-//      solves the panel, 4x4 register tiles apply the rank-16 trailing update);
-//   2. W = L^-1 in place (diagonal 16x16 blocks inverted by 8 warps in parallel,
-//      then block rows top to bottom), all fp32 on CUDA cores;
-//   3. P = W^T W on tcgen05 (W split into bf16 hi + lo; P = Wh'Wh + Wh'Wl + Wl'Wh,
-//      fp32 accumulation in TMEM; error ~2^-16 relative);
-//   4. M = Diag(alpha) P written as fp32 and as the bf16 hi/lo operand images the
-//      tensor-core scan loads as they are; P kept as bf16 hi/lo operand in smem;
-//   5. C = B P on tcgen05 with the same three-term split (B_t arrives by a bulk
-//      copy issued at kernel start, overlapping steps 1-4).
-// The text slot (slot 0) produces only C = S_T.
+// Per (b, h, slot), d = 128, one CTA of 256 threads, two CTAs per SM. Blocked
+// right-looking Cholesky X = I + A = L L^T and the inverse W = L^-1 run together
+// in one loop over 16-wide block columns kb, with X and the inverse's
+// accumulator R (starting at I) held in TMEM as fp32:
+//   1. read X's block column kb (one row per thread) and R's block row kb;
+//   2. one warp factors the 16x16 diagonal block L_kk and inverts it;
+//   3. the panel L[:, kb] = X[:, kb] L_kk^-T (independent 16-term dots per row)
+//      and W's block row kb = L_kk^-1 R[kb, :] are formed on CUDA cores and
+//      stored as bf16 hi/lo operand images;
+//   4. tcgen05 applies both rank-16 updates, X -= Lp Lp^T and R -= Lp W[kb, :],
+//      as three-term split products (error ~2^-16 relative) with fp32 accumulation.
+// Then P = W^T W (tcgen05, same split), M = Diag(alpha) P (fp32 and the bf16
+// hi/lo operand images the tensor-core scan loads as they are), and C = B P with
+// B_t split into hi/lo in TMEM as the A operand. The text slot produces only C = S_T.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -25,20 +26,22 @@ namespace vda {
 namespace {
 
 constexpr int D = 128;
-constexpr int LDX = D + 4;  // padded fp32 row stride: rows stay 16-byte aligned
 constexpr int NB = D / 16;
 constexpr int kThreads = 256;
-constexpr int kImgBytes = D * D * 2;  // one bf16 operand image (two 64-column atoms)
-constexpr int kR1 = 0;                                  // X (fp32), later the P image
-constexpr int kR2 = ((LDX * D * 4 + 1023) / 1024) * 1024;  // W image, later the B image
-constexpr int kR3 = kR2 + 2 * kImgBytes;                // B_t (fp32) landing buffer
-constexpr int kWd = kR3 + D * D * 4;                    // 8 diagonal inverses, 16x16 fp32
-constexpr int kTb = kWd + NB * 256 * 4;                 // block-row temporary 16 x D fp32
-constexpr int kBar = kTb + 16 * D * 4;
-constexpr int kSmemBytes = kBar + 64 + 1024;
-constexpr uint32_t kIdescP = sm100::idesc_bf16_f32(128, 128, true, true);   // A, B MN-major
-constexpr uint32_t kIdescC = sm100::idesc_bf16_f32(128, 128, false, true);  // A K-major, B MN-major
-static_assert(kR2 >= 2 * kImgBytes, "P image must fit in the X region");
+constexpr int kImg = D * D * 2;       // one bf16 operand image (two 64-column atoms of D rows)
+constexpr int kWOff = 0;              // W image (hi, lo), later the P image
+constexpr int kLOff = 2 * kImg;       // current panel as a K-major image (hi, lo): one atom each
+constexpr int kLPart = D * 128;       // 16 KB per part
+constexpr int kRvOff = kLOff + 2 * kLPart;  // 1 / L_kk[j][j] (16 fp32)
+constexpr int kLkOff = kRvOff + 1024;       // L_kk (16x16 fp32)
+constexpr int kTbOff = kLkOff + 1024;       // R's block row kb (16 x D fp32)
+constexpr int kBarOff = kTbOff + 16 * D * 4;
+constexpr int kSmemBytes = kBarOff + 64 + 1024;
+constexpr uint32_t kNegA = 1u << 13;
+constexpr uint32_t kIdKK = sm100::idesc_bf16_f32(128, 128, false, false);  // A, B K-major
+constexpr uint32_t kIdKM = sm100::idesc_bf16_f32(128, 128, false, true);   // A K-major, B MN-major
+constexpr uint32_t kIdMM = sm100::idesc_bf16_f32(128, 128, true, true);    // A, B MN-major
+constexpr uint32_t kAccX = 0, kAccR = 128, kTmemB = 128;  // TMEM columns
 
 struct SolveArgs {
   int B, H, T;
@@ -47,17 +50,17 @@ struct SolveArgs {
   const float* alpha;
   float* M;
   float* C;
-  __nv_bfloat16* Msplit;
+  uint8_t* Msplit;
   uint32_t* status;
   unsigned long long wait_ns;
 };
 
-// Byte offset of element (row, col) in a bf16 operand image: 128-byte rows of 64
-// elements, 16-byte chunks XOR-swizzled by (row % 8), 64-column atoms of `rows`
-// rows stored one after the other (the 128-byte-swizzle canonical layout).
-__device__ __forceinline__ uint32_t img_off(int row, int col, int rows) {
+// Byte offset of element (row, col) in a bf16 operand image with 128-byte rows of
+// 64 elements, 16-byte chunks XOR-swizzled by (row % 8) and 64-column atoms of D
+// rows one after the other (the 128-byte-swizzle canonical layout).
+__device__ __forceinline__ uint32_t img_off(int row, int col) {
   const int atom = col >> 6, cc = col & 63;
-  return (uint32_t)(atom * rows * 128 + row * 128 + ((((cc >> 3) ^ (row & 7))) << 4) + (cc & 7) * 2);
+  return (uint32_t)(atom * D * 128 + row * 128 + ((((cc >> 3) ^ (row & 7))) << 4) + (cc & 7) * 2);
 }
 
 __device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
@@ -72,252 +75,270 @@ __device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
   }
 }
 
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          sm100::smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(sm100::smem_u32(bar))
-      : "memory");
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Three-term split product D = Ah Bh + Ah Bl + Al Bh over K = 128.
-// a_mn: A operand MN-major (advance 16 rows per K step) or K-major (32 bytes).
-__device__ __forceinline__ void mma_split3(uint32_t dtm, uint32_t a_hi, uint32_t a_lo, bool a_mn, uint32_t b_hi,
-                                           uint32_t b_lo, uint32_t idesc) {
-  using namespace sm100;
-  const uint32_t as[3] = {a_hi, a_hi, a_lo}, bs[3] = {b_hi, b_lo, b_hi};
-#pragma unroll
-  for (int t = 0; t < 3; ++t) {
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint64_t da = a_mn ? smem_desc_sw128(as[t] + kk * 2048, D * 128, 1024)
-                               : smem_desc_sw128(as[t] + (kk / 4) * (D * 128) + (kk % 4) * 32, 16, 1024);
-      const uint64_t db = smem_desc_sw128(bs[t] + kk * 2048, D * 128, 1024);
-      mma_f16(dtm, da, db, idesc, (t == 0 && kk == 0) ? 0u : 1u);
-    }
-  }
+// Three-term split product: D (+/-)= Ah Bh + Ah Bl + Al Bh, K = 16 per call
+// (one MMA per term) or K = 128 (eight K steps per term, MN-major operands).
+__device__ __forceinline__ void mma3(uint32_t d, uint64_t ah, uint64_t al, uint64_t bh, uint64_t bl,
+                                     uint32_t idesc, uint32_t acc_first) {
+  sm100::mma_f16(d, ah, bh, idesc, acc_first);
+  sm100::mma_f16(d, ah, bl, idesc, 1u);
+  sm100::mma_f16(d, al, bh, idesc, 1u);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) solve_tc_kernel(const SolveArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* X = reinterpret_cast<float*>(smem + kR1);
-  uint8_t* img1 = smem + kR1;  // P image (after X is consumed)
-  uint8_t* img2 = smem + kR2;  // W image, then B image
-  float* Bf = reinterpret_cast<float*>(smem + kR3);
-  float* Wd = reinterpret_cast<float*>(smem + kWd);  // [NB][16][16]
-  float* Tb = reinterpret_cast<float*>(smem + kTb);  // [16][D]
-  uint64_t* bar_b = reinterpret_cast<uint64_t*>(smem + kBar);
-  uint64_t* bar_p = bar_b + 1;
-  uint64_t* bar_c = bar_b + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_b + 3);
+  uint8_t* wimg = smem + kWOff;
+  uint8_t* limg = smem + kLOff;
+  float* Rv = reinterpret_cast<float*>(smem + kRvOff);
+  float* Lk = reinterpret_cast<float*>(smem + kLkOff);
+  float* Tb = reinterpret_cast<float*>(smem + kTbOff);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kBarOff);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const int slot = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const long long off = (((long long)b * a.H + h) * (a.T - 1) + slot) * (long long)D * D;
+  const int q = warp % 4, hc = warp / 4;
+  const int ri = q * 32 + lane;  // TMEM lane / matrix row of this thread
+  uint32_t phase = 0;            // parity of the next completion of `bar`
+  int commits = 0;
 
   if (tid == 0) {
-    mbar_init(bar_b, 1);
-    mbar_init(bar_p, 1);
-    mbar_init(bar_c, 1);
+    mbar_init(bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    mbar_arrive_expect_tx(bar_b, D * D * 4);
-    bulk_load(Bf, a.Bm + off, D * D * 4, bar_b);
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, 256);
     tmem_relinquish();
   }
-  // X = I + A
-  {
-    const float4* src = reinterpret_cast<const float4*>(a.A + off);
-    for (int e = tid; e < D * D / 4; e += kThreads) {
-      const int i = e / (D / 4), c4 = e % (D / 4);
-      float4 v = src[e];
-      const int j = c4 * 4;
-      if (i == j) v.x += 1.f;
-      if (i == j + 1) v.y += 1.f;
-      if (i == j + 2) v.z += 1.f;
-      if (i == j + 3) v.w += 1.f;
-      *reinterpret_cast<float4*>(X + i * LDX + j) = v;
-    }
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
 
-  // ---------------- 1. blocked Cholesky, lower, in place
-  for (int kb = 0; kb < NB; ++kb) {
-    const int k0 = kb * 16;
-    if (warp == 0) {  // factor the 16x16 diagonal block in registers
-      const int r = lane & 15;
-      float x[16];
-#pragma unroll
-      for (int c = 0; c < 16; ++c) x[c] = X[(k0 + r) * LDX + k0 + c];
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float dj = __shfl_sync(0xffffffffu, x[j], j);
-        const float ljj = sqrtf(dj);
-        const float inv = 1.f / ljj;
-        if (r == j) x[j] = ljj;
-        else if (r > j) x[j] *= inv;
-#pragma unroll
-        for (int m = j + 1; m < 16; ++m) {
-          const float lmj = __shfl_sync(0xffffffffu, x[j], m);
-          if (r >= m) x[m] = fmaf(-x[j], lmj, x[m]);
-        }
-      }
-      if (lane < 16) {
-#pragma unroll
-        for (int c = 0; c < 16; ++c)
-          if (c <= r) X[(k0 + r) * LDX + k0 + c] = x[c];
-      }
-    }
-    __syncthreads();
-    const int n = D - k0 - 16;
-    if (n == 0) break;
-    if (tid < n) {  // panel: row i solves L_kk y = x (forward substitution)
-      const int i = k0 + 16 + tid;
-      float y[16];
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        const float4 v = *reinterpret_cast<const float4*>(X + i * LDX + k0 + 4 * c4);
-        y[4 * c4] = v.x; y[4 * c4 + 1] = v.y; y[4 * c4 + 2] = v.z; y[4 * c4 + 3] = v.w;
-      }
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        float acc = y[c];
-#pragma unroll
-        for (int m = 0; m < c; ++m) acc = fmaf(-y[m], X[(k0 + c) * LDX + k0 + m], acc);
-        y[c] = acc / X[(k0 + c) * LDX + k0 + c];
-      }
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4)
-        *reinterpret_cast<float4*>(X + i * LDX + k0 + 4 * c4) =
-            make_float4(y[4 * c4], y[4 * c4 + 1], y[4 * c4 + 2], y[4 * c4 + 3]);
-    }
-    __syncthreads();
-    {  // rank-16 trailing update of the lower triangle, 4x4 tiles
-      const int nt = n / 4;
-      const int ntiles = nt * (nt + 1) / 2;
-      for (int t = tid; t < ntiles; t += kThreads) {
-        int ti = (int)((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
-        while ((ti + 1) * (ti + 2) / 2 <= t) ++ti;
-        while (ti * (ti + 1) / 2 > t) --ti;
-        const int tj = t - ti * (ti + 1) / 2;
-        const int i0 = k0 + 16 + 4 * ti, j0 = k0 + 16 + 4 * tj;
-        float acc[4][4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const float4 v = *reinterpret_cast<const float4*>(X + (i0 + r) * LDX + j0);
-          acc[r][0] = v.x; acc[r][1] = v.y; acc[r][2] = v.z; acc[r][3] = v.w;
-        }
-#pragma unroll
-        for (int m4 = 0; m4 < 4; ++m4) {
-          float4 li[4], lj[4];
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            li[r] = *reinterpret_cast<const float4*>(X + (i0 + r) * LDX + k0 + 4 * m4);
-            lj[r] = *reinterpret_cast<const float4*>(X + (j0 + r) * LDX + k0 + 4 * m4);
-          }
-#pragma unroll
-          for (int r = 0; r < 4; ++r)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              float s = acc[r][c];
-              s = fmaf(-li[r].x, lj[c].x, s);
-              s = fmaf(-li[r].y, lj[c].y, s);
-              s = fmaf(-li[r].z, lj[c].z, s);
-              s = fmaf(-li[r].w, lj[c].w, s);
-              acc[r][c] = s;
-            }
-        }
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-          *reinterpret_cast<float4*>(X + (i0 + r) * LDX + j0) = make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
-      }
-    }
-    __syncthreads();
-  }
-
-  // ---------------- 2. W = L^-1 in place
-  if (warp < NB) {  // diagonal blocks: lane c computes column c of (L_ww)^-1
-    const int w0 = warp * 16, c = lane & 15;
-    float wv[16];
-#pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      float acc = (r == c) ? 1.f : 0.f;
-#pragma unroll
-      for (int m = 0; m < r; ++m) acc = fmaf(-X[(w0 + r) * LDX + w0 + m], wv[m], acc);
-      wv[r] = acc / X[(w0 + r) * LDX + w0 + r];
-    }
-    if (lane < 16) {
-#pragma unroll
-      for (int r = 0; r < 16; ++r) Wd[warp * 256 + r * 16 + c] = wv[r];
-    }
-  }
-  __syncthreads();
+  // X = I + A into TMEM columns 0..127 and R = I into 128..255 (this thread: row
+  // ri, columns hc*64 .. hc*64+63). All sixteen loads are issued before use.
   {
-    const int r = tid / 16, c = tid % 16;
-    X[r * LDX + c] = Wd[r * 16 + c];
-    for (int ib = 1; ib < NB; ++ib) {
-      __syncthreads();
-      const int row = ib * 16 + r;
-      for (int jb = 0; jb < ib; ++jb) {  // T_jb = L[ib, jb..ib-1] W[jb..ib-1, jb]
-        float acc = 0.f;
-        for (int k = jb * 16; k < ib * 16; ++k) acc = fmaf(X[row * LDX + k], X[k * LDX + jb * 16 + c], acc);
-        Tb[r * D + jb * 16 + c] = acc;
-      }
-      __syncthreads();
-      for (int jb = 0; jb < ib; ++jb) {  // W_ib,jb = -W_ib,ib T_jb
-        float acc = 0.f;
+    const float4* src = reinterpret_cast<const float4*>(a.A + off + (long long)ri * D + hc * 64);
+    float4 v[16];
 #pragma unroll
-        for (int m = 0; m < 16; ++m) acc = fmaf(Wd[ib * 256 + r * 16 + m], Tb[m * D + jb * 16 + c], acc);
-        X[row * LDX + jb * 16 + c] = -acc;
+    for (int t = 0; t < 16; ++t) v[t] = src[t];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t x[16], r[16];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int col = hc * 64 + c * 16 + 4 * t;
+        const float4 w = v[c * 4 + t];
+        x[4 * t] = __float_as_uint(w.x + (ri == col ? 1.f : 0.f));
+        x[4 * t + 1] = __float_as_uint(w.y + (ri == col + 1 ? 1.f : 0.f));
+        x[4 * t + 2] = __float_as_uint(w.z + (ri == col + 2 ? 1.f : 0.f));
+        x[4 * t + 3] = __float_as_uint(w.w + (ri == col + 3 ? 1.f : 0.f));
+#pragma unroll
+        for (int u = 0; u < 4; ++u) r[4 * t + u] = __float_as_uint(ri == col + u ? 1.f : 0.f);
       }
-      X[row * LDX + ib * 16 + c] = Wd[ib * 256 + r * 16 + c];
+      tmem_st16(tl + kAccX + hc * 64 + c * 16, x);
+      tmem_st16(tl + kAccR + hc * 64 + c * 16, r);
     }
+    tmem_st_wait();
   }
+  tc_fence_before();
   __syncthreads();
-
-  // ---------------- 3. W image (rows k, columns i; zero above the diagonal), P = W^T W
-  for (int e = tid; e < D * (D / 8); e += kThreads) {
-    const int k = e / (D / 8), i0 = (e % (D / 8)) * 8;
-    float x[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) x[q] = (i0 + q <= k) ? X[k * LDX + i0 + q] : 0.f;
-    uint4 hi, lo;
-    split8(x, hi, lo);
-    const uint32_t o = img_off(k, i0, D);
-    *reinterpret_cast<uint4*>(img2 + o) = hi;
-    *reinterpret_cast<uint4*>(img2 + kImgBytes + o) = lo;
-  }
-  fence_proxy_async_smem();
-  __syncthreads();
-  if (tid == 0) {
-    tc_fence_after();
-    const uint32_t wh = smem_u32(img2), wl = wh + kImgBytes;
-    mma_split3(tmem, wh, wl, true, wh, wl, kIdescP);
-    mma_commit(bar_p);
-  }
-  bool ok = mbar_wait(bar_p, 0, abort_flag, a.status, a.wait_ns);
   tc_fence_after();
 
-  // ---------------- 4. M = Diag(alpha) P (fp32 + hi/lo images), P image into smem
-  const int q = warp % 4, half = warp / 4;
-  const int i = q * 32 + lane;  // TMEM lane / matrix row of this thread
+  const uint32_t wbase = smem_u32(wimg), lbase = smem_u32(limg);
+  for (int kb = 0; kb < NB; ++kb) {
+    const int k0 = kb * 16;
+    const int pw = k0 / 32, l0 = k0 % 32;  // warp and first lane holding rows k0..k0+15
+    // ---- 1. block column kb of X (rows ri), block row kb of R (into Tb)
+    float x[16];
+    if (hc == 0) {
+      uint32_t v[16];
+      tmem_ld16(tl + kAccX + k0, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int t = 0; t < 16; ++t) x[t] = __uint_as_float(v[t]);
+    }
+    if (q == pw) {
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[16];
+        tmem_ld16(tl + kAccR + hc * 64 + c * 16, v);
+        tmem_ld_wait();
+        const int r = lane - l0;
+        if (r >= 0 && r < 16) {
+          float4* dst = reinterpret_cast<float4*>(Tb + r * D + hc * 64 + c * 16);
+#pragma unroll
+          for (int t = 0; t < 4; ++t)
+            dst[t] = make_float4(__uint_as_float(v[4 * t]), __uint_as_float(v[4 * t + 1]),
+                                 __uint_as_float(v[4 * t + 2]), __uint_as_float(v[4 * t + 3]));
+        }
+      }
+    }
+    // ---- 2. factor the diagonal block (warp pw, lanes l0..l0+15). Register arrays
+    // are only ever indexed by constants: the current column is always g[0] and
+    // the row shifts left after every pivot.
+    if (warp == pw) {
+      const int r = lane - l0;  // row within the block for lanes l0..l0+15
+      const bool in = r >= 0 && r < 16;
+      float g[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c) g[c] = x[c];
+      for (int j = 0; j < 16; ++j) {
+        const float dj = __shfl_sync(0xffffffffu, g[0], l0 + j);
+        const float inv = rsqrtf(dj);
+        const float lrj = (r == j) ? dj * inv : g[0] * inv;  // L[r][j] for r >= j
+        if (in && r >= j) Lk[r * 16 + j] = lrj;
+        if (in && r == j) Rv[j] = inv;                        // 1 / L[j][j]
+#pragma unroll
+        for (int t = 1; t < 16; ++t) {
+          const float lmj = __shfl_sync(0xffffffffu, lrj, (l0 + j + t) & 31);
+          g[t - 1] = (in && j + t < 16 && r >= j + t) ? fmaf(-lrj, lmj, g[t]) : g[t];
+        }
+      }
+      if (in) {
+        for (int c = r + 1; c < 16; ++c) Lk[r * 16 + c] = 0.f;
+      }
+    }
+    __syncthreads();
+    if (hc == 0) {
+      // ---- 3a. panel row ri: L[ri, kb] L_kk^T = X[ri, kb] by forward substitution,
+      // into the K-major panel image (K columns 0..15)
+      float pv[16];
+      if (ri >= k0 + 16) {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) pv[c] = 0.f;
+        for (int c = 0; c < 16; ++c) {
+          const float y = x[0] * Rv[c];
+#pragma unroll
+          for (int t = 0; t < 15; ++t) {
+            const float l = (c + 1 + t < 16) ? Lk[(c + 1 + t) * 16 + c] : 0.f;
+            x[t] = fmaf(-y, l, x[t + 1]);
+          }
+#pragma unroll
+          for (int t = 0; t < 15; ++t) pv[t] = pv[t + 1];
+          pv[15] = y;
+        }
+      } else if (ri >= k0) {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) pv[c] = Lk[(ri - k0) * 16 + c];
+      } else {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) pv[c] = 0.f;
+      }
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint4 hi, lo;
+        split8(pv + 8 * hh, hi, lo);
+        const uint32_t o = img_off(ri, 8 * hh);
+        *reinterpret_cast<uint4*>(limg + o) = hi;
+        *reinterpret_cast<uint4*>(limg + kLPart + o) = lo;
+      }
+    } else {
+      // ---- 3b. column j of W[kb, :]: L_kk W[kb, j] = R[kb, j] by forward substitution
+      const int j = ri;  // column 0..127
+      float z[16];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) z[r] = Tb[r * D + j];
+      __nv_bfloat16* wh = reinterpret_cast<__nv_bfloat16*>(wimg);
+      __nv_bfloat16* wl = reinterpret_cast<__nv_bfloat16*>(wimg + kImg);
+      for (int r = 0; r < 16; ++r) {
+        const float w = z[0] * Rv[r];
+#pragma unroll
+        for (int t = 0; t < 15; ++t) {
+          const float l = (r + 1 + t < 16) ? Lk[(r + 1 + t) * 16 + r] : 0.f;
+          z[t] = fmaf(-w, l, z[t + 1]);
+        }
+        const __nv_bfloat16 hb = __float2bfloat16_rn(w);
+        const uint32_t o = img_off(k0 + r, j) >> 1;
+        wh[o] = hb;
+        wl[o] = __float2bfloat16_rn(w - __bfloat162float(hb));
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    // ---- 4. rank-16 updates on tcgen05: X -= Lp Lp^T, R -= Lp W[kb, :]
+    if (kb + 1 < NB) {
+      if (tid == 0 && !*abort_flag) {
+        tc_fence_after();
+        const uint64_t lh = smem_desc_sw128(lbase, 16, 1024), ll = smem_desc_sw128(lbase + kLPart, 16, 1024);
+        const uint64_t wh = smem_desc_sw128(wbase + kb * 2048, D * 128, 1024);
+        const uint64_t wl = smem_desc_sw128(wbase + kImg + kb * 2048, D * 128, 1024);
+        mma3(tmem + kAccX, lh, ll, lh, ll, kIdKK | kNegA, 1u);
+        mma3(tmem + kAccR, lh, ll, wh, wl, kIdKM | kNegA, 1u);
+        mma_commit(bar);
+      }
+      ++commits;
+      mbar_wait(bar, phase, abort_flag, a.status, a.wait_ns);
+      phase ^= 1;
+      tc_fence_after();
+    }
+  }
+
+  // ---------------- P = W^T W into TMEM columns 0..127
+  if (tid == 0 && !*abort_flag) {
+    tc_fence_after();
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t dh = smem_desc_sw128(wbase + kk * 2048, D * 128, 1024);
+      const uint64_t dl = smem_desc_sw128(wbase + kImg + kk * 2048, D * 128, 1024);
+      mma3(tmem + kAccX, dh, dl, dh, dl, kIdMM, kk > 0 ? 1u : 0u);
+    }
+    mma_commit(bar);
+  }
+  ++commits;
+  // B_t (row ri, columns hc*64..) -> TMEM columns 128.. as hi | lo bf16 pairs, while P runs.
+  {
+    const float4* src = reinterpret_cast<const float4*>(a.Bm + off + (long long)ri * D + hc * 64);
+    float4 v[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) v[t] = src[t];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      uint32_t ph[16], pl[16];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const float4 w = v[c * 8 + t];
+        const float xs[4] = {w.x, w.y, w.z, w.w};
+        float hv[4], lv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          hv[u] = __bfloat162float(__float2bfloat16_rn(xs[u]));
+          lv[u] = xs[u] - hv[u];
+        }
+        ph[2 * t] = pack_bf16(hv[0], hv[1]);
+        ph[2 * t + 1] = pack_bf16(hv[2], hv[3]);
+        pl[2 * t] = pack_bf16(lv[0], lv[1]);
+        pl[2 * t + 1] = pack_bf16(lv[2], lv[3]);
+      }
+      tmem_st16(tl + kTmemB + hc * 32 + c * 16, ph);
+      tmem_st16(tl + kTmemB + 64 + hc * 32 + c * 16, pl);
+    }
+    tmem_st_wait();
+  }
+  bool ok = mbar_wait(bar, phase, abort_flag, a.status, a.wait_ns);
+  phase ^= 1;
+  tc_fence_after();
+
+  // ---------------- M = Diag(alpha) P (fp32 + hi/lo images); P image over the W image
   if (ok) {
-    const float al = slot > 0 ? a.alpha[(((long long)b * a.H + h) * a.T + slot) * D + i] : 0.f;
-    uint8_t* mimg = reinterpret_cast<uint8_t*>(a.Msplit) + off * 4;  // 2 images of D*D bf16 per slot
+    const float al = slot > 0 ? a.alpha[(((long long)b * a.H + h) * a.T + slot) * D + ri] : 0.f;
+    uint8_t* mimg = a.Msplit + off * 4;  // two D*D bf16 images per slot
 #pragma unroll 1
     for (int cc = 0; cc < 4; ++cc) {
-      const int j0 = half * 64 + cc * 16;
+      const int j0 = hc * 64 + cc * 16;
       uint32_t v[16];
-      tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + j0, v);
+      tmem_ld16(tl + kAccX + j0, v);
       tmem_ld_wait();
       float pv[16], mv[16];
 #pragma unroll
@@ -329,57 +350,51 @@ __global__ void __launch_bounds__(kThreads, 1) solve_tc_kernel(const SolveArgs a
       for (int hh = 0; hh < 2; ++hh) {
         uint4 hi, lo;
         split8(pv + 8 * hh, hi, lo);
-        const uint32_t o = img_off(i, j0 + 8 * hh, D);
-        *reinterpret_cast<uint4*>(img1 + o) = hi;
-        *reinterpret_cast<uint4*>(img1 + kImgBytes + o) = lo;
+        const uint32_t o = img_off(ri, j0 + 8 * hh);
+        *reinterpret_cast<uint4*>(wimg + o) = hi;
+        *reinterpret_cast<uint4*>(wimg + kImg + o) = lo;
         if (slot > 0) {
           split8(mv + 8 * hh, hi, lo);
           *reinterpret_cast<uint4*>(mimg + o) = hi;
-          *reinterpret_cast<uint4*>(mimg + kImgBytes + o) = lo;
+          *reinterpret_cast<uint4*>(mimg + kImg + o) = lo;
         }
       }
       if (slot > 0) {
-        float4* md = reinterpret_cast<float4*>(a.M + off + (long long)i * D + j0);
+        float4* md = reinterpret_cast<float4*>(a.M + off + (long long)ri * D + j0);
 #pragma unroll
         for (int t = 0; t < 4; ++t) md[t] = make_float4(mv[4 * t], mv[4 * t + 1], mv[4 * t + 2], mv[4 * t + 3]);
       }
     }
   }
-  // ---------------- 5. C = B P: B (K-major image) from the landed fp32 copy
-  if (ok) ok = mbar_wait(bar_b, 0, abort_flag, a.status, a.wait_ns);
-  if (ok) {
-    for (int e = tid; e < D * (D / 8); e += kThreads) {
-      const int r = e / (D / 8), k0 = (e % (D / 8)) * 8;
-      const float4 v0 = *reinterpret_cast<const float4*>(Bf + r * D + k0);
-      const float4 v1 = *reinterpret_cast<const float4*>(Bf + r * D + k0 + 4);
-      const float x[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-      uint4 hi, lo;
-      split8(x, hi, lo);
-      const uint32_t o = img_off(r, k0, D);
-      *reinterpret_cast<uint4*>(img2 + o) = hi;
-      *reinterpret_cast<uint4*>(img2 + kImgBytes + o) = lo;
-    }
-  }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
+  // ---------------- C = B P (A operand B_t from TMEM, B operand the P image)
   if (tid == 0 && !*abort_flag) {
     tc_fence_after();
-    const uint32_t bh = smem_u32(img2), bl = bh + kImgBytes;
-    const uint32_t ph = smem_u32(img1), pl = ph + kImgBytes;
-    mma_split3(tmem + 128, bh, bl, false, ph, pl, kIdescC);
-    mma_commit(bar_c);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t ph = smem_desc_sw128(wbase + kk * 2048, D * 128, 1024);
+      const uint64_t pl = smem_desc_sw128(wbase + kImg + kk * 2048, D * 128, 1024);
+      const uint32_t bh = tmem + kTmemB + kk * 8, bl = tmem + kTmemB + 64 + kk * 8;
+      mma_f16_ts(tmem + kAccX, bh, ph, kIdKM, kk > 0 ? 1u : 0u);
+      mma_f16_ts(tmem + kAccX, bh, pl, kIdKM, 1u);
+      mma_f16_ts(tmem + kAccX, bl, ph, kIdKM, 1u);
+    }
+    mma_commit(bar);
   }
-  if (ok) ok = mbar_wait(bar_c, 0, abort_flag, a.status, a.wait_ns);
+  ++commits;
+  if (ok) ok = mbar_wait(bar, phase, abort_flag, a.status, a.wait_ns);
+  phase ^= 1;
   tc_fence_after();
   if (ok) {
 #pragma unroll 1
     for (int cc = 0; cc < 4; ++cc) {
-      const int j0 = half * 64 + cc * 16;
+      const int j0 = hc * 64 + cc * 16;
       uint32_t v[16];
-      tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + 128 + j0, v);
+      tmem_ld16(tl + kAccX + j0, v);
       tmem_ld_wait();
-      float4* cd = reinterpret_cast<float4*>(a.C + off + (long long)i * D + j0);
+      float4* cd = reinterpret_cast<float4*>(a.C + off + (long long)ri * D + j0);
 #pragma unroll
       for (int t = 0; t < 4; ++t)
         cd[t] = make_float4(__uint_as_float(v[4 * t]), __uint_as_float(v[4 * t + 1]), __uint_as_float(v[4 * t + 2]),
@@ -387,12 +402,12 @@ __global__ void __launch_bounds__(kThreads, 1) solve_tc_kernel(const SolveArgs a
     }
   }
 
-  // ---------------- teardown
+  // ---------------- teardown: no MMA may still be running when TMEM is freed
   tc_fence_before();
   __syncthreads();
-  if (tid == 0 && *abort_flag) {
-    mbar_wait(bar_b, 0, nullptr, a.status, a.wait_ns);  // the bulk copy must have landed
-    mbar_wait(bar_p, 0, nullptr, a.status, a.wait_ns);
+  if (tid == 0 && *abort_flag && commits > 0) {
+    // Completions arrive in order: waiting for the last committed phase covers all.
+    mbar_wait(bar, phase ^ 1, nullptr, a.status, a.wait_ns);
   }
   __syncthreads();
   if (warp == 0) {
@@ -412,7 +427,7 @@ cudaError_t launch_solve_tc(const Problem& p, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  SolveArgs a{p.B, p.H, p.T, p.A, p.Bm, p.alpha, p.M, p.C, static_cast<__nv_bfloat16*>(p.Msplit), p.status,
+  SolveArgs a{p.B, p.H, p.T, p.A, p.Bm, p.alpha, p.M, p.C, static_cast<uint8_t*>(p.Msplit), p.status,
               p.spin_limit};
   dim3 grid(p.T - 1, p.H, p.B);
   solve_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(a);
