@@ -1,0 +1,58 @@
+// One-call entry point whose scratch memory is a static device array, for
+// callers that cannot allocate device memory: code running where no allocator
+// is available (a plugin handed only input and output buffers by its host
+// application, a process that must not grow its device footprint after start
+// up, or a caller that must not trigger the allocator's synchronisation). The
+// caller still owns Q, K, V, ..., gate and O; everything in between lives in
+// `g_static_workspace`, which every GPU that loads this library holds (64 MiB)
+// until the process exits.
+#include <cuda_runtime.h>
+
+#include "internal.h"
+
+namespace {
+
+constexpr size_t kStaticWorkspaceBytes = 64ull << 20;  // 64 MiB
+__device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
+
+constexpr int kMaxDevices = 64;
+void* g_workspace_addr[kMaxDevices] = {};  // device address of the array, per device
+
+}  // namespace
+
+extern "C" {
+
+size_t vda_static_workspace_capacity(void) { return kStaticWorkspaceBytes; }
+
+vda_status vda_run_static_workspace(const vda_config* cfg, const void* Q, const void* K, const void* V,
+                                    const void* K_txt, const void* V_txt, const float* alpha, const float* beta,
+                                    const float* beta_txt, const float* conv_w, const void* gate, void* O,
+                                    void* stream) {
+  size_t need = 0;
+  vda_status st = vda_workspace_size(cfg, &need);
+  if (st != VDA_OK) return st;
+  if (need > kStaticWorkspaceBytes) return VDA_ERR_WORKSPACE_TOO_SMALL;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return VDA_ERR_CUDA;
+  if (g_workspace_addr[dev] == nullptr) {
+    // In host code `g_static_workspace` names a host-side stand-in, not a device
+    // address: ask the runtime for this device's address of the array once.
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr) return VDA_ERR_CUDA;
+    g_workspace_addr[dev] = p;
+  }
+  vda_ctx* ctx = nullptr;
+  st = vda_create(cfg, &ctx);
+  if (st != VDA_OK) return st;
+  // vda_prepare clears the status word at the start of the workspace; every other
+  // region is fully written before it is read, so stale contents of an earlier
+  // call do not matter.
+  st = vda_prepare(ctx, Q, K, V, K_txt, V_txt, alpha, beta, beta_txt, conv_w, g_workspace_addr[dev],
+                   kStaticWorkspaceBytes, stream);
+  if (st == VDA_OK) st = vda_scan_bidir(ctx, stream);
+  if (st == VDA_OK) st = vda_readout(ctx, gate, O, stream);
+  vda_destroy(ctx);
+  return st;
+}
+
+}  // extern "C"

@@ -30,7 +30,8 @@ REGIONS = {"status": 0, "A": 1, "B": 2, "M": 3, "C": 4, "S_fwd": 5, "S_rev": 6,
 EXPORTS = ["vda_create", "vda_destroy", "vda_workspace_size", "vda_prepare", "vda_scan_bidir",
            "vda_readout", "vda_poll_device_status", "vda_workspace_region", "vda_status_string",
            "vda_last_error", "vda_profile_enable", "vda_num_kernels", "vda_profile_read",
-           "vda_launch_count", "vda_describe", "vda_selftest_bounded_wait"]
+           "vda_launch_count", "vda_describe", "vda_selftest_bounded_wait",
+           "vda_static_workspace_capacity", "vda_run_static_workspace"]
 
 
 class VDAError(RuntimeError):
@@ -79,8 +80,11 @@ def lib() -> ctypes.CDLL:
         L.vda_launch_count.argtypes = [vp, ctypes.POINTER(ctypes.c_uint64)]
         L.vda_describe.argtypes = [cfgp, ctypes.POINTER(ctypes.c_char_p)]
         L.vda_selftest_bounded_wait.argtypes = [vp, ctypes.c_uint64, vp]
+        L.vda_static_workspace_capacity.argtypes = []
+        L.vda_static_workspace_capacity.restype = ctypes.c_size_t
+        L.vda_run_static_workspace.argtypes = [cfgp] + [vp] * 11 + [vp]
         for name in EXPORTS:
-            if name not in ("vda_status_string", "vda_last_error"):
+            if name not in ("vda_status_string", "vda_last_error", "vda_static_workspace_capacity"):
                 getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -225,6 +229,15 @@ class VDA:
         n = ctypes.c_uint64(0)
         self._check(lib().vda_launch_count(self._ctx, ctypes.byref(n)), "vda_launch_count")
         return n.value
+
+
+def run_static_workspace(cfg: VDAConfig, inp: Dict[str, torch.Tensor], O: torch.Tensor, stream=None) -> int:
+    """The whole path through vda_run_static_workspace (library-owned scratch)."""
+    c = make_config(cfg)
+    return lib().vda_run_static_workspace(
+        ctypes.byref(c), _ptr(inp["Q"]), _ptr(inp["K"]), _ptr(inp["V"]), _ptr(inp["K_txt"]), _ptr(inp["V_txt"]),
+        _ptr(inp["alpha"]), _ptr(inp["beta"]), _ptr(inp["beta_txt"]), _ptr(inp.get("conv_w")),
+        _ptr(inp.get("gate")), _ptr(O), _stream_handle(stream))
 
 
 def selftest_bounded_wait(status: torch.Tensor, spins: int, stream=None) -> int:

@@ -204,6 +204,34 @@ vda_status vda_describe(const vda_config* cfg, const char** text);
  */
 vda_status vda_selftest_bounded_wait(uint32_t* status_dev, uint64_t spins, void* stream);
 
+/*
+ * The whole path (vda_prepare, vda_scan_bidir, vda_readout) in one call whose
+ * scratch lives in a static device array owned by the library, for callers that
+ * cannot allocate device memory: code that has no allocator at hand (a plugin
+ * given only its input and output buffers by a host application), a process that
+ * must not grow its device footprint after start-up, or a caller that must avoid
+ * the allocator's implicit synchronisation. The method pages have no counterpart
+ * of this call; it is a deployment convenience.
+ *  - Capacity: vda_static_workspace_capacity() bytes (64 MiB) on every device that
+ *    loads the library, held until the process exits. A cfg whose
+ *    vda_workspace_size() exceeds it returns VDA_ERR_WORKSPACE_TOO_SMALL before any
+ *    launch (the small workloads fit; the full-size clips need the caller-workspace
+ *    calls above).
+ *  - The first call on a device looks up that device's address of the array
+ *    (cudaGetSymbolAddress); make that first call before any stream capture.
+ *  - Every call shares the one array and leaves its contents behind: calls that
+ *    overlap on the GPU (other streams, other host threads) race and corrupt each
+ *    other's results, so serialise them.
+ *  - No cudaMalloc, cudaFree or allocating library routine is called.
+ * Arguments are those of vda_prepare and vda_readout; the call only enqueues
+ * work on `stream`.
+ */
+size_t vda_static_workspace_capacity(void);
+vda_status vda_run_static_workspace(const vda_config* cfg, const void* Q, const void* K, const void* V,
+                                    const void* K_txt, const void* V_txt, const float* alpha,
+                                    const float* beta, const float* beta_txt, const float* conv_w,
+                                    const void* gate, void* O, void* stream);
+
 #ifdef __cplusplus
 }
 #endif
