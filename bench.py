@@ -66,6 +66,12 @@ def kernel_bytes(name: str, cfg) -> float:
         return BH * ((F * U + L) * (2 * d * esz + 4) + 2 * NS * dd4)
     if name == "solve_simt":
         return BH * (4 * NS * dd4 + F * d * 4)
+    if name == "solve_tc":  # A, B read; M, C (fp32) and M's hi/lo operand images written
+        return BH * (4 * NS * dd4 + F * dd4 + F * d * 4)
+    if name == "scan_tc":  # per scanned frame: M's hi/lo images + C; S_T; readout states
+        fwd = max(0, c * (J - 2) - 1)
+        rev = max(0, (T - 2) - 2 * c + 1)
+        return BH * ((fwd + rev) * 2 * dd4 + 2 * dd4 + 2 * J * dd4)
     if name == "scan_simt":
         fwd = max(0, c * (J - 2) - 1)
         rev = max(0, (T - 2) - 2 * c + 1)
@@ -80,6 +86,28 @@ def kernel_bytes(name: str, cfg) -> float:
     if name == "prep_text":
         return BH * 4 * L * d * esz
     return 0.0
+
+
+def kernel_flops(name: str, cfg) -> float:
+    """Algorithmic flops per launch (the method's arithmetic, not the hi/lo split's)."""
+    B, H, d, T, U, L, c = cfg.B, cfg.H, cfg.d, cfg.T, cfg.U, cfg.L, cfg.chunk
+    F, NS, J = T - 2, T - 1, cfg.J
+    if name.startswith("gram"):
+        return B * H * (F * U + L) * 4 * d * d
+    if name.startswith("solve"):  # Cholesky d^3/3, L^-1 d^3/3, P d^3/3, C = B P 2 d^3
+        return B * H * NS * 3 * d ** 3
+    if name.startswith("scan"):
+        fwd = max(0, c * (J - 2) - 1)
+        rev = max(0, (T - 2) - 2 * c + 1)
+        return B * H * (fwd + rev) * 2 * d ** 3
+    if name.startswith("readout"):
+        return B * H * F * U * 2 * d * d
+    return 0.0
+
+
+# Kernels whose time is set by dense contractions and their serial dependencies
+# rather than by HBM streaming: their roofline is the bf16 tensor peak.
+TENSOR_BOUND = ("solve_tc", "solve_simt")
 
 
 def path_bytes(cfg) -> float:
@@ -108,7 +136,8 @@ def path_flops(cfg) -> float:
 
 
 def source_digest(kernel: str):
-    files = {"gram_tc": "gram_tc.cu", "readout_tc": "readout_tc.cu"}
+    files = {"gram_tc": "gram_tc.cu", "readout_tc": "readout_tc.cu", "solve_tc": "solve_tc.cu",
+             "scan_tc": "scan_tc.cu"}
     fn = files.get(kernel, "kernels_simt.cu")
     p = os.path.join(ROOT, "frame_level_delta_b200", "csrc", fn)
     with open(p, "rb") as f:
@@ -284,10 +313,14 @@ def main():
     ap.add_argument("--impl", default="vda", choices=["vda", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work (0: skip)")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="override H (a smaller case of the same workload, e.g. for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     cfg = CONFIGS[args.config]
+    if args.heads > 0:
+        cfg = cfg.with_(H=args.heads)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -377,11 +410,23 @@ def main():
     dom_name, (dom_n, dom_ms) = dom
     dom_avg_s = dom_ms / dom_n / 1e3
     dom_bytes = kernel_bytes(dom_name, cfg)
-    achieved = dom_bytes / dom_avg_s / 1e9
-    peak = float(peaks["hbm_gbs"])
     traffic = traffic_for(dom_name, cfg.name)
+    if dom_name in TENSOR_BOUND:
+        # timed inside a long step: the sustained bf16 figure is the denominator
+        bound, unit = "tensor", "TFLOP/s"
+        achieved = kernel_flops(dom_name, cfg) / dom_avg_s / 1e12
+        peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+        peak_note = f"bf16_tflops_sustained of {peak_src}"
+    else:
+        bound, unit = "hbm", "GB/s"
+        achieved = dom_bytes / dom_avg_s / 1e9
+        peak = float(peaks["hbm_gbs"])
+        peak_note = f"hbm_gbs of {peak_src}"
+    hbm_peak = float(peaks["hbm_gbs"])
     kernels = {k: {"launches": n, "avg_us": tot / n * 1e3, "share": tot / sum(x[1] for x in prof.values()),
-                   "algorithmic_GBps": kernel_bytes(k, cfg) / (tot / n / 1e3) / 1e9}
+                   "algorithmic_GBps": kernel_bytes(k, cfg) / (tot / n / 1e3) / 1e9,
+                   "hbm_frac": kernel_bytes(k, cfg) / (tot / n / 1e3) / 1e9 / hbm_peak,
+                   "algorithmic_TFLOPs": kernel_flops(k, cfg) / (tot / n / 1e3) / 1e12}
                for k, (n, tot) in prof.items()}
 
     if rank == 0:
@@ -396,13 +441,14 @@ def main():
                        "l2": "no flush: each step reads and writes > 1 GB, far above the 126 MB L2",
                        "path": V.describe(lib.c),
                        "stream": "one CUDA stream, kernels back to back"},
-            "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved, "peak": peak,
-                         "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
-                         "peak_source": f"hbm_gbs of {peak_src}",
-                         "algorithmic_bytes_per_launch": dom_bytes},
+            "roofline": {"bound": bound, "kernel": dom_name, "achieved": achieved, "peak": peak,
+                         "unit": unit, "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": peak_note,
+                         "algorithmic_bytes_per_launch": dom_bytes,
+                         "algorithmic_flops_per_launch": kernel_flops(dom_name, cfg)},
             "path_roofline": {"algorithmic_bytes_per_step": path_bytes(cfg),
                               "hbm_GBps": path_bytes(cfg) / step_s / 1e9,
-                              "hbm_frac": path_bytes(cfg) / step_s / 1e9 / peak,
+                              "hbm_frac": path_bytes(cfg) / step_s / 1e9 / hbm_peak,
                               "tflops": path_flops(cfg) / step_s / 1e12,
                               "tensor_frac_of_bf16_burst": path_flops(cfg) / step_s / 1e12 / float(peaks["bf16_tflops"])},
             "kernels": kernels,
