@@ -7,10 +7,11 @@
 // Both products contract over tokens, the slow axis of a [tokens x d] tile, so
 // both tcgen05 operands are MN-major: TMA brings K and V token tiles (64 tokens
 // x 64 channels per box, 128-byte swizzle, zero fill past the frame's last token)
-// into shared memory, four warps form beta*K in place of a third buffer (bf16,
-// round to nearest), and one thread issues tcgen05.mma with fp32 accumulation
-// in TMEM. Warp roles: 0 = TMA producer, 1 = TMEM owner + MMA issuer,
-// 2..5 = beta scaling, then the TMEM -> global epilogue.
+// into shared memory (six stages in flight), four warps write beta*K (bf16,
+// round to nearest) into a two-slot ring that the MMAs release, and one thread
+// issues tcgen05.mma with fp32 accumulation in TMEM: A = K^T (beta K),
+// B = V^T (beta K). Warp roles: 0 = TMA producer, 1 = TMEM owner + MMA issuer,
+// 2..5 = beta scaling, 6..9 = TMEM -> global epilogue.
 //
 // d = 128: two M=128 N=128 MMAs per 16-token step (K-part -> TMEM columns
 // 0..127, V-part -> 128..255). d = 64: one M=128 N=64 MMA whose A operand is
@@ -27,17 +28,23 @@ namespace {
 
 constexpr int kTileU = 64;                    // tokens per pipeline stage
 constexpr int kBoxBytes = kTileU * 128;       // one box: 64 tokens x 64 bf16
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // 10 warps: producer, MMA, 4 scaling, 4 epilogue
 
 template <int D>
 struct GramCfg {
   static constexpr int kBoxes = D / 64;                     // boxes per operand tile
-  static constexpr int kStageBytes = 3 * kBoxes * kBoxBytes;  // K, V, beta*K
-  static constexpr int kStages = D == 128 ? 4 : 8;
+  static constexpr int kStageBytes = 2 * kBoxes * kBoxBytes;  // K and V token tiles
+  static constexpr int kStages = D == 128 ? 6 : 12;         // HBM reads in flight per SM
+  static constexpr int kBkSlots = 2;                        // beta*K ring, released by the MMAs
+  static constexpr int kBkBytes = kBoxes * kBoxBytes;
   static constexpr int kTmemCols = D == 128 ? 256 : 64;
   static constexpr uint32_t kIdesc =
       D == 128 ? sm100::idesc_bf16_f32(128, 128, true, true) : sm100::idesc_bf16_f32(128, 64, true, true);
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int kBetaBytes = kStages * kTileU * 4;  // beta of each stage's tokens
+  static constexpr int kBarrierBytes = (2 * kStages + 2 * kBkSlots + 5) * 8 + 16;  // mbarriers + TMEM slot, flags
+  static constexpr int kSmemBytes = kStages * kStageBytes + kBkSlots * kBkBytes + kBetaBytes + 1024 /*align*/ + 512;
+  static_assert(kBarrierBytes <= 512, "barrier block overflows its allowance");
+  static_assert(kSmemBytes <= 232448, "more shared memory than a CTA may use");
 };
 
 struct GramArgs {
@@ -51,6 +58,24 @@ struct GramArgs {
   unsigned long long wait_ns;
 };
 
+// Unit u = (b, h, slot) with heads fastest, so the CTAs working at any moment
+// cover all heads of neighbouring frames (one 6 KB token row holds every head).
+struct Unit {
+  int b, h, slot, n;
+};
+__device__ __forceinline__ Unit unit_of(const GramArgs& a, int u) {
+  Unit x;
+  x.h = u % a.H;
+  const int r = u / a.H;
+  x.slot = r % (a.T - 1);
+  x.b = r / (a.T - 1);
+  x.n = x.slot == 0 ? a.L : a.U;
+  return x;
+}
+
+// Persistent: CTA p takes units p, p + G, p + 2G, ... and streams their token
+// tiles through one continuous TMA pipeline; the accumulator alternates between
+// two TMEM buffers so the epilogue of one unit overlaps the MMAs of the next.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     gram_tc_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
@@ -60,38 +85,47 @@ __global__ void __launch_bounds__(kThreads, 1)
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
-  uint64_t* bkf = full + C::kStages;
-  uint64_t* empty = bkf + C::kStages;
-  uint64_t* accb = empty + C::kStages;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accb + 1);
+  uint8_t* bkring = smem + C::kStages * C::kStageBytes;  // beta*K slots
+  float* sbeta = reinterpret_cast<float*>(bkring + C::kBkSlots * C::kBkBytes);  // [kStages][kTileU]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sbeta + C::kStages * kTileU);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* bkf = empty + C::kStages;     // [kBkSlots] beta*K written
+  uint64_t* bke = bkf + C::kBkSlots;      // [kBkSlots] beta*K slot free again
+  uint64_t* tfull = bke + C::kBkSlots;    // [2]
+  uint64_t* tempty = tfull + 2;          // [2]
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* issued_slot = reinterpret_cast<int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int slot = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const bool text = slot == 0;
-  const int n = text ? a.L : a.U;
-  const int ntiles = (n + kTileU - 1) / kTileU;
-  const CUtensorMap* mk = text ? &mKt : &mK;
-  const CUtensorMap* mv = text ? &mVt : &mV;
-  const int tc = text ? 0 : slot;
+  const int nunits = a.B * a.H * (a.T - 1);
+  const int G = gridDim.x;
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&bkf[s], 4);
+      mbar_init(&full[s], 1 + 32);  // TMA bytes + the 32 lanes' beta copies
       mbar_init(&empty[s], 1);
     }
-    mbar_init(accb, 1);
+    for (int i = 0; i < C::kBkSlots; ++i) {
+      mbar_init(&bkf[i], 4);
+      mbar_init(&bke[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4);
+    }
+    mbar_init(drain, 1);
     *abort_flag = 0;
     *issued_slot = 0;
     fence_mbar_init();
-    prefetch_tmap(mk);
-    prefetch_tmap(mv);
+    prefetch_tmap(&mK);
+    prefetch_tmap(&mV);
+    prefetch_tmap(&mKt);
+    prefetch_tmap(&mVt);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_alloc(tmem_slot, 2 * C::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -100,66 +134,102 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------- TMA producer
-    if (lane == 0) {
-      int it = 0;
-      for (; it < ntiles; ++it) {
+    // ---------------- producer warp: TMA loads of K, V (lane 0) and asynchronous
+    // copies of the stage's beta values (all lanes), all completing on full[s],
+    // so beta arrives as far ahead of its use as the token tiles do.
+    int it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < nunits && ok; u += G) {
+      const Unit x = unit_of(a, u);
+      const CUtensorMap* mk = x.slot == 0 ? &mKt : &mK;
+      const CUtensorMap* mv = x.slot == 0 ? &mVt : &mV;
+      const float* beta = x.slot == 0 ? a.beta_txt + ((long long)x.b * a.H + x.h) * a.L
+                                      : a.beta + (((long long)x.b * a.H + x.h) * a.T + x.slot) * (long long)a.U;
+      const int ntiles = (x.n + kTileU - 1) / kTileU;
+      for (int tt = 0; tt < ntiles; ++tt, ++it) {
         const int s = it % C::kStages;
         const uint32_t ph = (it / C::kStages) & 1;
-        if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, a.status, a.wait_ns)) break;
-        uint8_t* st = smem + s * C::kStageBytes;
-        mbar_arrive_expect_tx(&full[s], 2 * C::kBoxes * kBoxBytes);
-        const int u0 = it * kTileU;
+        int good = 1;
+        if (lane == 0) good = mbar_wait(&empty[s], ph ^ 1, abort_flag, a.status, a.wait_ns) ? 1 : 0;
+        good = __shfl_sync(0xffffffffu, good, 0);
+        if (!good) { ok = false; break; }
+        const int u0 = tt * kTileU;
+        if (lane == 0) {
+          uint8_t* st = smem + s * C::kStageBytes;
+          mbar_arrive_expect_tx(&full[s], 2 * C::kBoxes * kBoxBytes);
 #pragma unroll
-        for (int box = 0; box < C::kBoxes; ++box) {
-          const int d0 = box * 64;
-          if (a.layout == 0) {
-            tma_load_5d(st + box * kBoxBytes, mk, &full[s], d0, h, u0, tc, b);
-            tma_load_5d(st + (C::kBoxes + box) * kBoxBytes, mv, &full[s], d0, h, u0, tc, b);
-          } else {
-            tma_load_5d(st + box * kBoxBytes, mk, &full[s], d0, u0, tc, h, b);
-            tma_load_5d(st + (C::kBoxes + box) * kBoxBytes, mv, &full[s], d0, u0, tc, h, b);
+          for (int box = 0; box < C::kBoxes; ++box) {
+            const int d0 = box * 64;
+            if (a.layout == 0) {
+              tma_load_5d(st + box * kBoxBytes, mk, &full[s], d0, x.h, u0, x.slot, x.b);
+              tma_load_5d(st + (C::kBoxes + box) * kBoxBytes, mv, &full[s], d0, x.h, u0, x.slot, x.b);
+            } else {
+              tma_load_5d(st + box * kBoxBytes, mk, &full[s], d0, u0, x.slot, x.h, x.b);
+              tma_load_5d(st + (C::kBoxes + box) * kBoxBytes, mv, &full[s], d0, u0, x.slot, x.h, x.b);
+            }
           }
         }
+        // beta of tokens u0 + lane and u0 + 32 + lane (zero past the slot's last token)
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int uu = u0 + half * 32 + lane;
+          const bool in = uu < x.n;
+          cp_async_4(sbeta + s * kTileU + half * 32 + lane, in ? beta + uu : beta, in ? 4u : 0u);
+        }
+        cp_async_mbar_arrive_noinc(&full[s]);
       }
-      *issued_slot = it;
     }
+    if (lane == 0) *issued_slot = it;
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
-      uint32_t acc = 0;
-      for (int it = 0; it < ntiles; ++it) {
-        const int s = it % C::kStages;
-        const uint32_t ph = (it / C::kStages) & 1;
-        if (!mbar_wait(&full[s], ph, abort_flag, a.status, a.wait_ns)) break;
-        if (!mbar_wait(&bkf[s], ph, abort_flag, a.status, a.wait_ns)) break;
+      int it = 0, k = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < nunits && ok; u += G, ++k) {
+        const Unit x = unit_of(a, u);
+        const int ntiles = (x.n + kTileU - 1) / kTileU;
+        const int ub = k & 1;
+        const uint32_t tacc = tmem + ub * C::kTmemCols;
+        if (!mbar_wait(&tempty[ub], ((k >> 1) & 1) ^ 1, abort_flag, a.status, a.wait_ns)) break;
         tc_fence_after();
-        const uint32_t base = smem_u32(smem + s * C::kStageBytes);
-#pragma unroll
-        for (int k = 0; k < kTileU / 16; ++k) {
-          const uint32_t koff = k * 16 * 128;  // 16 token rows of 128 bytes
-          if constexpr (D == 128) {
-            const uint64_t dK = smem_desc_sw128(base + koff, kBoxBytes, 1024);
-            const uint64_t dV = smem_desc_sw128(base + 2 * kBoxBytes + koff, kBoxBytes, 1024);
-            const uint64_t dB = smem_desc_sw128(base + 4 * kBoxBytes + koff, kBoxBytes, 1024);
-            mma_f16(tmem, dK, dB, C::kIdesc, acc);
-            mma_f16(tmem + 128, dV, dB, C::kIdesc, acc);
-          } else {
-            const uint64_t dKV = smem_desc_sw128(base + koff, kBoxBytes, 1024);  // K box then V box
-            const uint64_t dB = smem_desc_sw128(base + 2 * kBoxBytes + koff, kBoxBytes, 1024);
-            mma_f16(tmem, dKV, dB, C::kIdesc, acc);
+        for (int tt = 0; tt < ntiles; ++tt, ++it) {
+          const int s = it % C::kStages;
+          const uint32_t ph = (it / C::kStages) & 1;
+          const int bs = it % C::kBkSlots;
+          const uint32_t bph = (it / C::kBkSlots) & 1;
+          if (!mbar_wait(&full[s], ph, abort_flag, a.status, a.wait_ns) ||
+              !mbar_wait(&bkf[bs], bph, abort_flag, a.status, a.wait_ns)) {
+            ok = false;
+            break;
           }
-          acc = 1;
+          tc_fence_after();
+          const uint32_t base = smem_u32(smem + s * C::kStageBytes);
+          const uint32_t bkb = smem_u32(bkring + bs * C::kBkBytes);
+#pragma unroll
+          for (int kk = 0; kk < kTileU / 16; ++kk) {
+            const uint32_t koff = kk * 16 * 128;  // 16 token rows of 128 bytes
+            const uint32_t acc = (tt > 0 || kk > 0) ? 1u : 0u;
+            const uint64_t dB = smem_desc_sw128(bkb + koff, kBoxBytes, 1024);  // beta*K
+            if constexpr (D == 128) {
+              const uint64_t dK = smem_desc_sw128(base + koff, kBoxBytes, 1024);
+              const uint64_t dV = smem_desc_sw128(base + 2 * kBoxBytes + koff, kBoxBytes, 1024);
+              mma_f16(tacc, dK, dB, C::kIdesc, acc);
+              mma_f16(tacc + 128, dV, dB, C::kIdesc, acc);
+            } else {
+              const uint64_t dKV = smem_desc_sw128(base + koff, kBoxBytes, 1024);  // K box then V box
+              mma_f16(tacc, dKV, dB, C::kIdesc, acc);
+            }
+          }
+          mma_commit(&empty[s]);
+          mma_commit(&bke[bs]);
         }
-        mma_commit(&empty[s]);
+        if (ok) mma_commit(&tfull[ub]);
       }
-      mma_commit(accb);  // completes once every MMA issued above has finished
+      mma_commit(drain);  // completes once every MMA issued above has finished
     }
-  } else {
-    // ---------------- beta scaling (warps 2..5), then the epilogue
+  } else if (warp < 6) {
+    // ---------------- beta*K into the ring (warps 2..5)
     const int tid = threadIdx.x - 64;  // 0..127
-    const float* beta = text ? a.beta_txt + ((long long)b * a.H + h) * a.L
-                             : a.beta + (((long long)b * a.H + h) * a.T + slot) * (long long)a.U;
     int row, box, c0, c1;
     if constexpr (D == 128) {
       box = tid / 64;
@@ -172,42 +242,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       c0 = (tid % 2) * 4;
       c1 = c0 + 4;
     }
+    int it = 0;
     bool ok = true;
-    for (int it = 0; it < ntiles; ++it) {
-      const int s = it % C::kStages;
-      const uint32_t ph = (it / C::kStages) & 1;
-      if (!mbar_wait(&full[s], ph, abort_flag, a.status, a.wait_ns)) {
-        ok = false;
-        break;
-      }
-      uint8_t* st = smem + s * C::kStageBytes;
-      const int u = it * kTileU + row;
-      const float bb = u < n ? __ldg(beta + u) : 0.f;
-      const uint8_t* src = st + box * kBoxBytes + row * 128;
-      uint8_t* dst = st + (2 * C::kBoxes + box) * kBoxBytes + row * 128;
-      for (int c = c0; c < c1; ++c) {
-        const int pc = c ^ (row & 7);  // any chunk order works; this one avoids bank conflicts
-        uint4 v = *reinterpret_cast<const uint4*>(src + pc * 16);
-        __nv_bfloat162* e = reinterpret_cast<__nv_bfloat162*>(&v);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float2 f = __bfloat1622float2(e[q]);
-          e[q] = __floats2bfloat162_rn(f.x * bb, f.y * bb);
+    for (int u = blockIdx.x; u < nunits && ok; u += G) {
+      const Unit x = unit_of(a, u);
+      const int ntiles = (x.n + kTileU - 1) / kTileU;
+      for (int tt = 0; tt < ntiles; ++tt, ++it) {
+        const int s = it % C::kStages;
+        const uint32_t ph = (it / C::kStages) & 1;
+        const int bs = it % C::kBkSlots;
+        const uint32_t bph = (it / C::kBkSlots) & 1;
+        if (!mbar_wait(&bke[bs], bph ^ 1, abort_flag, a.status, a.wait_ns) ||
+            !mbar_wait(&full[s], ph, abort_flag, a.status, a.wait_ns)) {
+          ok = false;
+          break;
         }
-        *reinterpret_cast<uint4*>(dst + pc * 16) = v;
+        const float bb = sbeta[s * kTileU + row];  // zero past the slot's last token
+        const uint8_t* src = smem + s * C::kStageBytes + box * kBoxBytes + row * 128;
+        uint8_t* dst = bkring + bs * C::kBkBytes + box * kBoxBytes + row * 128;
+        for (int c = c0; c < c1; ++c) {
+          const int pc = c ^ (row & 7);  // any chunk order works; this one avoids bank conflicts
+          uint4 v = *reinterpret_cast<const uint4*>(src + pc * 16);
+          __nv_bfloat162* e = reinterpret_cast<__nv_bfloat162*>(&v);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float2 f = __bfloat1622float2(e[q]);
+            e[q] = __floats2bfloat162_rn(f.x * bb, f.y * bb);
+          }
+          *reinterpret_cast<uint4*>(dst + pc * 16) = v;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bkf[bs]);
       }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bkf[s]);
     }
-    if (ok && mbar_wait(accb, 0, abort_flag, a.status, a.wait_ns)) {
+  } else {
+    // ---------------- epilogue (warps 6..9): TMEM -> A, B in global memory
+    const int q = warp % 4;  // this warp may read TMEM lanes 32q .. 32q+31
+    const int r = q * 32 + lane;
+    int k = 0;
+    for (int u = blockIdx.x; u < nunits; u += G, ++k) {
+      const Unit x = unit_of(a, u);
+      const int ub = k & 1;
+      if (!mbar_wait(&tfull[ub], (k >> 1) & 1, abort_flag, a.status, a.wait_ns)) break;
       tc_fence_after();
-      const int q = warp % 4;  // this warp may read TMEM lanes 32q .. 32q+31
-      const int r = q * 32 + lane;
-      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16);
-      const long long off = (((long long)b * a.H + h) * (a.T - 1) + slot) * (long long)D * D;
+      const uint32_t taddr = tmem + ub * C::kTmemCols + ((uint32_t)(q * 32) << 16);
+      const long long off = (((long long)x.b * a.H + x.h) * (a.T - 1) + x.slot) * (long long)D * D;
       if constexpr (D == 128) {
-#pragma unroll 1
+#pragma unroll 2
         for (int c = 0; c < 16; ++c) {
           uint32_t v[16];
           tmem_ld16(taddr + c * 16, v);
@@ -233,6 +315,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[ub]);
     }
   }
 
@@ -249,10 +334,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   if (warp == 1) {
-    if (lane == 0) mbar_wait(accb, 0, nullptr, a.status, a.wait_ns);  // all MMAs retired
+    if (lane == 0) mbar_wait(drain, 0, nullptr, a.status, a.wait_ns);  // all MMAs retired
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
+    tmem_dealloc(tmem, 2 * C::kTmemCols);
   }
 }
 
@@ -303,7 +388,11 @@ cudaError_t launch_d(const Problem& p, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid(p.T - 1, p.H, p.B);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int nunits = p.B * p.H * (p.T - 1);
+  const int grid = nunits < sms ? nunits : sms;
   gram_tc_kernel<D><<<grid, kThreads, C::kSmemBytes, s>>>(mK, mV, mKt, mVt, a);
   return cudaGetLastError();
 }

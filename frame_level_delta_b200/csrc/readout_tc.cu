@@ -31,9 +31,8 @@ namespace {
 
 constexpr int kTileM = 128;
 constexpr int kThreads = 192;
-constexpr int kStages = 2;
 
-template <int D>
+template <int D, bool GATE>
 struct RoCfg {
   static constexpr int kBoxes = D / 64;                   // 64-channel boxes per token tile
   static constexpr int kTileBytes = kTileM * D * 2;       // one bf16 token tile
@@ -41,8 +40,14 @@ struct RoCfg {
   static constexpr int kSBytes = kBoxes * kSAtomBytes;    // one bf16 copy of S
   static constexpr int kTmemCols = 2 * D;                 // two accumulators
   static constexpr uint32_t kIdesc = sm100::idesc_bf16_f32(128, D, false, false);
-  // layout: S_hi | S_lo | Q[kStages] | AUX[kStages] | barriers
-  static constexpr int kSmemBytes = 2 * kSBytes + 2 * kStages * kTileBytes + 1024 + 256;
+  // Q tiles are the only stream without the gate: four stages deep. With the
+  // gate, a stage holds a Q tile and a gate tile: two stages.
+  static constexpr int kStages = GATE ? 2 : (D == 128 ? 4 : 6);
+  static constexpr int kStageBytes = kTileBytes * (GATE ? 2 : 1);
+  // layout: S_hi | S_lo | stages | output staging tile | barriers
+  static constexpr int kSmemBytes = 2 * kSBytes + kStages * kStageBytes + kTileBytes + 1024 + 256;
+  static_assert((2 * kStages + 7) * 8 + 16 <= 256, "barrier block overflows its allowance");
+  static_assert(kSmemBytes <= 232448, "more shared memory than a CTA may use");
 };
 
 struct RoArgs {
@@ -54,8 +59,9 @@ struct RoArgs {
   __nv_bfloat16* O;
   uint32_t* status;
   unsigned long long wait_ns;
-  long long total_tiles;
-  long long tiles_per_cta;
+  int BH;           // B * H
+  int nseg;         // token segments per (b, h); CTA p serves (b, h) = p % BH, segment p / BH
+  int tiles_per_seg;
 };
 
 // Non-anchor frame range [t_lo, t_hi) of chunk j.
@@ -76,10 +82,9 @@ struct TileInfo {
   int nvalid;        // rows of the tile inside the chunk
 };
 
-__device__ __forceinline__ TileInfo tile_info(const RoArgs& a, long long id, int tiles_per_head) {
+__device__ __forceinline__ TileInfo tile_info(const RoArgs& a, int bh, int local) {
   TileInfo ti;
-  ti.bh = (int)(id / tiles_per_head);
-  int local = (int)(id % tiles_per_head);
+  ti.bh = bh;
   int j = 0;
   for (;; ++j) {
     const int n = chunk_tiles(a, j);
@@ -109,19 +114,20 @@ __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_
 
 __device__ __forceinline__ float sigmoid_f(float x) { return 1.0f / (1.0f + __expf(-x)); }
 
-template <int D>
+template <int D, bool GATE>
 __global__ void __launch_bounds__(kThreads, 1)
     readout_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mG,
                       const __grid_constant__ CUtensorMap mO, const RoArgs a) {
-  using C = RoCfg<D>;
+  using C = RoCfg<D, GATE>;
+  constexpr int kStages = C::kStages;
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sShi = smem;
   uint8_t* sSlo = smem + C::kSBytes;
-  uint8_t* sQ = smem + 2 * C::kSBytes;
-  uint8_t* sAux = sQ + kStages * C::kTileBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sAux + kStages * C::kTileBytes);
+  uint8_t* sQ = smem + 2 * C::kSBytes;  // stage s: Q tile at s * kStageBytes, gate tile after it
+  uint8_t* sO = sQ + kStages * C::kStageBytes;  // output tile staged for the TMA store
+  uint64_t* full = reinterpret_cast<uint64_t*>(sO + C::kTileBytes);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
   uint64_t* tempty = tfull + 2;
@@ -132,18 +138,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const bool gate = (a.flags & VDA_READOUT_NORM_GATE) != 0;
+  constexpr bool gate = GATE;
   const bool qnorm = (a.flags & VDA_PREP_CONV) != 0;
+  const bool stage_read = qnorm || GATE;  // the epilogue reads the stage's tiles
   int tiles_per_head = 0;
   for (int j = 0; j < a.J; ++j) tiles_per_head += chunk_tiles(a, j);
-  const long long t_begin = (long long)blockIdx.x * a.tiles_per_cta;
-  const long long t_end = min(a.total_tiles, t_begin + a.tiles_per_cta);
-  const int ntiles = t_begin < t_end ? (int)(t_end - t_begin) : 0;
+  // CTA p serves head pair bh = p % BH over its token segment p / BH: the CTAs of
+  // one segment walk the same tokens of all heads in step, which keeps their
+  // strided reads and writes within the same DRAM rows.
+  const int my_bh = blockIdx.x % a.BH, seg = blockIdx.x / a.BH;
+  const int t_begin = seg * a.tiles_per_seg;
+  const int t_end = min(tiles_per_head, t_begin + a.tiles_per_seg);
+  const int ntiles = t_begin < t_end ? t_end - t_begin : 0;
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 2);  // MMA commit + epilogue
+      mbar_init(&empty[s], stage_read ? 5 : 1);  // MMA commit (+ 4 epilogue warps)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
@@ -176,15 +187,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
         if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, a.status, a.wait_ns)) break;
-        const TileInfo ti = tile_info(a, t_begin + it, tiles_per_head);
+        const TileInfo ti = tile_info(a, my_bh, t_begin + it);
         const int h = ti.bh % a.H;
         mbar_arrive_expect_tx(&full[s], bytes);
 #pragma unroll
         for (int box = 0; box < C::kBoxes; ++box) {
-          tma_load_3d(sQ + s * C::kTileBytes + box * (kTileM * 128), &mQ, &full[s], box * 64, h, (int)ti.tok0);
-          if (gate)
-            tma_load_3d(sAux + s * C::kTileBytes + box * (kTileM * 128), &mG, &full[s], box * 64, h,
-                        (int)ti.tok0);
+          tma_load_3d(sQ + s * C::kStageBytes + box * (kTileM * 128), &mQ, &full[s], box * 64, h, (int)ti.tok0);
+          if constexpr (GATE)
+            tma_load_3d(sQ + s * C::kStageBytes + C::kTileBytes + box * (kTileM * 128), &mG, &full[s], box * 64,
+                        h, (int)ti.tok0);
         }
         issued = it + 1;
       }
@@ -194,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int g_prev = -1, gi = 0;
       for (int it = 0; it < ntiles; ++it) {
-        const TileInfo ti = tile_info(a, t_begin + it, tiles_per_head);
+        const TileInfo ti = tile_info(a, my_bh, t_begin + it);
         const int g = ti.bh * a.J + ti.j;
         if (g != g_prev) {
           if (!mbar_wait(sready, gi & 1, abort_flag, a.status, a.wait_ns)) break;
@@ -208,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&full[s], ph, abort_flag, a.status, a.wait_ns)) break;
         if (!mbar_wait(&tempty[tb], tph ^ 1, abort_flag, a.status, a.wait_ns)) break;
         tc_fence_after();
-        const uint32_t qb = smem_u32(sQ + s * C::kTileBytes);
+        const uint32_t qb = smem_u32(sQ + s * C::kStageBytes);
         const uint32_t hb = smem_u32(sShi), lb = smem_u32(sSlo);
         const uint32_t dtm = tmem + tb * D;
 #pragma unroll
@@ -243,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       return r;
     };
     for (int it = 0; it < ntiles && ok; ++it) {
-      const TileInfo ti = tile_info(a, t_begin + it, tiles_per_head);
+      const TileInfo ti = tile_info(a, my_bh, t_begin + it);
       const int g = ti.bh * a.J + ti.j;
       if (g != g_prev) {
         // The MMAs of the previous tile are complete (its accumulator was read
@@ -282,10 +293,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tb = it & 1;
       const uint32_t tph = (it >> 1) & 1;
       if (!mbar_wait(&tfull[tb], tph, abort_flag, a.status, a.wait_ns)) { ok = false; break; }
-      if (!mbar_wait(&full[s], ph, abort_flag, a.status, a.wait_ns)) { ok = false; break; }
       tc_fence_after();
-      const uint8_t* qrow = sQ + s * C::kTileBytes + r * 128;
-      uint8_t* arow = sAux + s * C::kTileBytes + r * 128;
+      // The Q tile (and gate tile) of this stage stay valid until this epilogue
+      // releases the stage; without q-norm or gate the MMA commit alone releases it.
+      if (stage_read && !mbar_wait(&full[s], ph, abort_flag, a.status, a.wait_ns)) { ok = false; break; }
+      const uint8_t* qrow = sQ + s * C::kStageBytes + r * 128;
+      const uint8_t* grow = qrow + C::kTileBytes;
       float scale = 1.f;
       if (qnorm) {
         float qq = 0.f;
@@ -305,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + tb * D;
       float rn = 1.f;
-      if (gate) {
+      if constexpr (GATE) {
         float ss = 0.f;
 #pragma unroll 1
         for (int cc = 0; cc < D / 16; ++cc) {
@@ -320,22 +333,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         rn = rsqrtf(ss / D + a.rms_eps);
       }
-      const bool partial = ti.nvalid < kTileM;
-      const int h = ti.bh % a.H;
-      __nv_bfloat16* orow = a.O + ((ti.tok0 + r) * a.H + h) * (long long)D;
-#pragma unroll 1
+      // Output row into registers: 16-byte chunk pair (2cc, 2cc+1) holds columns 16cc..16cc+15.
+      uint4 outs[D / 8];
+#pragma unroll
       for (int cc = 0; cc < D / 16; ++cc) {
         uint32_t v[16];
         tmem_ld16(taddr + cc * 16, v);
         tmem_ld_wait();
-        const int box = cc / 4, c16 = (cc % 4) * 2;  // two 16-byte chunks per 16 columns
-        uint4 outv[2];
+        const int box = cc / 4, c16 = (cc % 4) * 2;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          const int pc = (c16 + half) ^ (r & 7);
           float g8[8];
-          if (gate) {
-            const uint4 gv = *reinterpret_cast<const uint4*>(arow + box * (kTileM * 128) + pc * 16);
+          if constexpr (GATE) {
+            const int pc = (c16 + half) ^ (r & 7);
+            const uint4 gv = *reinterpret_cast<const uint4*>(grow + box * (kTileM * 128) + pc * 16);
             const __nv_bfloat162* ge = reinterpret_cast<const __nv_bfloat162*>(&gv);
 #pragma unroll
             for (int k2 = 0; k2 < 4; ++k2) {
@@ -347,35 +358,43 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < 8; ++k) g8[k] = 1.f;
           }
-          __nv_bfloat162* op = reinterpret_cast<__nv_bfloat162*>(&outv[half]);
+          __nv_bfloat162* op = reinterpret_cast<__nv_bfloat162*>(&outs[2 * cc + half]);
 #pragma unroll
           for (int k2 = 0; k2 < 4; ++k2)
             op[k2] = __floats2bfloat162_rn(__uint_as_float(v[half * 8 + 2 * k2]) * scale * g8[2 * k2],
                                            __uint_as_float(v[half * 8 + 2 * k2 + 1]) * scale * g8[2 * k2 + 1]);
-          if (!partial) {
-            *reinterpret_cast<uint4*>(arow + box * (kTileM * 128) + pc * 16) = outv[half];
-          }
-        }
-        if (partial && r < ti.nvalid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + cc * 16);
-          dst[0] = outv[0];
-          dst[1] = outv[1];
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[tb]);
+      if (lane == 0) {
+        mbar_arrive(&tempty[tb]);
+        if (stage_read) mbar_arrive(&empty[s]);
+      }
+      // The staging buffer must have been read by the previous tile's TMA store.
+      if (et == 0) bulk_wait_read0();
+      if (!epi_sync()) { ok = false; break; }
+      const bool partial = ti.nvalid < kTileM;
+      const int h = ti.bh % a.H;
+      if (!partial) {
+        uint8_t* orow = sO + r * 128;
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          const int box = c / 8, pc = (c % 8) ^ (r & 7);
+          *reinterpret_cast<uint4*>(orow + box * (kTileM * 128) + pc * 16) = outs[c];
+        }
+      } else if (r < ti.nvalid) {
+        uint4* dst = reinterpret_cast<uint4*>(a.O + ((ti.tok0 + r) * a.H + h) * (long long)D);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) dst[c] = outs[c];
+      }
       fence_proxy_async_smem();
       if (!epi_sync()) { ok = false; break; }
-      if (et == 0) {
-        if (!partial) {
+      if (et == 0 && !partial) {
 #pragma unroll
-          for (int box = 0; box < C::kBoxes; ++box)
-            tma_store_3d(&mO, sAux + s * C::kTileBytes + box * (kTileM * 128), box * 64, h, (int)ti.tok0);
-          bulk_commit();
-          bulk_wait_read0();
-        }
-        mbar_arrive(&empty[s]);
+        for (int box = 0; box < C::kBoxes; ++box)
+          tma_store_3d(&mO, sO + box * (kTileM * 128), box * 64, h, (int)ti.tok0);
+        bulk_commit();
       }
     }
     if (et == 0) bulk_wait0();  // all output writes done before the CTA retires
@@ -399,9 +418,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
-cudaError_t launch_d(const Problem& p, const void* gate, void* O, cudaStream_t s) {
-  using C = RoCfg<D>;
+template <int D, bool GATE>
+cudaError_t launch_dg(const Problem& p, const void* gate, void* O, cudaStream_t s) {
+  using C = RoCfg<D, GATE>;
   RoArgs a{};
   a.B = p.B; a.H = p.H; a.T = p.T; a.U = p.U; a.c = p.c; a.J = p.J;
   a.flags = p.flags; a.l2_eps = p.l2_eps; a.rms_eps = p.rms_eps;
@@ -412,24 +431,25 @@ cudaError_t launch_d(const Problem& p, const void* gate, void* O, cudaStream_t s
     const int lo = std::max(p.c * j, 1), hi = std::min(p.c * (j + 1), p.T - 1);
     if (lo < hi) tiles_per_head += ((long long)(hi - lo) * p.U + kTileM - 1) / kTileM;
   }
-  a.total_tiles = tiles_per_head * p.B * p.H;
-  if (a.total_tiles == 0) return cudaSuccess;
+  if (tiles_per_head == 0) return cudaSuccess;
+  a.BH = p.B * p.H;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   static bool attr_set = false;
   cudaError_t e;
   if (!attr_set) {
-    e = cudaFuncSetAttribute(readout_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    e = cudaFuncSetAttribute(readout_tc_kernel<D, GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   int per_sm = 1;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, readout_tc_kernel<D>, kThreads, C::kSmemBytes);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, readout_tc_kernel<D, GATE>, kThreads, C::kSmemBytes);
   if (per_sm < 1) per_sm = 1;
-  const long long grid = std::min<long long>(a.total_tiles, (long long)sms * per_sm);
-  a.tiles_per_cta = (a.total_tiles + grid - 1) / grid;
-  const long long ncta = (a.total_tiles + a.tiles_per_cta - 1) / a.tiles_per_cta;
+  const long long slots = (long long)sms * per_sm;
+  a.nseg = (int)std::max<long long>(1, std::min<long long>(slots / a.BH, tiles_per_head));
+  a.tiles_per_seg = (int)((tiles_per_head + a.nseg - 1) / a.nseg);
+  const long long ncta = (long long)a.BH * a.nseg;
 
   // [B*T*U tokens, H, D] views of Q, gate and O: dims (d, h, token)
   const uint64_t D64 = D, H = p.H, NT = (uint64_t)p.B * p.T * p.U;
@@ -440,8 +460,14 @@ cudaError_t launch_d(const Problem& p, const void* gate, void* O, cudaStream_t s
   if ((e = make_tmap_bf16(&mQ, p.Q, 3, dims, strides, box)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16(&mO, O, 3, dims, strides, box)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16(&mG, gate ? gate : p.Q, 3, dims, strides, box)) != cudaSuccess) return e;
-  readout_tc_kernel<D><<<(unsigned)ncta, kThreads, C::kSmemBytes, s>>>(mQ, mG, mO, a);
+  readout_tc_kernel<D, GATE><<<(unsigned)ncta, kThreads, C::kSmemBytes, s>>>(mQ, mG, mO, a);
   return cudaGetLastError();
+}
+
+
+template <int D>
+cudaError_t launch_d(const Problem& p, const void* gate, void* O, cudaStream_t s) {
+  return (p.flags & VDA_READOUT_NORM_GATE) ? launch_dg<D, true>(p, gate, O, s) : launch_dg<D, false>(p, gate, O, s);
 }
 
 }  // namespace

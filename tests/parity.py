@@ -14,12 +14,14 @@ from oracle import vda_oracle as vo
 TOL_O = {"f32": 1e-4, "bf16": 2e-2}
 # Bounds on the fp32 intermediates (A, B, M, C, S_T, readout states), per slot.
 # The CUDA-core kernels compute them in fp32 from the exact stored inputs
-# (relative error ~1e-6, amplified by cond(I + A) <= ~1e3): 1e-4. Where a bf16
-# rounding enters before the statistics -- the tcgen05 statistics kernel rounds
-# beta*K to bf16, and under the conv prep the prepared K, V copies are stored in
-# bf16 -- each term carries up to 2^-9 relative error: 4e-3.
+# (relative error ~1e-6, amplified by cond(I + A) <= ~1e3): 1e-4. Each bf16
+# rounding of an operand before the statistics adds up to 2^-9 relative error
+# per rounded operand (~2e-3): the tcgen05 statistics kernel rounds beta*K to
+# bf16, and under the conv prep the prepared K, V copies are stored in bf16.
+# Bound: 4e-3 per rounding level.
 TOL_STAGE_SIMT = 1e-4
-TOL_STAGE_TC = 4e-3
+TOL_STAGE_PER_ROUNDING = 4e-3
+TOL_STAGE_TC = TOL_STAGE_PER_ROUNDING
 
 
 def rel_fro(a, b) -> float:
@@ -76,9 +78,10 @@ def check_config(cfg, heads=None, force_simt=False, inp=None, stage_tol=None):
     O_g = O_gpu.numpy()
     err_o = rel_fro(O_g[np.ix_(bs, range(O_g.shape[1]), hs)], O_ref[np.ix_(bs, range(O_ref.shape[1]), hs)])
     stages = staged_errors(cfg, regions, ref)
-    uses_tc = "tcgen05" in V.describe(lib.c).split("readout")[0]
-    bf16_before_stats = uses_tc or (cfg.prep_conv and cfg.dtype == "bf16")
-    tol_s = stage_tol if stage_tol is not None else (TOL_STAGE_TC if bf16_before_stats else TOL_STAGE_SIMT)
+    uses_tc = "gram=tcgen05" in V.describe(lib.c)
+    roundings = int(uses_tc) + int(cfg.prep_conv and cfg.dtype == "bf16")
+    tol_s = stage_tol if stage_tol is not None else (
+        TOL_STAGE_PER_ROUNDING * roundings if roundings else TOL_STAGE_SIMT)
     assert err_o <= TOL_O[cfg.dtype], (err_o, stages)
     for k, e in stages.items():
         assert e <= tol_s, (k, e, stages)
