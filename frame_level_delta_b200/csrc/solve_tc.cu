@@ -193,6 +193,7 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
       float g[16];
 #pragma unroll
       for (int c = 0; c < 16; ++c) g[c] = x[c];
+#pragma unroll
       for (int j = 0; j < 16; ++j) {
         const float dj = __shfl_sync(0xffffffffu, g[0], l0 + j);
         const float inv = rsqrtf(dj);
@@ -206,7 +207,9 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
         }
       }
       if (in) {
-        for (int c = r + 1; c < 16; ++c) Lk[r * 16 + c] = 0.f;
+#pragma unroll
+        for (int c = 1; c < 16; ++c)
+          if (c > r) Lk[r * 16 + c] = 0.f;
       }
     }
     __syncthreads();
@@ -217,6 +220,7 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
       if (ri >= k0 + 16) {
 #pragma unroll
         for (int c = 0; c < 16; ++c) pv[c] = 0.f;
+#pragma unroll
         for (int c = 0; c < 16; ++c) {
           const float y = x[0] * Rv[c];
 #pragma unroll
@@ -251,6 +255,7 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
       for (int r = 0; r < 16; ++r) z[r] = Tb[r * D + j];
       __nv_bfloat16* wh = reinterpret_cast<__nv_bfloat16*>(wimg);
       __nv_bfloat16* wl = reinterpret_cast<__nv_bfloat16*>(wimg + kImg);
+#pragma unroll
       for (int r = 0; r < 16; ++r) {
         const float w = z[0] * Rv[r];
 #pragma unroll
