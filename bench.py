@@ -56,6 +56,18 @@ def load_peaks():
 # Algorithmic bytes / flops per launch of each kernel (each input byte read
 # once, each output byte written once).
 # ----------------------------------------------------------------------------
+def composed_chunks(cfg):
+    """Frame counts of the chunk maps the tensor-core scan composes (forward
+    chunks 0..J-3 over frames max(1, c m)..c(m+1)-1, reverse chunks 2..J-1 over
+    c m..min(c(m+1)-1, T-2)); empty when the scan steps over frames directly."""
+    c, T, J = cfg.chunk, cfg.T, cfg.J
+    if c <= 1 or J < 3:
+        return []
+    fwd = [max(0, c * (m + 1) - 1 - max(1, c * m) + 1) for m in range(0, J - 2)]
+    rev = [max(0, min(c * (m + 1) - 1, T - 2) - c * m + 1) for m in range(2, J)]
+    return fwd + rev
+
+
 def kernel_bytes(name: str, cfg) -> float:
     B, H, d, T, U, L, c = cfg.B, cfg.H, cfg.d, cfg.T, cfg.U, cfg.L, cfg.chunk
     esz = 4 if cfg.dtype == "f32" else 2
@@ -68,10 +80,15 @@ def kernel_bytes(name: str, cfg) -> float:
         return BH * (4 * NS * dd4 + F * d * 4)
     if name == "solve_tc":  # A, B read; M, C (fp32) and M's hi/lo operand images written
         return BH * (4 * NS * dd4 + F * dd4 + F * d * 4)
-    if name == "scan_tc":  # per scanned frame: M's hi/lo images + C; S_T; readout states
-        fwd = max(0, c * (J - 2) - 1)
-        rev = max(0, (T - 2) - 2 * c + 1)
-        return BH * ((fwd + rev) * 2 * dd4 + 2 * dd4 + 2 * J * dd4)
+    if name == "scan_tc":  # per step: a (chunk) map's hi/lo images + its C; S_T; readout states
+        if composed_chunks(cfg):
+            steps = 2 * (J - 2)
+        else:
+            steps = max(0, c * (J - 2) - 1) + max(0, (T - 2) - 2 * c + 1)
+        return BH * (steps * 2 * dd4 + 2 * dd4 + 2 * J * dd4)
+    if name == "compose_tc":  # per frame of a composed chunk: M images + C; per chunk: map + C out
+        ch = composed_chunks(cfg)
+        return BH * (sum(ch) * 2 * dd4 + len(ch) * 2 * dd4)
     if name == "scan_simt":
         fwd = max(0, c * (J - 2) - 1)
         rev = max(0, (T - 2) - 2 * c + 1)
@@ -96,6 +113,10 @@ def kernel_flops(name: str, cfg) -> float:
         return B * H * (F * U + L) * 4 * d * d
     if name.startswith("solve"):  # Cholesky d^3/3, L^-1 d^3/3, P d^3/3, C = B P 2 d^3
         return B * H * NS * 3 * d ** 3
+    if name == "compose_tc":  # two d x d x d products per absorbed frame
+        return B * H * sum(max(0, n - 1) for n in composed_chunks(cfg)) * 2 * 2 * d ** 3
+    if name == "scan_tc" and composed_chunks(cfg):
+        return B * H * 2 * (J - 2) * 2 * d ** 3
     if name.startswith("scan"):
         fwd = max(0, c * (J - 2) - 1)
         rev = max(0, (T - 2) - 2 * c + 1)
@@ -137,7 +158,7 @@ def path_flops(cfg) -> float:
 
 def source_digest(kernel: str):
     files = {"gram_tc": "gram_tc.cu", "readout_tc": "readout_tc.cu", "solve_tc": "solve_tc.cu",
-             "scan_tc": "scan_tc.cu"}
+             "scan_tc": "scan_tc.cu", "compose_tc": "compose_tc.cu"}
     fn = files.get(kernel, "kernels_simt.cu")
     p = os.path.join(ROOT, "frame_level_delta_b200", "csrc", fn)
     with open(p, "rb") as f:

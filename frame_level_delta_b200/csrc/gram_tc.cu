@@ -294,15 +294,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t v[16];
           tmem_ld16(taddr + c * 16, v);
           tmem_ld_wait();
-          float* dst = (c < 8 ? a.A : a.Bm) + off + (long long)r * D + (c % 8) * 16;
+          float4* dst = reinterpret_cast<float4*>((c < 8 ? a.A : a.Bm) + off);
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            reinterpret_cast<float4*>(dst)[j] =
+            dst[((c % 8) * 4 + j) * D + r] =
                 make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
                             __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
         }
       } else {
-        float* rowp = (r < 64 ? a.A + off + (long long)r * 64 : a.Bm + off + (long long)(r - 64) * 64);
+        // Rows 0..63 of the stacked accumulator are A_t, rows 64..127 are B_t.
+        float4* dst = reinterpret_cast<float4*>((r < 64 ? a.A : a.Bm) + off);
+        const int rr = r & 63;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t v[16];
@@ -310,7 +312,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            reinterpret_cast<float4*>(rowp + c * 16)[j] =
+            dst[(c * 4 + j) * 64 + rr] =
                 make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
                             __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
         }

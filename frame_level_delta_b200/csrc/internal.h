@@ -42,6 +42,8 @@ struct Problem {
   void* Ktp;    // [B,H,L,D]
   void* Vtp;
   void* Msplit;  // [B,H,T-1] x 2 bf16 d*d images of M_t (hi, lo) for the tensor-core scan
+  void* CMi;     // [B,H,2,J] x 2 bf16 d*d images: composed chunk transitions per direction
+  float* CC;     // [B,H,2,J,D,D]: composed chunk injections per direction
   unsigned long long spin_limit;  // wall-time bound (ns) of every device-side wait
 };
 
@@ -52,6 +54,19 @@ inline __host__ __device__ long long slot_off(const Problem& p, int b, int h, in
 inline __host__ __device__ long long chunk_off(const Problem& p, int b, int h, int j) {
   return (((long long)b * p.H + h) * p.J + j) * (long long)p.D * p.D;
 }
+
+// Every d x d fp32 matrix of the workspace (A_t, B_t, M_t, C_t, the readout
+// states, the composed chunk injections) is stored in column quads: element
+// (i, j) at float index ((j / 4) * d + i) * 4 + j % 4, i.e. float4 number
+// (j / 4) * d + i. Threads that own consecutive rows (the tensor-core epilogues
+// map matrix row i to TMEM lane i) then move 512 contiguous bytes per warp and
+// float4 access instead of touching 32 separate lines.
+inline __host__ __device__ long long quad_off(int D, int i, int j) {
+  return ((long long)(j >> 2) * D + i) * 4 + (j & 3);
+}
+// Row and column of storage index e (0 <= e < d*d) in that layout.
+inline __host__ __device__ int quad_row(int D, int e) { return (e >> 2) % D; }
+inline __host__ __device__ int quad_col(int D, int e) { return ((e >> 2) / D) * 4 + (e & 3); }
 
 // Kernel ids for launch accounting and profiling.
 enum KernelId {
@@ -66,6 +81,7 @@ enum KernelId {
   K_ZERO_ANCHORS,
   K_SOLVE_TC,
   K_SCAN_TC,
+  K_COMPOSE_TC,
   K_NUM_KERNELS
 };
 const char* kernel_name(int id);
@@ -88,7 +104,8 @@ bool readout_tc_supported(const Problem& p);
 bool solve_tc_supported(const Problem& p);
 cudaError_t launch_solve_tc(const Problem& p, cudaStream_t s);
 bool scan_tc_supported(const Problem& p);
-cudaError_t launch_scan_tc(const Problem& p, cudaStream_t s);
+cudaError_t launch_scan_tc(const Problem& p, cudaStream_t s, bool chunked);
+cudaError_t launch_compose_tc(const Problem& p, cudaStream_t s);
 cudaError_t launch_readout_tc(const Problem& p, const void* gate, void* O, cudaStream_t s);
 
 }  // namespace vda

@@ -96,8 +96,8 @@ __global__ void __launch_bounds__(256) gram_simt_kernel(Problem p) {
 #pragma unroll
     for (int c = 0; c < TI; ++c) {
       const int i = ty + 16 * a, j = tx + 16 * c;
-      p.A[off + (long long)i * D + j] = accA[a][c];
-      p.Bm[off + (long long)i * D + j] = accB[a][c];
+      p.A[off + quad_off(D, i, j)] = accA[a][c];
+      p.Bm[off + quad_off(D, i, j)] = accB[a][c];
     }
 }
 
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(256) solve_simt_kernel(Problem p) {
   const long long off = slot_off(p, b, h, s);
   const float* A = p.A + off;
   for (int e = tid; e < D * D; e += nt) {
-    const int i = e / D, j = e % D;
+    const int i = quad_row(D, e), j = quad_col(D, e);
     X[i * LD + j] = A[e] + (i == j ? 1.f : 0.f);
   }
   __syncthreads();
@@ -156,15 +156,15 @@ __global__ void __launch_bounds__(256) solve_simt_kernel(Problem p) {
   if (s > 0) {
     const float* alpha = p.alpha + (((long long)b * p.H + h) * p.T + s) * D;
     for (int e = tid; e < D * D; e += nt) {
-      const int i = e / D, j = e % D;
+      const int i = quad_row(D, e), j = quad_col(D, e);
       p.M[off + e] = alpha[i] * X[i * LD + j];
     }
   }
   const float* Bm = p.Bm + off;
   for (int e = tid; e < D * D; e += nt) {
-    const int i = e / D, j = e % D;
+    const int i = quad_row(D, e), j = quad_col(D, e);
     float acc = 0.f;
-    for (int k = 0; k < D; ++k) acc = fmaf(Bm[i * D + k], X[k * LD + j], acc);
+    for (int k = 0; k < D; ++k) acc = fmaf(Bm[quad_off(D, i, k)], X[k * LD + j], acc);
     p.C[off + e] = acc;
   }
 }
@@ -188,12 +188,12 @@ __global__ void __launch_bounds__(256) scan_simt_kernel(Problem p) {
   float* out = dir == 0 ? p.Sf : p.Sr;
   const int c = p.c, T = p.T, J = p.J;
 #pragma unroll
-  for (int m = 0; m < NC; ++m) sS[r][l + 16 * m] = 0.5f * S_T[(r0 + r) * D + l + 16 * m];
+  for (int m = 0; m < NC; ++m) sS[r][l + 16 * m] = 0.5f * S_T[quad_off(D, r0 + r, l + 16 * m)];
   __syncthreads();
   auto store = [&](int j) {
-    const long long o = chunk_off(p, b, h, j) + (long long)(r0 + r) * D;
+    const long long o = chunk_off(p, b, h, j);
 #pragma unroll
-    for (int m = 0; m < NC; ++m) out[o + l + 16 * m] = sS[r][l + 16 * m];
+    for (int m = 0; m < NC; ++m) out[o + quad_off(D, r0 + r, l + 16 * m)] = sS[r][l + 16 * m];
   };
   for (int j = 0; j < J; ++j)
     if (dir == 0 ? (c * (j - 1) - 1 <= 0) : (c * (j + 2) >= T - 1)) store(j);
@@ -203,15 +203,15 @@ __global__ void __launch_bounds__(256) scan_simt_kernel(Problem p) {
   for (int st = 0; st < nsteps; ++st) {
     const int f = dir == 0 ? f_first + st : f_first - st;
     const float* Mf = p.M + slot_off(p, b, h, f);
-    const float* Cf = p.C + slot_off(p, b, h, f) + (long long)(r0 + r) * D;
+    const float* Cf = p.C + slot_off(p, b, h, f);
     float acc[NC];
 #pragma unroll
-    for (int m = 0; m < NC; ++m) acc[m] = Cf[l + 16 * m];
+    for (int m = 0; m < NC; ++m) acc[m] = Cf[quad_off(D, r0 + r, l + 16 * m)];
 #pragma unroll 4
     for (int k = 0; k < D; ++k) {
       const float sv = sS[r][k];
 #pragma unroll
-      for (int m = 0; m < NC; ++m) acc[m] = fmaf(sv, Mf[k * D + l + 16 * m], acc[m]);
+      for (int m = 0; m < NC; ++m) acc[m] = fmaf(sv, Mf[quad_off(D, k, l + 16 * m)], acc[m]);
     }
     __syncthreads();
 #pragma unroll
@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(256) readout_simt_kernel(Problem p, const void
   const int ntok = (int)min((long long)TT, tok_hi - tok0);
   const long long co = chunk_off(p, b, h, j);
   for (int e = threadIdx.x; e < D * D; e += blockDim.x)
-    sS[(e / D) * LD + e % D] = p.Sf[co + e] + p.Sr[co + e];
+    sS[quad_row(D, e) * LD + quad_col(D, e)] = p.Sf[co + e] + p.Sr[co + e];
   const long long rowstride = (long long)p.H * D;
   const long long qbase = ((long long)b * p.T * p.U) * rowstride + (long long)h * D;
   for (int e = threadIdx.x; e < TT * D; e += blockDim.x) {

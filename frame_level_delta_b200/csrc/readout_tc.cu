@@ -260,12 +260,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // The MMAs of the previous tile are complete (its accumulator was read
         // below) and the next MMA waits for `sready`: S may be overwritten.
         const long long off = ((long long)ti.bh * a.J + ti.j) * (long long)D * D;
+        const float4* pf = reinterpret_cast<const float4*>(a.Sf + off);
+        const float4* pr = reinterpret_cast<const float4*>(a.Sr + off);
         for (int e = et; e < D * (D / 8); e += 128) {
-          const int i = e / (D / 8), c8 = e % (D / 8);  // row i, 8 consecutive k
-          const float4* pf = reinterpret_cast<const float4*>(a.Sf + off + (long long)i * D + c8 * 8);
-          const float4* pr = reinterpret_cast<const float4*>(a.Sr + off + (long long)i * D + c8 * 8);
+          const int c8 = e / D, i = e % D;  // row i, 8 consecutive k (column quads 2 c8, 2 c8 + 1)
           float x[8];
-          const float4 f0 = pf[0], f1 = pf[1], r0 = pr[0], r1 = pr[1];
+          const float4 f0 = pf[(2 * c8) * D + i], f1 = pf[(2 * c8 + 1) * D + i];
+          const float4 r0 = pr[(2 * c8) * D + i], r1 = pr[(2 * c8 + 1) * D + i];
           x[0] = f0.x + r0.x; x[1] = f0.y + r0.y; x[2] = f0.z + r0.z; x[3] = f0.w + r0.w;
           x[4] = f1.x + r1.x; x[5] = f1.y + r1.y; x[6] = f1.z + r1.z; x[7] = f1.w + r1.w;
           uint4 hv, lv;

@@ -2,7 +2,8 @@
 // onedev.kr/papers/80, section "how it works": a forward and a reverse state,
 // both started at S_T/2; section "how to use": S_t = S_{t-1} M_t + C_t).
 //
-// One CTA per (b, h, direction) runs the recurrence frame by frame:
+// One CTA per (b, h, direction) runs the recurrence frame by frame, or chunk by
+// chunk over the maps the composition kernel formed (same step, same operands):
 //   S <- S M_t + C_t,  S = Sh + Sl, M_t = Mh + Ml (bf16 parts, ~2^-16 relative),
 //   S M_t ~= Sh Mh + Sh Ml + Sl Mh  (24 MMAs of 128x128x16, fp32 in TMEM).
 // The fp32 state is rebuilt every step from TMEM plus C_t in the epilogue
@@ -32,8 +33,11 @@ constexpr uint32_t kIdesc = sm100::idesc_bf16_f32(128, 128, false, true);  // A 
 
 struct ScanArgs {
   int B, H, T, c, J;
+  int chunked;        // 1: step over composed chunk maps, 0: over frames
   const float* C;     // [B,H,T-1,D,D]; slot 0 = S_T
   const uint8_t* Mi;  // [B,H,T-1] x (hi, lo) operand images
+  const uint8_t* CMi; // [B,H,2,J] x (hi, lo) composed chunk transitions
+  const float* CC;    // [B,H,2,J,D,D] composed chunk injections
   float* Sf;
   float* Sr;
   uint32_t* status;
@@ -84,8 +88,18 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
   const int c = a.c, T = a.T, J = a.J;
   const int f_first = dir == 0 ? 1 : T - 2;
   const int f_last = dir == 0 ? c * (J - 2) - 1 : 2 * c;
-  const int nsteps = max(0, dir == 0 ? f_last - f_first + 1 : f_first - f_last + 1);
+  const int nsteps = a.chunked ? max(0, J - 2) : max(0, dir == 0 ? f_last - f_first + 1 : f_first - f_last + 1);
   const long long slots = (long long)bh * (T - 1);
+  // Step st absorbs frame f(st), or chunk m(st) (forward m = st, reverse m = J-1-st),
+  // whose transition image and injection rows are:
+  auto step_img = [&](int st) -> const uint8_t* {
+    if (a.chunked) return a.CMi + (((long long)bh * 2 + dir) * J + (dir == 0 ? st : J - 1 - st)) * (long long)kMBuf;
+    return a.Mi + (slots + (dir == 0 ? f_first + st : f_first - st)) * (long long)kMBuf;
+  };
+  auto step_c = [&](int st) -> const float* {
+    if (a.chunked) return a.CC + (((long long)bh * 2 + dir) * J + (dir == 0 ? st : J - 1 - st)) * (long long)D * D;
+    return a.C + (slots + (dir == 0 ? f_first + st : f_first - st)) * (long long)D * D;
+  };
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -113,9 +127,8 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
       for (int st = 0; st < nsteps; ++st) {
         const int s = st & 1;
         if (!mbar_wait(&mempty[s], ((st >> 1) & 1) ^ 1, abort_flag, a.status, a.wait_ns)) break;
-        const int f = dir == 0 ? f_first + st : f_first - st;
         mbar_arrive_expect_tx(&mfull[s], kMBuf);
-        const uint8_t* src = a.Mi + (slots + f) * (long long)kMBuf;
+        const uint8_t* src = step_img(st);
         bulk_load(sM + s * kMBuf, src, kImg, &mfull[s]);
         bulk_load(sM + s * kMBuf + kImg, src + kImg, kImg, &mfull[s]);
         issued = st + 1;
@@ -149,19 +162,20 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
     const int i = q * 32 + lane;  // state row == TMEM lane
     float* out = dir == 0 ? a.Sf : a.Sr;
     auto store_row = [&](int j, const float* x, int col0, int n) {
-      float4* d4 = reinterpret_cast<float4*>(out + ((long long)bh * J + j) * D * D + (long long)i * D + col0);
-      for (int t = 0; t < n / 4; ++t) d4[t] = make_float4(x[4 * t], x[4 * t + 1], x[4 * t + 2], x[4 * t + 3]);
+      float4* d4 = reinterpret_cast<float4*>(out + ((long long)bh * J + j) * D * D);
+      for (int t = 0; t < n / 4; ++t)
+        d4[(col0 / 4 + t) * D + i] = make_float4(x[4 * t], x[4 * t + 1], x[4 * t + 2], x[4 * t + 3]);
     };
     // Initial state S_T / 2: readout states of the chunks that see no frame of
     // this direction, and the first operand image.
     {
-      const float* st0 = a.C + slots * (long long)D * D + (long long)i * D;
+      const float4* st0 = reinterpret_cast<const float4*>(a.C + slots * (long long)D * D);
 #pragma unroll 1
       for (int c16 = 0; c16 < D / 16; ++c16) {
         float x[16];
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-          const float4 v = reinterpret_cast<const float4*>(st0 + c16 * 16)[t];
+          const float4 v = st0[(c16 * 4 + t) * D + i];
           x[4 * t] = 0.5f * v.x; x[4 * t + 1] = 0.5f * v.y; x[4 * t + 2] = 0.5f * v.z; x[4 * t + 3] = 0.5f * v.w;
         }
         for (int j = 0; j < J; ++j)
@@ -181,18 +195,20 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
     }
     for (int st = 0; st < nsteps; ++st) {
       const int f = dir == 0 ? f_first + st : f_first - st;
-      // Prefetch C_f row i while the MMAs run.
+      // Prefetch the injection's row i while the MMAs run.
       float crow[D];
-      const float4* csrc = reinterpret_cast<const float4*>(a.C + (slots + f) * (long long)D * D + (long long)i * D);
+      const float4* csrc = reinterpret_cast<const float4*>(step_c(st));
 #pragma unroll
       for (int t = 0; t < D / 4; ++t) {
-        const float4 v = csrc[t];
+        const float4 v = csrc[t * D + i];
         crow[4 * t] = v.x; crow[4 * t + 1] = v.y; crow[4 * t + 2] = v.z; crow[4 * t + 3] = v.w;
       }
       if (!mbar_wait(tfull, st & 1, abort_flag, a.status, a.wait_ns)) break;
       tc_fence_after();
       int jout = -1;
-      if (dir == 0) {
+      if (a.chunked) {
+        jout = dir == 0 ? st + 2 : (J - 1 - st) - 2;  // after chunk m: readout state of chunk m+2 / m-2
+      } else if (dir == 0) {
         if ((f + 1) % c == 0 && (f + 1) / c + 1 < J) jout = (f + 1) / c + 1;
       } else {
         if (f % c == 0 && f / c - 2 >= 0) jout = f / c - 2;
@@ -243,15 +259,15 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
 
 bool scan_tc_supported(const Problem& p) { return solve_tc_supported(p); }
 
-cudaError_t launch_scan_tc(const Problem& p, cudaStream_t s) {
+cudaError_t launch_scan_tc(const Problem& p, cudaStream_t s, bool chunked) {
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  ScanArgs a{p.B, p.H, p.T, p.c, p.J, p.C, static_cast<const uint8_t*>(p.Msplit), p.Sf, p.Sr, p.status,
-             p.spin_limit};
+  ScanArgs a{p.B, p.H, p.T, p.c, p.J, chunked ? 1 : 0, p.C, static_cast<const uint8_t*>(p.Msplit),
+             static_cast<const uint8_t*>(p.CMi), p.CC, p.Sf, p.Sr, p.status, p.spin_limit};
   dim3 grid(p.B * p.H, 2);
   scan_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(a);
   return cudaGetLastError();

@@ -128,10 +128,10 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
   // X = I + A into TMEM columns 0..127 and R = I into 128..255 (this thread: row
   // ri, columns hc*64 .. hc*64+63). All sixteen loads are issued before use.
   {
-    const float4* src = reinterpret_cast<const float4*>(a.A + off + (long long)ri * D + hc * 64);
+    const float4* src = reinterpret_cast<const float4*>(a.A + off);
     float4 v[16];
 #pragma unroll
-    for (int t = 0; t < 16; ++t) v[t] = src[t];
+    for (int t = 0; t < 16; ++t) v[t] = src[(hc * 16 + t) * D + ri];
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       uint32_t x[16], r[16];
@@ -304,10 +304,10 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
   ++commits;
   // B_t (row ri, columns hc*64..) -> TMEM columns 128.. as hi | lo bf16 pairs, while P runs.
   {
-    const float4* src = reinterpret_cast<const float4*>(a.Bm + off + (long long)ri * D + hc * 64);
+    const float4* src = reinterpret_cast<const float4*>(a.Bm + off);
     float4 v[16];
 #pragma unroll
-    for (int t = 0; t < 16; ++t) v[t] = src[t];
+    for (int t = 0; t < 16; ++t) v[t] = src[(hc * 16 + t) * D + ri];
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       uint32_t ph[16], pl[16];
@@ -365,9 +365,9 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
         }
       }
       if (slot > 0) {
-        float4* md = reinterpret_cast<float4*>(a.M + off + (long long)ri * D + j0);
+        float4* md = reinterpret_cast<float4*>(a.M + off);
 #pragma unroll
-        for (int t = 0; t < 4; ++t) md[t] = make_float4(mv[4 * t], mv[4 * t + 1], mv[4 * t + 2], mv[4 * t + 3]);
+        for (int t = 0; t < 4; ++t) md[(j0 / 4 + t) * D + ri] = make_float4(mv[4 * t], mv[4 * t + 1], mv[4 * t + 2], mv[4 * t + 3]);
       }
     }
   }
@@ -399,10 +399,10 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
       uint32_t v[16];
       tmem_ld16(tl + kAccX + j0, v);
       tmem_ld_wait();
-      float4* cd = reinterpret_cast<float4*>(a.C + off + (long long)ri * D + j0);
+      float4* cd = reinterpret_cast<float4*>(a.C + off);
 #pragma unroll
       for (int t = 0; t < 4; ++t)
-        cd[t] = make_float4(__uint_as_float(v[4 * t]), __uint_as_float(v[4 * t + 1]), __uint_as_float(v[4 * t + 2]),
+        cd[(j0 / 4 + t) * D + ri] = make_float4(__uint_as_float(v[4 * t]), __uint_as_float(v[4 * t + 1]), __uint_as_float(v[4 * t + 2]),
                             __uint_as_float(v[4 * t + 3]));
     }
   }

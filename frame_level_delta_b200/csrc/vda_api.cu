@@ -15,7 +15,7 @@ namespace vda {
 const char* kernel_name(int id) {
   static const char* names[K_NUM_KERNELS] = {
       "prep_video", "prep_text", "gram_simt", "gram_tc", "solve_simt",
-      "scan_simt", "readout_simt", "readout_tc", "zero_anchors", "solve_tc", "scan_tc"};
+      "scan_simt", "readout_simt", "readout_tc", "zero_anchors", "solve_tc", "scan_tc", "compose_tc"};
   return (id >= 0 && id < K_NUM_KERNELS) ? names[id] : "?";
 }
 
@@ -105,6 +105,8 @@ Layout make_layout(const vda_config& c) {
   L.bytes[VDA_REGION_KT_PREP] = prep ? BH * c.L * d * esz : 0;
   L.bytes[VDA_REGION_VT_PREP] = prep ? BH * c.L * d * esz : 0;
   L.bytes[VDA_REGION_M_SPLIT] = BH * (c.T - 1) * 2 * d * d * 2;
+  L.bytes[VDA_REGION_CHUNK_M] = BH * 2 * J_of(c) * 2 * d * d * 2;
+  L.bytes[VDA_REGION_CHUNK_C] = BH * 2 * J_of(c) * d * d * 4;
   size_t o = 0;
   for (int r = 0; r < VDA_NUM_REGIONS; ++r) {
     L.off[r] = o;
@@ -291,6 +293,8 @@ vda_status vda_prepare(vda_ctx* ctx, const void* Q, const void* K, const void* V
   p.Sf = reinterpret_cast<float*>(ws + L.off[VDA_REGION_S_FWD]);
   p.Sr = reinterpret_cast<float*>(ws + L.off[VDA_REGION_S_REV]);
   p.Msplit = ws + L.off[VDA_REGION_M_SPLIT];
+  p.CMi = ws + L.off[VDA_REGION_CHUNK_M];
+  p.CC = reinterpret_cast<float*>(ws + L.off[VDA_REGION_CHUNK_C]);
   p.spin_limit = 2000000000ull;  // 2 s of wall time per device-side wait
   const long long D = p.D, H = p.H, T = p.T, U = p.U, Lt = p.L;
   if (prep) {
@@ -337,9 +341,16 @@ vda_status vda_scan_bidir(vda_ctx* ctx, void* stream) {
   if (!ctx->prepared) return fail(ctx, VDA_ERR_STATE, "vda_scan_bidir before a successful vda_prepare");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   vda_status st;
-  if (!use_simt_only(ctx->cfg) && scan_tc_supported(ctx->p))
-    st = run_kernel(ctx, K_SCAN_TC, s, [&] { return launch_scan_tc(ctx->p, s); });
-  else
+  if (!use_simt_only(ctx->cfg) && scan_tc_supported(ctx->p)) {
+    // Compose each chunk's frame maps in parallel, then scan the chunks; with
+    // single-frame chunks composition is a copy, so scan the frames directly.
+    const bool chunked = ctx->p.c > 1 && ctx->p.J >= 3;
+    if (chunked) {
+      st = run_kernel(ctx, K_COMPOSE_TC, s, [&] { return launch_compose_tc(ctx->p, s); });
+      if (st != VDA_OK) return st;
+    }
+    st = run_kernel(ctx, K_SCAN_TC, s, [&] { return launch_scan_tc(ctx->p, s, chunked); });
+  } else
     st = run_kernel(ctx, K_SCAN_SIMT, s, [&] { return launch_scan_simt(ctx->p, s); });
   if (st != VDA_OK) return st;
   ctx->scanned = true;

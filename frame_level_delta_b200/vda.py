@@ -24,7 +24,8 @@ VDA_PREP_CONV = 0x1
 VDA_READOUT_NORM_GATE = 0x2
 VDA_FORCE_SIMT = 0x100
 REGIONS = {"status": 0, "A": 1, "B": 2, "M": 3, "C": 4, "S_fwd": 5, "S_rev": 6,
-           "K_prep": 7, "V_prep": 8, "Kt_prep": 9, "Vt_prep": 10, "M_split": 11}
+           "K_prep": 7, "V_prep": 8, "Kt_prep": 9, "Vt_prep": 10, "M_split": 11,
+           "chunk_M": 12, "chunk_C": 13}
 
 # Exported symbols, in the order include/vda.h declares them.
 EXPORTS = ["vda_create", "vda_destroy", "vda_workspace_size", "vda_prepare", "vda_scan_bidir",
@@ -201,11 +202,15 @@ class VDA:
         cfg = self.cfg
         D, BH = cfg.d, cfg.B * cfg.H
         if name in ("A", "B", "M", "C"):
-            return raw.view(torch.float32).view(cfg.B, cfg.H, cfg.T - 1, D, D)
+            return _from_quads(raw, (cfg.B, cfg.H, cfg.T - 1), D)
         if name in ("S_fwd", "S_rev"):
-            return raw.view(torch.float32).view(cfg.B, cfg.H, cfg.J, D, D)
+            return _from_quads(raw, (cfg.B, cfg.H, cfg.J), D)
         if name == "status":
             return raw.view(torch.int32)
+        if name == "chunk_C":
+            return _from_quads(raw, (cfg.B, cfg.H, 2, cfg.J), D)
+        if name in ("M_split", "chunk_M"):  # bf16 hi/lo operand images, raw bytes
+            return raw
         dt = torch.float32 if cfg.dtype == "f32" else torch.bfloat16
         if name in ("K_prep", "V_prep"):
             return raw.view(dt).view(cfg.B, cfg.H, cfg.T, cfg.U, D)
@@ -229,6 +234,13 @@ class VDA:
         n = ctypes.c_uint64(0)
         self._check(lib().vda_launch_count(self._ctx, ctypes.byref(n)), "vda_launch_count")
         return n.value
+
+
+def _from_quads(raw: torch.Tensor, lead: tuple, D: int) -> torch.Tensor:
+    """Row-major (..., D, D) copy of fp32 d x d matrices stored in column quads
+    (element (i, j) at float ((j // 4) * D + i) * 4 + j % 4)."""
+    q = raw.view(torch.float32).view(*lead, D // 4, D, 4)
+    return q.movedim(-3, -2).reshape(*lead, D, D)
 
 
 def run_static_workspace(cfg: VDAConfig, inp: Dict[str, torch.Tensor], O: torch.Tensor, stream=None) -> int:

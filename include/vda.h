@@ -149,7 +149,13 @@ vda_status vda_readout(vda_ctx* ctx, const void* gate, void* O, void* stream);
  */
 vda_status vda_poll_device_status(vda_ctx* ctx, void* stream);
 
-/* Regions of the workspace, for staged parity checks and debugging. */
+/*
+ * Regions of the workspace, for staged parity checks and debugging. Every
+ * float32 d x d matrix below (one per slot, chunk or direction) is stored in
+ * column quads: element (i, j) at float index ((j / 4) * d + i) * 4 + j % 4 of
+ * its matrix, so that threads owning consecutive rows access contiguous
+ * memory. The shapes name the logical indices, outermost first.
+ */
 typedef enum vda_region {
   VDA_REGION_STATUS = 0, /* uint32 device status word (+ padding) */
   VDA_REGION_A = 1,      /* float32 [B, H, T-1, d_k, d_k]; slot 0 = text, slot t = frame t */
@@ -165,7 +171,10 @@ typedef enum vda_region {
   VDA_REGION_M_SPLIT = 11, /* bf16 [B, H, T-1, 2, d*d]: M_t as hi + lo parts (M = hi + lo to ~2^-16),
                               each in the swizzled shared-memory operand layout of the tensor-core
                               scan (used when that scan runs, unused otherwise) */
-  VDA_NUM_REGIONS = 12
+  VDA_REGION_CHUNK_M = 12, /* bf16 [B, H, 2, J, 2, d*d]: per direction and chunk, the composed transition
+                              of the chunk's frames (hi, lo operand images; identity for empty chunks) */
+  VDA_REGION_CHUNK_C = 13, /* float32 [B, H, 2, J, d_v, d_k]: the composed injection of those frames */
+  VDA_NUM_REGIONS = 14
 } vda_region;
 
 /* Byte offset and size of a region inside the workspace (size 0 if unused). Host-only. */

@@ -130,3 +130,17 @@ def test_status_strings_and_describe():
     assert "gram=" in text and "readout=" in text
     assert "tcgen05" not in text  # fp32 storage always takes the CUDA-core path
     assert "tcgen05" not in V.describe(V.make_config(CONFIGS["h3"], force_simt=True))
+
+
+def test_region_view_undoes_column_quad_layout():
+    """Workspace matrices are stored in column quads: element (i, j) at float
+    ((j // 4) * d + i) * 4 + j % 4. The region view must return row-major."""
+    import torch
+    from frame_level_delta_b200.vda import _from_quads
+    D = 16
+    raw = torch.arange(2 * D * D, dtype=torch.float32).view(torch.uint8)
+    m = _from_quads(raw, (2,), D)
+    for s in range(2):
+        for i in range(D):
+            for j in range(D):
+                assert m[s, i, j] == s * D * D + ((j // 4) * D + i) * 4 + j % 4

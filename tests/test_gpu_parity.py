@@ -113,6 +113,27 @@ def test_edge_cases(name, kw, dtype):
     check_config(cfg)
 
 
+# Chunk structures of the tensor-core scan (d = 128, bf16): composed chunk maps
+# with one frame (a copy), none (the identity), a ragged last chunk, the
+# smallest clip that has a composed chunk, and single-frame chunks (no
+# composition: the scan steps over frames).
+EDGE_CHUNKS = [
+    ("d128_ragged_last_chunk", dict(T=23, chunk=5)),
+    ("d128_last_chunk_anchor_only", dict(T=13, chunk=4)),
+    ("d128_two_frame_chunks", dict(T=12, chunk=2)),
+    ("d128_three_chunks", dict(T=8, chunk=3)),
+    ("d128_chunk_one", dict(T=9, chunk=1)),
+    ("d128_wide_chunks", dict(T=20, chunk=8)),
+    ("d128_batch_two", dict(B=2, T=11, chunk=3)),
+]
+
+
+@pytest.mark.parametrize("name,kw", EDGE_CHUNKS, ids=[e[0] for e in EDGE_CHUNKS])
+def test_edge_chunk_structures_tensor_core_scan(name, kw):
+    cfg = CONFIGS["small"].with_(name=name, d=128, H=2, grid_h=4, grid_w=5, L=9, **kw)
+    check_config(cfg)
+
+
 def test_edge_conv_gate_small():
     cfg = CONFIGS["hires"].with_(H=2, d=64, T=9, grid_h=6, grid_w=7, L=5, chunk=2)
     check_config(cfg)
