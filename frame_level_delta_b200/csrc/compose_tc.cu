@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(kThreads, 1) compose_tc_kernel(const ComposeAr
   }
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = sm100::align_smem_1024(smem_raw);
   uint8_t* sMM = smem + kMMOff;
   uint8_t* sJJ = smem + kJJOff;
   uint8_t* sMf = smem + kMfOff;

@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   using C = GramCfg<D>;
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = sm100::align_smem_1024(smem_raw);
   uint8_t* bkring = smem + C::kStages * C::kStageBytes;  // beta*K slots
   float* sbeta = reinterpret_cast<float*>(bkring + C::kBkSlots * C::kBkBytes);  // [kStages][kTileU]
   uint64_t* full = reinterpret_cast<uint64_t*>(sbeta + C::kStages * kTileU);

@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kStages = C::kStages;
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = sm100::align_smem_1024(smem_raw);
   uint8_t* sShi = smem;
   uint8_t* sSlo = smem + C::kSBytes;
   uint8_t* sQ = smem + 2 * C::kSBytes;  // stage s: Q tile at s * kStageBytes, gate tile after it

@@ -72,7 +72,7 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = sm100::align_smem_1024(smem_raw);
   uint8_t* sM = smem;           // [2][hi, lo]
   uint8_t* sS = smem + kSOff;   // [hi, lo]
   uint64_t* mfull = reinterpret_cast<uint64_t*>(smem + kBarOff);

@@ -19,6 +19,14 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The dynamic shared-memory array advanced to the next 1024-byte boundary by
+// pointer arithmetic on the array itself, so the compiler still knows the
+// result points into shared memory and emits shared (not generic) loads and
+// stores through it. Dynamic allocations must reserve 1024 bytes of slack.
+__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* raw) {
+  return raw + ((1024u - (smem_u32(raw) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
