@@ -78,7 +78,7 @@ def kernel_bytes(name: str, cfg) -> float:
         return BH * ((F * U + L) * (2 * d * esz + 4) + 2 * NS * dd4)
     if name == "solve_simt":
         return BH * (4 * NS * dd4 + F * d * 4)
-    if name == "solve_tc":  # A, B read; M, C (fp32) and M's hi/lo operand images written
+    if name in ("solve_tc", "solve_chol_tc"):  # A, B read; M, C (fp32) and M's hi/lo operand images written
         return BH * (4 * NS * dd4 + F * dd4 + F * d * 4)
     if name == "scan_tc":  # per step: a (chunk) map's hi/lo images + its C; S_T; readout states
         if composed_chunks(cfg):
@@ -128,7 +128,7 @@ def kernel_flops(name: str, cfg) -> float:
 
 # Kernels whose time is set by dense contractions and their serial dependencies
 # rather than by HBM streaming: their roofline is the bf16 tensor peak.
-TENSOR_BOUND = ("solve_tc", "solve_simt")
+TENSOR_BOUND = ("solve_tc", "solve_chol_tc", "solve_simt")
 
 
 def path_bytes(cfg) -> float:
@@ -158,7 +158,7 @@ def path_flops(cfg) -> float:
 
 def source_digest(kernel: str):
     files = {"gram_tc": "gram_tc.cu", "readout_tc": "readout_tc.cu", "solve_tc": "solve_tc.cu",
-             "scan_tc": "scan_tc.cu", "compose_tc": "compose_tc.cu"}
+             "scan_tc": "scan_tc.cu", "compose_tc": "compose_tc.cu", "solve_chol_tc": "solve_chol_tc.cu"}
     fn = files.get(kernel, "kernels_simt.cu")
     p = os.path.join(ROOT, "frame_level_delta_b200", "csrc", fn)
     with open(p, "rb") as f:
@@ -334,6 +334,8 @@ def main():
     ap.add_argument("--impl", default="vda", choices=["vda", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work (0: skip)")
+    ap.add_argument("--solve", default="sweep", choices=["sweep", "cholesky"],
+                    help="tensor-core frame solve: symmetric sweep (default) or blocked Cholesky")
     ap.add_argument("--heads", type=int, default=0,
                     help="override H (a smaller case of the same workload, e.g. for profiler captures)")
     args = ap.parse_args()
@@ -364,7 +366,7 @@ def main():
     inp_cpu = make_inputs(cfg, seed=cfg.seed + rank)
     inp_host = {k: v.pin_memory() for k, v in inp_cpu.items()}
     inp_dev = {k: v.to(dev, non_blocking=True) for k, v in inp_host.items()}
-    lib = V.VDA(cfg, device=dev)
+    lib = V.VDA(cfg, device=dev, cholesky=args.solve == "cholesky")
     O = lib.new_output()
     stream = torch.cuda.current_stream(dev)
     for _ in range(args.warmup):

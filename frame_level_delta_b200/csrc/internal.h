@@ -82,6 +82,7 @@ enum KernelId {
   K_SOLVE_TC,
   K_SCAN_TC,
   K_COMPOSE_TC,
+  K_SOLVE_CHOL_TC,
   K_NUM_KERNELS
 };
 const char* kernel_name(int id);
@@ -103,6 +104,7 @@ cudaError_t launch_gram_tc(const Problem& p, cudaStream_t s);
 bool readout_tc_supported(const Problem& p);
 bool solve_tc_supported(const Problem& p);
 cudaError_t launch_solve_tc(const Problem& p, cudaStream_t s);
+cudaError_t launch_solve_chol_tc(const Problem& p, cudaStream_t s);
 bool scan_tc_supported(const Problem& p);
 cudaError_t launch_scan_tc(const Problem& p, cudaStream_t s, bool chunked);
 cudaError_t launch_compose_tc(const Problem& p, cudaStream_t s);

@@ -15,7 +15,8 @@ namespace vda {
 const char* kernel_name(int id) {
   static const char* names[K_NUM_KERNELS] = {
       "prep_video", "prep_text", "gram_simt", "gram_tc", "solve_simt",
-      "scan_simt", "readout_simt", "readout_tc", "zero_anchors", "solve_tc", "scan_tc", "compose_tc"};
+      "scan_simt", "readout_simt", "readout_tc", "zero_anchors", "solve_tc", "scan_tc", "compose_tc",
+      "solve_chol_tc"};
   return (id >= 0 && id < K_NUM_KERNELS) ? names[id] : "?";
 }
 
@@ -63,7 +64,8 @@ vda_status check_config(const vda_config* c, std::string* why) {
   if (c->chunk < 1) return bad("chunk must be >= 1");
   if (c->dtype != VDA_F32 && c->dtype != VDA_BF16) return bad("dtype must be VDA_F32 or VDA_BF16");
   if (!(c->l2_eps >= 0.f) || !(c->rms_eps >= 0.f)) return bad("eps must be >= 0");
-  if (c->flags & ~(VDA_PREP_CONV | VDA_READOUT_NORM_GATE | VDA_FORCE_SIMT)) return bad("unknown flag bits");
+  if (c->flags & ~(VDA_PREP_CONV | VDA_READOUT_NORM_GATE | VDA_SOLVE_CHOLESKY | VDA_FORCE_SIMT))
+    return bad("unknown flag bits");
   if (c->d_k != c->d_v) {
     if (why) *why = "d_k != d_v is not supported";
     return VDA_ERR_UNSUPPORTED;
@@ -249,10 +251,11 @@ vda_status vda_describe(const vda_config* cfg, const char** text) {
   const bool simt = use_simt_only(*cfg);
   const bool g = !simt && gram_tc_supported(p), r = !simt && readout_tc_supported(p);
   const bool v = !simt && solve_tc_supported(p), n = !simt && scan_tc_supported(p);
-  static char table[2][2][2][2][80];
-  char* t = table[g][v][n][r];
-  std::snprintf(t, 80, "gram=%s solve=%s scan=%s readout=%s", g ? "tcgen05" : "simt", v ? "tcgen05" : "simt",
-                n ? "tcgen05" : "simt", r ? "tcgen05" : "simt");
+  const bool chol = v && (cfg->flags & VDA_SOLVE_CHOLESKY);
+  static char table[2][2][2][2][2][96];
+  char* t = table[g][v][chol][n][r];
+  std::snprintf(t, 96, "gram=%s solve=%s scan=%s readout=%s", g ? "tcgen05" : "simt",
+                v ? (chol ? "tcgen05-cholesky" : "tcgen05") : "simt", n ? "tcgen05" : "simt", r ? "tcgen05" : "simt");
   *text = t;
   return VDA_OK;
 }
@@ -327,7 +330,9 @@ vda_status vda_prepare(vda_ctx* ctx, const void* Q, const void* K, const void* V
   else
     st = run_kernel(ctx, K_GRAM_SIMT, s, [&] { return launch_gram_simt(p, s); });
   if (st != VDA_OK) return st;
-  if (!use_simt_only(c) && solve_tc_supported(p))
+  if (!use_simt_only(c) && solve_tc_supported(p) && (c.flags & VDA_SOLVE_CHOLESKY))
+    st = run_kernel(ctx, K_SOLVE_CHOL_TC, s, [&] { return launch_solve_chol_tc(p, s); });
+  else if (!use_simt_only(c) && solve_tc_supported(p))
     st = run_kernel(ctx, K_SOLVE_TC, s, [&] { return launch_solve_tc(p, s); });
   else
     st = run_kernel(ctx, K_SOLVE_SIMT, s, [&] { return launch_solve_simt(p, s); });

@@ -72,6 +72,9 @@ typedef enum vda_dtype {
                                       cross-correlation (zero padding, no bias) then SiLU; text K, V:
                                       SiLU; then K, K_txt and Q divided by sqrt(|x|^2 + l2_eps) */
 #define VDA_READOUT_NORM_GATE 0x2u /* o <- o / sqrt(mean(o^2) + rms_eps) * sigmoid(gate) */
+#define VDA_SOLVE_CHOLESKY 0x4u    /* tensor-core frame solve by blocked Cholesky of I + A_t and
+                                      the triangular inverse, instead of the default symmetric
+                                      sweep (Gauss-Jordan) in registers; the same M_t and C_t */
 #define VDA_FORCE_SIMT 0x100u      /* run the generic CUDA-core kernels even where a tensor-core
                                       kernel exists (diagnostics and cross-checks) */
 

@@ -31,10 +31,10 @@ def rel_fro(a, b) -> float:
     return float(np.linalg.norm(a - b) / (nb if nb > 0 else 1.0))
 
 
-def run_gpu(cfg, inp_cpu, force_simt=False):
+def run_gpu(cfg, inp_cpu, force_simt=False, cholesky=False):
     dev = torch.device("cuda:0")
     inp = {k: v.to(dev) for k, v in inp_cpu.items()}
-    lib = V.VDA(cfg, force_simt=force_simt, device=dev)
+    lib = V.VDA(cfg, force_simt=force_simt, device=dev, cholesky=cholesky)
     O = lib.run(inp)
     torch.cuda.synchronize()
     assert lib.poll_device_status() == 0
@@ -66,11 +66,13 @@ def staged_errors(cfg, regions, ref):
     return worst
 
 
-def check_config(cfg, heads=None, force_simt=False, inp=None, stage_tol=None):
+def check_config(cfg, heads=None, force_simt=False, inp=None, stage_tol=None, cholesky=False):
     """Run both sides and assert the bounds. Returns (O error, staged errors)."""
     if inp is None:
         inp = make_inputs(cfg)
-    O_gpu, regions, lib = run_gpu(cfg, inp, force_simt=force_simt)
+    O_gpu, regions, lib = run_gpu(cfg, inp, force_simt=force_simt, cholesky=cholesky)
+    if cholesky and not force_simt and cfg.dtype == "bf16" and cfg.d == 128:
+        assert "solve=tcgen05-cholesky" in V.describe(lib.c)
     ref = vo.vda_reference(inp, cfg, heads=heads)
     hs = sorted({h for (_, h) in ref["heads"]})
     bs = sorted({b for (b, _) in ref["heads"]})
