@@ -95,7 +95,8 @@ def kernel_bytes(name: str, cfg) -> float:
         return BH * ((fwd + rev) * 2 * dd4 + 2 * dd4 + 2 * J * dd4)
     if name in ("readout_tc", "readout_simt"):
         gate = 1 if cfg.norm_gate else 0
-        return BH * (F * U * d * esz * (2 + gate) + 2 * J * dd4)
+        zeros = 2 * U * d * esz if name == "readout_tc" else 0  # the tensor-core readout zeroes the anchors
+        return BH * (F * U * d * esz * (2 + gate) + 2 * J * dd4 + zeros)
     if name == "zero_anchors":
         return BH * 2 * U * d * esz
     if name == "prep_video":

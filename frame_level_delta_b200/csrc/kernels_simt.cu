@@ -295,18 +295,17 @@ __global__ void __launch_bounds__(256) readout_simt_kernel(Problem p, const void
 
 // Anchor frames 0 and T-1 read out exactly zero: for each batch element both
 // frames are contiguous ranges of U*H*D elements of O.
+// Grid (x, 2 * B): blockIdx.y names one contiguous slab (batch b, anchor frame
+// 0 or T-1) of U * H * D values; the x blocks stride over its 16-byte words.
 __global__ void zero_anchors_kernel(Problem p, void* O) {
   const long long per = (long long)p.U * p.H * p.D;
   const int esz = p.bf16 ? 2 : 4;
   const long long words = per * esz / 16;  // per is a multiple of 16 (D >= 16)
-  const long long total = words * 2 * p.B;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const long long w = i % words, which = (i / words) % 2, b = i / (2 * words);
-    const long long frame = which == 0 ? 0 : p.T - 1;
-    const long long elem0 = (b * p.T + frame) * per;
-    reinterpret_cast<uint4*>(static_cast<char*>(O) + elem0 * esz)[w] = make_uint4(0, 0, 0, 0);
-  }
+  const long long b = blockIdx.y >> 1, frame = (blockIdx.y & 1) ? p.T - 1 : 0;
+  uint4* base = reinterpret_cast<uint4*>(static_cast<char*>(O) + (b * p.T + frame) * per * esz);
+  for (long long w = blockIdx.x * (long long)blockDim.x + threadIdx.x; w < words;
+       w += (long long)gridDim.x * blockDim.x)
+    base[w] = make_uint4(0, 0, 0, 0);
 }
 
 // ---------------------------------------------------------------------------
@@ -475,7 +474,7 @@ cudaError_t launch_readout_simt(const Problem& p, const void* gate, void* O, cud
 }
 
 cudaError_t launch_zero_anchors(const Problem& p, void* O, cudaStream_t s) {
-  zero_anchors_kernel<<<296, 256, 0, s>>>(p, O);
+  zero_anchors_kernel<<<dim3(148, 2 * p.B), 256, 0, s>>>(p, O);
   return cudaGetLastError();
 }
 

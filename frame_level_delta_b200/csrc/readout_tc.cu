@@ -242,6 +242,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int et = threadIdx.x - 64;  // 0..127 == tile row == TMEM lane
     const int q = warp % 4;
     const int r = q * 32 + lane;      // TMEM lane this warp may read
+    // Anchor frames 0 and T-1 read no linear memory: while the first tile's
+    // MMAs are in flight these threads zero this CTA's share of their rows
+    // (one contiguous slab of U * H * D values per batch and anchor).
+    {
+      const long long per16 = (long long)a.U * a.H * D * 2 / 16;  // uint4 words per slab
+      const long long G = gridDim.x;
+      const long long lo = per16 * blockIdx.x / G, hi = per16 * (blockIdx.x + 1) / G;
+      for (int slab = 0; slab < 2 * a.B; ++slab) {
+        const long long b = slab >> 1, f = (slab & 1) ? a.T - 1 : 0;
+        uint4* base = reinterpret_cast<uint4*>(a.O + (b * a.T + f) * (long long)a.U * a.H * D);
+        for (long long w = lo + et; w < hi; w += 128) base[w] = make_uint4(0, 0, 0, 0);
+      }
+    }
     int g_prev = -1;
     bool ok = true;
     uint32_t epi_phase = 0;

@@ -371,13 +371,12 @@ vda_status vda_readout(vda_ctx* ctx, const void* gate, void* O, void* stream) {
   if (!aligned16(O) || (gate && !aligned16(gate))) return fail(ctx, VDA_ERR_ALIGNMENT, "O and gate must be 16-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const Problem& p = ctx->p;
+  // The tensor-core readout zeroes the anchor frames itself.
+  if (!use_simt_only(ctx->cfg) && readout_tc_supported(p))
+    return run_kernel(ctx, K_READOUT_TC, s, [&] { return launch_readout_tc(p, gate, O, s); });
   vda_status st = run_kernel(ctx, K_ZERO_ANCHORS, s, [&] { return launch_zero_anchors(p, O, s); });
   if (st != VDA_OK) return st;
-  if (!use_simt_only(ctx->cfg) && readout_tc_supported(p))
-    st = run_kernel(ctx, K_READOUT_TC, s, [&] { return launch_readout_tc(p, gate, O, s); });
-  else
-    st = run_kernel(ctx, K_READOUT_SIMT, s, [&] { return launch_readout_simt(p, gate, O, s); });
-  return st;
+  return run_kernel(ctx, K_READOUT_SIMT, s, [&] { return launch_readout_simt(p, gate, O, s); });
 }
 
 vda_status vda_poll_device_status(vda_ctx* ctx, void* stream) {
