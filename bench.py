@@ -56,12 +56,17 @@ def load_peaks():
 # Algorithmic bytes / flops per launch of each kernel (each input byte read
 # once, each output byte written once).
 # ----------------------------------------------------------------------------
+# Whether the tensor-core scan runs over composed chunk maps (VDA_SCAN_CHUNKED)
+# or frame by frame (the default); set from --scan.
+SCAN_CHUNKED = False
+
+
 def composed_chunks(cfg):
     """Frame counts of the chunk maps the tensor-core scan composes (forward
     chunks 0..J-3 over frames max(1, c m)..c(m+1)-1, reverse chunks 2..J-1 over
     c m..min(c(m+1)-1, T-2)); empty when the scan steps over frames directly."""
     c, T, J = cfg.chunk, cfg.T, cfg.J
-    if c <= 1 or J < 3:
+    if not SCAN_CHUNKED or c <= 1 or J < 3:
         return []
     fwd = [max(0, c * (m + 1) - 1 - max(1, c * m) + 1) for m in range(0, J - 2)]
     rev = [max(0, min(c * (m + 1) - 1, T - 2) - c * m + 1) for m in range(2, J)]
@@ -337,6 +342,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work (0: skip)")
     ap.add_argument("--solve", default="sweep", choices=["sweep", "cholesky"],
                     help="tensor-core frame solve: symmetric sweep (default) or blocked Cholesky")
+    ap.add_argument("--scan", default="frames", choices=["frames", "chunked"],
+                    help="tensor-core scan frame by frame (default) or over composed chunk maps")
     ap.add_argument("--heads", type=int, default=0,
                     help="override H (a smaller case of the same workload, e.g. for profiler captures)")
     args = ap.parse_args()
@@ -367,7 +374,9 @@ def main():
     inp_cpu = make_inputs(cfg, seed=cfg.seed + rank)
     inp_host = {k: v.pin_memory() for k, v in inp_cpu.items()}
     inp_dev = {k: v.to(dev, non_blocking=True) for k, v in inp_host.items()}
-    lib = V.VDA(cfg, device=dev, cholesky=args.solve == "cholesky")
+    global SCAN_CHUNKED
+    SCAN_CHUNKED = args.scan == "chunked"
+    lib = V.VDA(cfg, device=dev, cholesky=args.solve == "cholesky", chunked=SCAN_CHUNKED)
     O = lib.new_output()
     stream = torch.cuda.current_stream(dev)
     for _ in range(args.warmup):

@@ -9,11 +9,16 @@
 //   (MM, JJ) <- (M_f0, C_f0);  for each next frame f: (MM, JJ) <- (MM M_f, JJ M_f + C_f).
 // Only the chunks the readout states need are composed: forward m = 0..J-3,
 // reverse m = 2..J-1; an empty chunk gets the identity map (I, 0).
-// Both products use the split operands of the tensor-core scan: MM and JJ as
-// bf16 hi/lo K-major images, M_f as the hi/lo image the solve wrote, three
-// products per pair, fp32 accumulation in TMEM (columns 0..127: MM M_f,
-// 128..255: JJ M_f). The final MM is stored as a hi/lo operand image and JJ as
-// fp32, exactly the operands of the chunk-level scan.
+//
+// Both products are three-term split products (bf16 hi/lo, ~2^-16 relative)
+// with fp32 accumulation. MM and JJ live in TMEM as the A operands (hi/lo bf16
+// pairs), next to their two fp32 accumulators, so each step's epilogue (one
+// thread per row) turns the accumulators into the next step's operands with
+// TMEM loads and stores only. M_f, the B operand, is the hi/lo image the solve
+// wrote, double-buffered in shared memory by bulk copies; C_f (fp32, column
+// quads) is staged in shared memory by a bulk copy as well. The last step
+// writes the composed map as a hi/lo operand image and JJ as fp32 column
+// quads, exactly the operands of the chunk-level scan.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -27,16 +32,22 @@ constexpr int D = 128;
 constexpr int kThreads = 128;
 constexpr int kImg = D * D * 2;   // one bf16 operand image
 constexpr int kPair = 2 * kImg;   // hi + lo
-constexpr int kMMOff = 0, kJJOff = kPair, kMfOff = 2 * kPair, kBarOff = 3 * kPair;
-constexpr int kSmemBytes = kBarOff + 64 + 1024;
+constexpr int kCBytes = D * D * 4;
+constexpr int kMfOff = 0;                      // two M_f buffers (hi, lo each)
+constexpr int kCOff = 2 * kPair;               // C_f, fp32 column quads
+constexpr int kBarOff = kCOff + kCBytes;
+constexpr int kSmemBytes = kBarOff + 128 + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+// TMEM columns: accumulators of MM M_f and JJ M_f, then MM and JJ as A operands.
+constexpr uint32_t kAccM = 0, kAccJ = 128, kMMh = 256, kMMl = 320, kJJh = 384, kJJl = 448;
 constexpr uint32_t kIdesc = sm100::idesc_bf16_f32(128, 128, false, true);  // A K-major, B MN-major
 
 struct ComposeArgs {
   int H, T, c, J;
   const uint8_t* Mi;  // per-frame M hi/lo images [B*H][T-1]
-  const float* C;     // per-frame C [B*H][T-1][D][D]
+  const float* C;     // per-frame C [B*H][T-1][D][D] (column quads)
   uint8_t* CMi;       // [B*H][2][J] hi/lo images
-  float* CC;          // [B*H][2][J][D][D]
+  float* CC;          // [B*H][2][J][D][D] (column quads)
   uint32_t* status;
   unsigned long long wait_ns;
 };
@@ -55,6 +66,18 @@ __device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
     const float2 hf = __bfloat1622float2(hh);
     h[q] = hh;
     l[q] = __floats2bfloat162_rn(x[2 * q] - hf.x, x[2 * q + 1] - hf.y);
+  }
+}
+
+// 32 consecutive values of a row as 16 hi and 16 lo bf16 pairs (lower column
+// in the low half): the TMEM A-operand layout.
+__device__ __forceinline__ void split32(const float (&x)[32], uint32_t (&hi)[16], uint32_t (&lo)[16]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 h, l;
+    split8(x + 8 * q, h, l);
+    hi[4 * q] = h.x; hi[4 * q + 1] = h.y; hi[4 * q + 2] = h.z; hi[4 * q + 3] = h.w;
+    lo[4 * q] = l.x; lo[4 * q + 1] = l.y; lo[4 * q + 2] = l.z; lo[4 * q + 3] = l.w;
   }
 }
 
@@ -104,10 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1) compose_tc_kernel(const ComposeAr
         float x[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) x[u] = (c8 * 8 + u == i) ? 1.f : 0.f;
-        uint4 hv, lv;
-        split8(x, hv, lv);
-        *reinterpret_cast<uint4*>(out_img + o) = hv;
-        *reinterpret_cast<uint4*>(out_img + kImg + o) = lv;
+        put8(out_img, i, c8 * 8, x);
       }
     }
     float4* cd = reinterpret_cast<float4*>(out_c);
@@ -117,147 +137,202 @@ __global__ void __launch_bounds__(kThreads, 1) compose_tc_kernel(const ComposeAr
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = sm100::align_smem_1024(smem_raw);
-  uint8_t* sMM = smem + kMMOff;
-  uint8_t* sJJ = smem + kJJOff;
-  uint8_t* sMf = smem + kMfOff;
-  uint64_t* ldbar = reinterpret_cast<uint64_t*>(smem + kBarOff);
-  uint64_t* mmabar = ldbar + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ldbar + 2);
+  uint8_t* sMf = smem + kMfOff;  // buffer s at sMf + s * kPair
+  const float4* sC = reinterpret_cast<const float4*>(smem + kCOff);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOff);  // [2]: M_f landed in buffer s
+  uint64_t* cbar = full + 2;                                     // C_f (and at first M_f0) landed
+  uint64_t* mmabar = full + 3;                                   // this step's MMAs are complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto mi = [&](int k) { return a.Mi + (slots + frame(k)) * (long long)kPair; };
+  auto ci = [&](int k) { return a.C + (slots + frame(k)) * (long long)D * D; };
 
+  // Thread 0 issues every copy and MMA and counts, per barrier, the completions
+  // it started and the ones it saw, so an abandoned step can be drained.
+  int issued_full[2] = {0, 0}, seen_full[2] = {0, 0};
+  int issued_c = 0, seen_c = 0, issued_mma = 0, seen_mma = 0;
   if (threadIdx.x == 0) {
-    mbar_init(ldbar, 1);
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
+    mbar_init(cbar, 1);
     mbar_init(mmabar, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    // MM <- M_f0 (its image is already the K-major operand layout) and the next frame's M.
-    mbar_arrive_expect_tx(ldbar, 2 * kPair);
-    const uint8_t* m0 = a.Mi + (slots + frame(0)) * (long long)kPair;
-    const uint8_t* m1 = a.Mi + (slots + frame(1)) * (long long)kPair;
-    bulk_load(sMM, m0, kImg, ldbar);
-    bulk_load(sMM + kImg, m0 + kImg, kImg, ldbar);
-    bulk_load(sMf, m1, kImg, ldbar);
-    bulk_load(sMf + kImg, m1 + kImg, kImg, ldbar);
+    // M_f0 (into buffer 1, read once by the threads) and C_f0; M_f1 into buffer 0.
+    mbar_arrive_expect_tx(cbar, kPair + kCBytes);
+    bulk_load(sMf + kPair, mi(0), kImg, cbar);
+    bulk_load(sMf + kPair + kImg, mi(0) + kImg, kImg, cbar);
+    bulk_load(smem + kCOff, ci(0), kCBytes, cbar);
+    issued_c = 1;
+    mbar_arrive_expect_tx(&full[0], kPair);
+    bulk_load(sMf, mi(1), kImg, &full[0]);
+    bulk_load(sMf + kImg, mi(1) + kImg, kImg, &full[0]);
+    issued_full[0] = 1;
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  // JJ <- C_f0 as a split image (row i).
-  {
-    const float4* src = reinterpret_cast<const float4*>(a.C + (slots + frame(0)) * (long long)D * D);
-    for (int c8 = 0; c8 < D / 8; ++c8) {
-      const float4 v0 = src[(2 * c8) * D + i];
-      const float4 v1 = src[(2 * c8 + 1) * D + i];
-      const float x[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-      put8(sJJ, i, c8 * 8, x);
-    }
-  }
-  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-  // Thread 0 owns the operand loads and the MMAs and tracks what is in flight,
-  // so that an abandoned step can be drained before TMEM and smem go away.
-  uint32_t ldph = 0, mph = 0;
-  bool ld_inflight = true, mma_inflight = false;
 
-  for (int k = 1; k < nf; ++k) {
-    const int f = frame(k);
-    bool ok = true;
+  // ---------------- MM <- M_f0 (its image rows are already bf16 hi/lo pairs), JJ <- C_f0
+  bool ok = mbar_wait(cbar, 0, abort_flag, a.status, a.wait_ns);
+  if (threadIdx.x == 0 && ok) seen_c = 1;
+  const bool started = !__syncthreads_or(!ok);
+  if (started) {
+    const uint8_t* m0 = sMf + kPair;
+#pragma unroll 1
+    for (int c32 = 0; c32 < D / 32; ++c32) {
+      uint32_t mh[16], ml[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t o = img_off(i, c32 * 32 + 8 * q);
+        const uint4 h = *reinterpret_cast<const uint4*>(m0 + o);
+        const uint4 l = *reinterpret_cast<const uint4*>(m0 + kImg + o);
+        mh[4 * q] = h.x; mh[4 * q + 1] = h.y; mh[4 * q + 2] = h.z; mh[4 * q + 3] = h.w;
+        ml[4 * q] = l.x; ml[4 * q + 1] = l.y; ml[4 * q + 2] = l.z; ml[4 * q + 3] = l.w;
+      }
+      tmem_st16(tl + kMMh + c32 * 16, mh);
+      tmem_st16(tl + kMMl + c32 * 16, ml);
+      float xj[32];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 v = sC[(c32 * 8 + q) * D + i];
+        xj[4 * q] = v.x; xj[4 * q + 1] = v.y; xj[4 * q + 2] = v.z; xj[4 * q + 3] = v.w;
+      }
+      uint32_t jh[16], jl[16];
+      split32(xj, jh, jl);
+      tmem_st16(tl + kJJh + c32 * 16, jh);
+      tmem_st16(tl + kJJl + c32 * 16, jl);
+    }
+    tmem_st_wait();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && started) {
+    // Buffer 1 and the C buffer are free again: M_f2 and C_f1.
+    if (nf > 2) {
+      mbar_arrive_expect_tx(&full[1], kPair);
+      bulk_load(sMf + kPair, mi(2), kImg, &full[1]);
+      bulk_load(sMf + kPair + kImg, mi(2) + kImg, kImg, &full[1]);
+      issued_full[1] = 1;
+    }
+    mbar_arrive_expect_tx(cbar, kCBytes);
+    bulk_load(smem + kCOff, ci(1), kCBytes, cbar);
+    issued_c = 2;
+  }
+
+  // ---------------- steps k = 1 .. nf-1: absorb frame(k), whose map sits in buffer (k-1) & 1
+#pragma unroll 1
+  for (int k = 1; k < nf && started; ++k) {
+    const int s = (k - 1) & 1;
+    ok = true;
     if (threadIdx.x == 0) {
-      ok = mbar_wait(ldbar, ldph, abort_flag, a.status, a.wait_ns);
+      ok = mbar_wait(&full[s], ((k - 1) >> 1) & 1, abort_flag, a.status, a.wait_ns);
       if (ok) {
-        ldph ^= 1;
-        ld_inflight = false;
+        ++seen_full[s];
         tc_fence_after();
-        const uint32_t mmh = smem_u32(sMM), mml = mmh + kImg, jjh = smem_u32(sJJ), jjl = jjh + kImg;
-        const uint32_t mfh = smem_u32(sMf), mfl = mfh + kImg;
-        const uint32_t as[3] = {0, 0, 1}, bs[3] = {0, 1, 0};
+        const uint32_t mfh = smem_u32(sMf + s * kPair), mfl = mfh + kImg;
+        const uint32_t am[3] = {kMMh, kMMh, kMMl}, aj[3] = {kJJh, kJJh, kJJl};
+        const uint32_t bs[3] = {mfh, mfl, mfh};
 #pragma unroll
         for (int t = 0; t < 3; ++t)
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t koffA = (kk / 4) * (D * 128) + (kk % 4) * 32;
-            const uint64_t db = smem_desc_sw128((bs[t] ? mfl : mfh) + kk * 2048, D * 128, 1024);
+            const uint64_t db = smem_desc_sw128(bs[t] + kk * 2048, D * 128, 1024);
             const uint32_t acc = (t == 0 && kk == 0) ? 0u : 1u;
-            mma_f16(tmem, smem_desc_sw128((as[t] ? mml : mmh) + koffA, 16, 1024), db, kIdesc, acc);
-            mma_f16(tmem + 128, smem_desc_sw128((as[t] ? jjl : jjh) + koffA, 16, 1024), db, kIdesc, acc);
+            mma_f16_ts(tmem + kAccM, tmem + am[t] + kk * 8, db, kIdesc, acc);
+            mma_f16_ts(tmem + kAccJ, tmem + aj[t] + kk * 8, db, kIdesc, acc);
           }
         mma_commit(mmabar);
-        mma_inflight = true;
+        ++issued_mma;
       }
     }
-    // C_f row i, fetched while the MMAs run.
-    const float4* csrc = reinterpret_cast<const float4*>(a.C + (slots + f) * (long long)D * D);
-    float crow[D];
-#pragma unroll
-    for (int t = 0; t < D / 4; ++t) {
-      const float4 v = csrc[t * D + i];
-      crow[4 * t] = v.x; crow[4 * t + 1] = v.y; crow[4 * t + 2] = v.z; crow[4 * t + 3] = v.w;
-    }
-    // A failed load wait in thread 0 sets the abort flag, which ends the others' waits.
-    if (ok) ok = mbar_wait(mmabar, mph, abort_flag, a.status, a.wait_ns);
-    if (ok) {
-      mph ^= 1;
-      if (threadIdx.x == 0) mma_inflight = false;
-    }
+    // A failed wait in thread 0 sets the abort flag, which ends the others' waits.
+    if (ok) ok = mbar_wait(mmabar, (k - 1) & 1, abort_flag, a.status, a.wait_ns);
+    if (ok && threadIdx.x == 0) ++seen_mma;
+    if (ok) ok = mbar_wait(cbar, k & 1, abort_flag, a.status, a.wait_ns);
+    if (ok && threadIdx.x == 0) ++seen_c;
     // Every thread takes the same exit, so the block barriers below stay matched.
     if (__syncthreads_or(!ok)) break;
     tc_fence_after();
-    // The MMAs are done with sMM, sJJ and sMf: prefetch the next frame's M.
-    if (threadIdx.x == 0 && k + 1 < nf) {
-      const uint8_t* mn = a.Mi + (slots + frame(k + 1)) * (long long)kPair;
-      mbar_arrive_expect_tx(ldbar, kPair);
-      bulk_load(sMf, mn, kImg, ldbar);
-      bulk_load(sMf + kImg, mn + kImg, kImg, ldbar);
-      ld_inflight = true;
+    // The MMAs are done with buffer s: the map two frames ahead goes there.
+    if (threadIdx.x == 0 && k + 2 < nf) {
+      mbar_arrive_expect_tx(&full[s], kPair);
+      bulk_load(sMf + s * kPair, mi(k + 2), kImg, &full[s]);
+      bulk_load(sMf + s * kPair + kImg, mi(k + 2) + kImg, kImg, &full[s]);
+      ++issued_full[s];
     }
     const bool last = k + 1 == nf;
-#pragma unroll
-    for (int c16 = 0; c16 < D / 16; ++c16) {
-      uint32_t v[16], w[16];
-      tmem_ld16(tl + c16 * 16, v);
-      tmem_ld16(tl + 128 + c16 * 16, w);
+#pragma unroll 1
+    for (int c32 = 0; c32 < D / 32; ++c32) {
+      uint32_t v0[16], v1[16], w0[16], w1[16];
+      tmem_ld16(tl + kAccM + c32 * 32, v0);
+      tmem_ld16(tl + kAccM + c32 * 32 + 16, v1);
+      tmem_ld16(tl + kAccJ + c32 * 32, w0);
+      tmem_ld16(tl + kAccJ + c32 * 32 + 16, w1);
       tmem_ld_wait();
-      float xm[16], xj[16];
+      float xm[32], xj[32];
 #pragma unroll
       for (int t = 0; t < 16; ++t) {
-        xm[t] = __uint_as_float(v[t]);
-        xj[t] = __uint_as_float(w[t]) + crow[c16 * 16 + t];
+        xm[t] = __uint_as_float(v0[t]);
+        xm[16 + t] = __uint_as_float(v1[t]);
+        xj[t] = __uint_as_float(w0[t]);
+        xj[16 + t] = __uint_as_float(w1[t]);
       }
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int col = c16 * 16 + 8 * hh;
-        if (last) {
-          put8(out_img, i, col, xm + 8 * hh);
-          float4* cd = reinterpret_cast<float4*>(out_c);
-          cd[(col / 4) * D + i] = make_float4(xj[8 * hh], xj[8 * hh + 1], xj[8 * hh + 2], xj[8 * hh + 3]);
-          cd[(col / 4 + 1) * D + i] = make_float4(xj[8 * hh + 4], xj[8 * hh + 5], xj[8 * hh + 6], xj[8 * hh + 7]);
-        } else {
-          put8(sMM, i, col, xm + 8 * hh);
-          put8(sJJ, i, col, xj + 8 * hh);
-        }
+      for (int q = 0; q < 8; ++q) {  // JJ M_f + C_f
+        const float4 v = sC[(c32 * 8 + q) * D + i];
+        xj[4 * q] += v.x; xj[4 * q + 1] += v.y; xj[4 * q + 2] += v.z; xj[4 * q + 3] += v.w;
+      }
+      if (last) {
+        float4* cd = reinterpret_cast<float4*>(out_c);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) put8(out_img, i, c32 * 32 + 8 * q, xm + 8 * q);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          cd[(c32 * 8 + q) * D + i] = make_float4(xj[4 * q], xj[4 * q + 1], xj[4 * q + 2], xj[4 * q + 3]);
+      } else {
+        uint32_t h[16], l[16];
+        split32(xm, h, l);
+        tmem_st16(tl + kMMh + c32 * 16, h);
+        tmem_st16(tl + kMMl + c32 * 16, l);
+        split32(xj, h, l);
+        tmem_st16(tl + kJJh + c32 * 16, h);
+        tmem_st16(tl + kJJl + c32 * 16, l);
       }
     }
+    tmem_st_wait();
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    // Everyone is done with C_f: the next frame's C goes into the buffer.
+    if (threadIdx.x == 0 && k + 1 < nf) {
+      mbar_arrive_expect_tx(cbar, kCBytes);
+      bulk_load(smem + kCOff, ci(k + 1), kCBytes, cbar);
+      ++issued_c;
+    }
   }
 
   // ---------------- teardown: nothing may be in flight when TMEM and smem go away
   tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 0) {
-    if (mma_inflight) mbar_wait(mmabar, mph, nullptr, a.status, a.wait_ns);
-    if (ld_inflight) mbar_wait(ldbar, ldph, nullptr, a.status, a.wait_ns);
+  if (threadIdx.x == 0 && *abort_flag) {
+    // Completions of one barrier arrive in order: waiting for the last one started covers all.
+    for (int s = 0; s < 2; ++s)
+      if (issued_full[s] > seen_full[s]) mbar_wait(&full[s], (issued_full[s] - 1) & 1, nullptr, a.status, a.wait_ns);
+    if (issued_c > seen_c) mbar_wait(cbar, (issued_c - 1) & 1, nullptr, a.status, a.wait_ns);
+    if (issued_mma > seen_mma) mbar_wait(mmabar, (issued_mma - 1) & 1, nullptr, a.status, a.wait_ns);
   }
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 

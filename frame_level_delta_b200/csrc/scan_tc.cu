@@ -12,7 +12,8 @@
 // for the next step. M_t's hi/lo images, written by the solve in the operand
 // layout, arrive by one bulk copy per frame, double-buffered; C_t rows are
 // prefetched into registers while the MMAs run.
-// Warp roles: 0 = bulk-copy producer, 1 = TMEM owner + MMA issuer, 2..5 = epilogue.
+// Warp roles: 0 = bulk-copy producer, 1 = TMEM owner + MMA issuer, 2..9 = epilogue
+// (two warps per TMEM lane quadrant, one per column half).
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -23,7 +24,7 @@ namespace vda {
 namespace {
 
 constexpr int D = 128;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // copy warp, MMA warp, eight epilogue warps
 constexpr int kImg = D * D * 2;           // one bf16 operand image
 constexpr int kMBuf = 2 * kImg;           // hi + lo images of one M_t
 constexpr int kSOff = 2 * kMBuf;          // S image (hi + lo) after two M buffers
@@ -78,8 +79,8 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
   uint64_t* mfull = reinterpret_cast<uint64_t*>(smem + kBarOff);
   uint64_t* mempty = mfull + 2;
   uint64_t* tfull = mempty + 2;
-  uint64_t* sready = tfull + 1;
-  uint64_t* drain = sready + 1;
+  uint64_t* sready = tfull + 1;  // [4]: K-chunk q (state columns 32q..32q+31) of the next image written
+  uint64_t* drain = sready + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -107,13 +108,13 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
       mbar_init(&mempty[s], 1);
     }
     mbar_init(tfull, 1);
-    mbar_init(sready, 4);
+    for (int q = 0; q < 4; ++q) mbar_init(&sready[q], 4);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 128);
+    tmem_alloc(tmem_slot, 256);  // two accumulators: step st uses columns (st & 1) * 128..
     tmem_relinquish();
   }
   tc_fence_before();
@@ -129,6 +130,10 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
         if (!mbar_wait(&mempty[s], ((st >> 1) & 1) ^ 1, abort_flag, a.status, a.wait_ns)) break;
         mbar_arrive_expect_tx(&mfull[s], kMBuf);
         const uint8_t* src = step_img(st);
+        // The step's injection rows are read by the epilogue threads with plain
+        // loads: bring them into L2 now, about two steps ahead.
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(step_c(st)), "r"((uint32_t)(D * D * 4))
+                     : "memory");
         bulk_load(sM + s * kMBuf, src, kImg, &mfull[s]);
         bulk_load(sM + s * kMBuf + kImg, src + kImg, kImg, &mfull[s]);
         issued = st + 1;
@@ -136,30 +141,44 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      for (int st = 0; st < nsteps; ++st) {
+      bool run = true;
+      for (int st = 0; st < nsteps && run; ++st) {
         const int s = st & 1;
-        if (!mbar_wait(sready, st & 1, abort_flag, a.status, a.wait_ns)) break;
+        const uint32_t acc = tmem + (uint32_t)(st & 1) * 128;
         if (!mbar_wait(&mfull[s], (st >> 1) & 1, abort_flag, a.status, a.wait_ns)) break;
-        tc_fence_after();
         const uint32_t sh = smem_u32(sS), sl = sh + kImg;
         const uint32_t mh = smem_u32(sM + s * kMBuf), ml = mh + kImg;
         const uint32_t as[3] = {sh, sh, sl}, bs[3] = {mh, ml, mh};
+        // K-chunk by K-chunk, as soon as the epilogue has written that part of S.
 #pragma unroll
-        for (int t = 0; t < 3; ++t)
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t da = smem_desc_sw128(as[t] + (kk / 4) * (D * 128) + (kk % 4) * 32, 16, 1024);
-            const uint64_t db = smem_desc_sw128(bs[t] + kk * 2048, D * 128, 1024);
-            mma_f16(tmem, da, db, kIdesc, (t == 0 && kk == 0) ? 0u : 1u);
+        for (int q = 0; q < 4; ++q) {
+          if (!mbar_wait(&sready[q], st & 1, abort_flag, a.status, a.wait_ns)) {
+            run = false;
+            break;
           }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 2 * q; kk < 2 * q + 2; ++kk)
+#pragma unroll
+            for (int t = 0; t < 3; ++t) {
+              const uint64_t da = smem_desc_sw128(as[t] + (kk / 4) * (D * 128) + (kk % 4) * 32, 16, 1024);
+              const uint64_t db = smem_desc_sw128(bs[t] + kk * 2048, D * 128, 1024);
+              mma_f16(acc, da, db, kIdesc, (kk == 0 && t == 0) ? 0u : 1u);
+            }
+        }
+        if (!run) break;
         mma_commit(&mempty[s]);
         mma_commit(tfull);
       }
       mma_commit(drain);
     }
   } else {
+    // Eight epilogue warps: warp w serves TMEM lanes (state rows) 32 (w % 4)..,
+    // columns 64 hf .. 64 hf + 63 (K-chunks 2 hf and 2 hf + 1 of the next image).
     const int q = warp % 4;
+    const int hf = (warp - 2) / 4;
     const int i = q * 32 + lane;  // state row == TMEM lane
+    constexpr int kCols = D / 2;
     float* out = dir == 0 ? a.Sf : a.Sr;
     auto store_row = [&](int j, const float* x, int col0, int n) {
       float4* d4 = reinterpret_cast<float4*>(out + ((long long)bh * J + j) * D * D);
@@ -170,37 +189,44 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
     // this direction, and the first operand image.
     {
       const float4* st0 = reinterpret_cast<const float4*>(a.C + slots * (long long)D * D);
-#pragma unroll 1
-      for (int c16 = 0; c16 < D / 16; ++c16) {
+      float4 row[kCols / 4];  // the whole half row first: one load latency
+#pragma unroll
+      for (int t = 0; t < kCols / 4; ++t) row[t] = st0[(hf * kCols / 4 + t) * D + i];
+#pragma unroll
+      for (int c16 = 0; c16 < kCols / 16; ++c16) {
+        const int col = hf * kCols + c16 * 16;
         float x[16];
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-          const float4 v = st0[(c16 * 4 + t) * D + i];
+          const float4 v = row[c16 * 4 + t];
           x[4 * t] = 0.5f * v.x; x[4 * t + 1] = 0.5f * v.y; x[4 * t + 2] = 0.5f * v.z; x[4 * t + 3] = 0.5f * v.w;
         }
         for (int j = 0; j < J; ++j)
-          if (dir == 0 ? (c * (j - 1) - 1 <= 0) : (c * (j + 2) >= T - 1)) store_row(j, x, c16 * 16, 16);
+          if (dir == 0 ? (c * (j - 1) - 1 <= 0) : (c * (j + 2) >= T - 1)) store_row(j, x, col, 16);
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           uint4 hi, lo;
           split8(x + 8 * hh, hi, lo);
-          const uint32_t o = img_off(i, c16 * 16 + 8 * hh);
+          const uint32_t o = img_off(i, col + 8 * hh);
           *reinterpret_cast<uint4*>(sS + o) = hi;
           *reinterpret_cast<uint4*>(sS + kImg + o) = lo;
         }
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(sready);
+      if (lane == 0) {
+        mbar_arrive(&sready[2 * hf]);
+        mbar_arrive(&sready[2 * hf + 1]);
+      }
     }
     for (int st = 0; st < nsteps; ++st) {
       const int f = dir == 0 ? f_first + st : f_first - st;
-      // Prefetch the injection's row i while the MMAs run.
-      float crow[D];
+      // Prefetch this warp's half of the injection's row i while the MMAs run.
+      float crow[kCols];
       const float4* csrc = reinterpret_cast<const float4*>(step_c(st));
 #pragma unroll
-      for (int t = 0; t < D / 4; ++t) {
-        const float4 v = csrc[t * D + i];
+      for (int t = 0; t < kCols / 4; ++t) {
+        const float4 v = csrc[(hf * kCols / 4 + t) * D + i];
         crow[4 * t] = v.x; crow[4 * t + 1] = v.y; crow[4 * t + 2] = v.z; crow[4 * t + 3] = v.w;
       }
       if (!mbar_wait(tfull, st & 1, abort_flag, a.status, a.wait_ns)) break;
@@ -213,28 +239,35 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
       } else {
         if (f % c == 0 && f / c - 2 >= 0) jout = f / c - 2;
       }
+      float xs[kCols];  // the new state's half row, stored once the MMAs have it
 #pragma unroll
-      for (int c16 = 0; c16 < D / 16; ++c16) {
+      for (int c16 = 0; c16 < kCols / 16; ++c16) {
+        const int col = hf * kCols + c16 * 16;
         uint32_t v[16];
-        tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + c16 * 16, v);
+        tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(st & 1) * 128 + col, v);
         tmem_ld_wait();
         float x[16];
 #pragma unroll
         for (int t = 0; t < 16; ++t) x[t] = __uint_as_float(v[t]) + crow[c16 * 16 + t];
-        if (jout >= 0) store_row(jout, x, c16 * 16, 16);
+#pragma unroll
+        for (int t = 0; t < 16; ++t) xs[c16 * 16 + t] = x[t];
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           uint4 hi, lo;
           split8(x + 8 * hh, hi, lo);
-          const uint32_t o = img_off(i, c16 * 16 + 8 * hh);
+          const uint32_t o = img_off(i, col + 8 * hh);
           *reinterpret_cast<uint4*>(sS + o) = hi;
           *reinterpret_cast<uint4*>(sS + kImg + o) = lo;
         }
+        if (c16 & 1) {  // K-chunk col / 32 of the next image is complete: release it to the MMAs
+          tc_fence_before();
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sready[col >> 5]);
+        }
       }
-      tc_fence_before();
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sready);
+      // The readout state leaves while the next step's MMAs run.
+      if (jout >= 0) store_row(jout, xs, hf * kCols, kCols);
     }
   }
 
@@ -251,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
     if (lane == 0) mbar_wait(drain, 0, nullptr, a.status, a.wait_ns);
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, 256);
   }
 }
 

@@ -23,6 +23,7 @@ VDA_F32, VDA_BF16 = 0, 1
 VDA_PREP_CONV = 0x1
 VDA_READOUT_NORM_GATE = 0x2
 VDA_SOLVE_CHOLESKY = 0x4
+VDA_SCAN_CHUNKED = 0x8
 VDA_FORCE_SIMT = 0x100
 REGIONS = {"status": 0, "A": 1, "B": 2, "M": 3, "C": 4, "S_fwd": 5, "S_rev": 6,
            "K_prep": 7, "V_prep": 8, "Kt_prep": 9, "Vt_prep": 10, "M_split": 11,
@@ -93,12 +94,14 @@ def lib() -> ctypes.CDLL:
 
 
 def make_config(cfg: VDAConfig, force_simt: bool = False, l2_eps: float = 1e-6,
-                rms_eps: float = 1e-6, cholesky: bool = False) -> vda_config:
+                rms_eps: float = 1e-6, cholesky: bool = False, chunked: bool = False) -> vda_config:
     flags = (VDA_PREP_CONV if cfg.prep_conv else 0) | (VDA_READOUT_NORM_GATE if cfg.norm_gate else 0)
     if force_simt:
         flags |= VDA_FORCE_SIMT
     if cholesky:
         flags |= VDA_SOLVE_CHOLESKY
+    if chunked:
+        flags |= VDA_SCAN_CHUNKED
     return vda_config(B=cfg.B, H=cfg.H, T=cfg.T, U=cfg.U, grid_h=cfg.grid_h, grid_w=cfg.grid_w, L=cfg.L,
                       d_k=cfg.d, d_v=cfg.d, chunk=cfg.chunk,
                       dtype=VDA_F32 if cfg.dtype == "f32" else VDA_BF16, flags=flags,
@@ -141,9 +144,10 @@ def describe(c: vda_config) -> str:
 class VDA:
     """One context of the library: prepare -> scan_bidir -> readout on a stream."""
 
-    def __init__(self, cfg: VDAConfig, force_simt: bool = False, device="cuda", cholesky: bool = False):
+    def __init__(self, cfg: VDAConfig, force_simt: bool = False, device="cuda", cholesky: bool = False,
+                 chunked: bool = False):
         self.cfg = cfg
-        self.c = make_config(cfg, force_simt=force_simt, cholesky=cholesky)
+        self.c = make_config(cfg, force_simt=force_simt, cholesky=cholesky, chunked=chunked)
         self._ctx = ctypes.c_void_p()
         st = lib().vda_create(ctypes.byref(self.c), ctypes.byref(self._ctx))
         if st != VDA_OK:

@@ -75,6 +75,9 @@ typedef enum vda_dtype {
 #define VDA_SOLVE_CHOLESKY 0x4u    /* tensor-core frame solve by blocked Cholesky of I + A_t and
                                       the triangular inverse, instead of the default symmetric
                                       sweep (Gauss-Jordan) in registers; the same M_t and C_t */
+#define VDA_SCAN_CHUNKED 0x8u      /* tensor-core scan over composed chunk maps (each chunk's frame
+                                      maps composed in parallel first) instead of the default scan
+                                      frame by frame; the same readout states */
 #define VDA_FORCE_SIMT 0x100u      /* run the generic CUDA-core kernels even where a tensor-core
                                       kernel exists (diagnostics and cross-checks) */
 

@@ -31,10 +31,10 @@ def rel_fro(a, b) -> float:
     return float(np.linalg.norm(a - b) / (nb if nb > 0 else 1.0))
 
 
-def run_gpu(cfg, inp_cpu, force_simt=False, cholesky=False):
+def run_gpu(cfg, inp_cpu, force_simt=False, cholesky=False, chunked=False):
     dev = torch.device("cuda:0")
     inp = {k: v.to(dev) for k, v in inp_cpu.items()}
-    lib = V.VDA(cfg, force_simt=force_simt, device=dev, cholesky=cholesky)
+    lib = V.VDA(cfg, force_simt=force_simt, device=dev, cholesky=cholesky, chunked=chunked)
     O = lib.run(inp)
     torch.cuda.synchronize()
     assert lib.poll_device_status() == 0
@@ -66,11 +66,11 @@ def staged_errors(cfg, regions, ref):
     return worst
 
 
-def check_config(cfg, heads=None, force_simt=False, inp=None, stage_tol=None, cholesky=False):
+def check_config(cfg, heads=None, force_simt=False, inp=None, stage_tol=None, cholesky=False, chunked=False):
     """Run both sides and assert the bounds. Returns (O error, staged errors)."""
     if inp is None:
         inp = make_inputs(cfg)
-    O_gpu, regions, lib = run_gpu(cfg, inp, force_simt=force_simt, cholesky=cholesky)
+    O_gpu, regions, lib = run_gpu(cfg, inp, force_simt=force_simt, cholesky=cholesky, chunked=chunked)
     if cholesky and not force_simt and cfg.dtype == "bf16" and cfg.d == 128:
         assert "solve=tcgen05-cholesky" in V.describe(lib.c)
     ref = vo.vda_reference(inp, cfg, heads=heads)

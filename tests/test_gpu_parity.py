@@ -43,6 +43,10 @@ def test_h3_full_size_cholesky_solve():
     check_config(CONFIGS["h3"], heads=[(0, 3), (0, 20)], cholesky=True)
 
 
+def test_h3_full_size_chunked_scan():
+    check_config(CONFIGS["h3"], heads=[(0, 7), (0, 16)], chunked=True)
+
+
 def test_long_full_size_sampled_heads():
     check_config(CONFIGS["long"], heads=[(0, 5), (0, 23)])
 
@@ -136,6 +140,7 @@ EDGE_CHUNKS = [
 def test_edge_chunk_structures_tensor_core_scan(name, kw):
     cfg = CONFIGS["small"].with_(name=name, d=128, H=2, grid_h=4, grid_w=5, L=9, **kw)
     check_config(cfg)
+    check_config(cfg, chunked=True)
     if name in ("d128_ragged_last_chunk", "d128_batch_two"):
         check_config(cfg, cholesky=True)
 
