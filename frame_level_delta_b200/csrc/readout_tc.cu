@@ -11,12 +11,13 @@
 //   O_tile = Q_tile S_hi^T + Q_tile S_lo^T   (M = 128 tokens, N = d_v, K = d_k)
 // accumulates in fp32 in TMEM with the state carried to ~2^-17 relative. Q tiles
 // arrive by TMA (K-major, 128-byte swizzle). TMEM is double-buffered so the
-// epilogue of one tile overlaps the MMAs of the next. The epilogue (one thread
-// per token row) applies 1/|q| (conv prep), RMSNorm and the gate, converts to
+// epilogue of one tile overlaps the MMAs of the next. The epilogue (two threads
+// per token row, one per half of the columns) applies 1/|q| (conv prep), RMSNorm and the gate, converts to
 // bf16, stages the tile in shared memory and writes it with a TMA store (plain
 // stores for the last, partial tile of a chunk).
-// Warp roles: 0 = TMA producer, 1 = TMEM owner + MMA issuer, 2..5 = prologue
-// and epilogue.
+// Warp roles: 0 = TMA producer, 1 = TMEM owner + MMA issuer, 2..9 = prologue
+// and epilogue (two warps per TMEM lane quadrant, one per half of the output
+// columns).
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -30,7 +31,8 @@ namespace vda {
 namespace {
 
 constexpr int kTileM = 128;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;     // TMA warp, MMA warp, eight epilogue warps
+constexpr int kEpiThreads = 256;
 
 template <int D, bool GATE>
 struct RoCfg {
@@ -44,8 +46,8 @@ struct RoCfg {
   // gate, a stage holds a Q tile and a gate tile: two stages.
   static constexpr int kStages = GATE ? 2 : (D == 128 ? 4 : 6);
   static constexpr int kStageBytes = kTileBytes * (GATE ? 2 : 1);
-  // layout: S_hi | S_lo | stages | output staging tile | barriers
-  static constexpr int kSmemBytes = 2 * kSBytes + kStages * kStageBytes + kTileBytes + 1024 + 256;
+  // layout: S_hi | S_lo | stages | output staging tile | barriers | RMS partial sums
+  static constexpr int kSmemBytes = 2 * kSBytes + kStages * kStageBytes + kTileBytes + 1024 + 256 + 1024;
   static_assert((2 * kStages + 7) * 8 + 16 <= 256, "barrier block overflows its allowance");
   static_assert(kSmemBytes <= 232448, "more shared memory than a CTA may use");
 };
@@ -136,6 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* epibar = drain + 1;  // bounded barrier of the 128 epilogue threads
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epibar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* ss_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + 256);  // [2][128]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   constexpr bool gate = GATE;
@@ -154,15 +157,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], stage_read ? 5 : 1);  // MMA commit (+ 4 epilogue warps)
+      mbar_init(&empty[s], stage_read ? 9 : 1);  // MMA commit (+ 8 epilogue warps)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4);
+      mbar_init(&tempty[i], 8);
     }
-    mbar_init(sready, 4);
+    mbar_init(sready, 8);
     mbar_init(drain, 1);
-    mbar_init(epibar, 128);
+    mbar_init(epibar, kEpiThreads);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&mQ);
@@ -239,9 +242,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------- prologue (S = S-> + S<-, split hi/lo) and epilogue
-    const int et = threadIdx.x - 64;  // 0..127 == tile row == TMEM lane
+    // Eight warps: warp w reads TMEM lanes (tile rows) 32 (w % 4).. and owns
+    // output columns hf * D / 2 .. of them.
+    const int et = threadIdx.x - 64;  // 0..255
     const int q = warp % 4;
-    const int r = q * 32 + lane;      // TMEM lane this warp may read
+    const int hf = (warp - 2) / 4;
+    const int r = q * 32 + lane;      // tile row == TMEM lane this warp may read
     // Anchor frames 0 and T-1 read no linear memory: while the first tile's
     // MMAs are in flight these threads zero this CTA's share of their rows
     // (one contiguous slab of U * H * D values per batch and anchor).
@@ -252,13 +258,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int slab = 0; slab < 2 * a.B; ++slab) {
         const long long b = slab >> 1, f = (slab & 1) ? a.T - 1 : 0;
         uint4* base = reinterpret_cast<uint4*>(a.O + (b * a.T + f) * (long long)a.U * a.H * D);
-        for (long long w = lo + et; w < hi; w += 128) base[w] = make_uint4(0, 0, 0, 0);
+        for (long long w = lo + et; w < hi; w += kEpiThreads) base[w] = make_uint4(0, 0, 0, 0);
       }
     }
     int g_prev = -1;
     bool ok = true;
     uint32_t epi_phase = 0;
-    // All 128 epilogue threads meet here; bounded, so a timed-out peer cannot
+    // All 256 epilogue threads meet here; bounded, so a timed-out peer cannot
     // leave the others waiting.
     auto epi_sync = [&]() -> bool {
       mbar_arrive(epibar);
@@ -275,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const long long off = ((long long)ti.bh * a.J + ti.j) * (long long)D * D;
         const float4* pf = reinterpret_cast<const float4*>(a.Sf + off);
         const float4* pr = reinterpret_cast<const float4*>(a.Sr + off);
-        for (int e = et; e < D * (D / 8); e += 128) {
+        for (int e = et; e < D * (D / 8); e += kEpiThreads) {
           const int c8 = e / D, i = e % D;  // row i, 8 consecutive k (column quads 2 c8, 2 c8 + 1)
           float x[8];
           const float4 f0 = pf[(2 * c8) * D + i], f1 = pf[(2 * c8 + 1) * D + i];
@@ -331,13 +337,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         scale = rsqrtf(qq + a.l2_eps);
       }
       const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + tb * D;
+      constexpr int kHalf = D / 2;  // output columns of this warp: col0 .. col0 + kHalf - 1
+      const int col0 = hf * kHalf;
       float rn = 1.f;
       if constexpr (GATE) {
+        // RMS over the whole row: each half sums its columns, the halves meet in shared memory.
         float ss = 0.f;
 #pragma unroll 1
-        for (int cc = 0; cc < D / 16; ++cc) {
+        for (int cc = 0; cc < kHalf / 16; ++cc) {
           uint32_t v[16];
-          tmem_ld16(taddr + cc * 16, v);
+          tmem_ld16(taddr + col0 + cc * 16, v);
           tmem_ld_wait();
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
@@ -345,16 +354,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             ss = fmaf(x, x, ss);
           }
         }
-        rn = rsqrtf(ss / D + a.rms_eps);
+        ss_part[hf * kTileM + r] = ss;
+        if (!epi_sync()) { ok = false; break; }
+        rn = rsqrtf((ss_part[r] + ss_part[kTileM + r]) / D + a.rms_eps);
       }
-      // Output row into registers: 16-byte chunk pair (2cc, 2cc+1) holds columns 16cc..16cc+15.
-      uint4 outs[D / 8];
+      // Output half row into registers: 16-byte chunk pair (2cc, 2cc+1) holds columns col0+16cc..+15.
+      uint4 outs[kHalf / 8];
 #pragma unroll
-      for (int cc = 0; cc < D / 16; ++cc) {
+      for (int cc = 0; cc < kHalf / 16; ++cc) {
         uint32_t v[16];
-        tmem_ld16(taddr + cc * 16, v);
+        tmem_ld16(taddr + col0 + cc * 16, v);
         tmem_ld_wait();
-        const int box = cc / 4, c16 = (cc % 4) * 2;
+        const int gc = col0 / 16 + cc;  // 16-column group of the whole row
+        const int box = gc / 4, c16 = (gc % 4) * 2;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           float g8[8];
@@ -393,14 +405,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!partial) {
         uint8_t* orow = sO + r * 128;
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          const int box = c / 8, pc = (c % 8) ^ (r & 7);
+        for (int c = 0; c < kHalf / 8; ++c) {
+          const int gcc = col0 / 8 + c;  // 8-column chunk of the whole row
+          const int box = gcc / 8, pc = (gcc % 8) ^ (r & 7);
           *reinterpret_cast<uint4*>(orow + box * (kTileM * 128) + pc * 16) = outs[c];
         }
       } else if (r < ti.nvalid) {
-        uint4* dst = reinterpret_cast<uint4*>(a.O + ((ti.tok0 + r) * a.H + h) * (long long)D);
+        uint4* dst = reinterpret_cast<uint4*>(a.O + ((ti.tok0 + r) * a.H + h) * (long long)D) + col0 / 8;
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) dst[c] = outs[c];
+        for (int c = 0; c < kHalf / 8; ++c) dst[c] = outs[c];
       }
       fence_proxy_async_smem();
       if (!epi_sync()) { ok = false; break; }
