@@ -6,14 +6,14 @@
 // chunk over the maps the composition kernel formed (same step, same operands):
 //   S <- S M_t + C_t,  S = Sh + Sl, M_t = Mh + Ml (bf16 parts, ~2^-16 relative),
 //   S M_t ~= Sh Mh + Sh Ml + Sl Mh  (24 MMAs of 128x128x16, fp32 in TMEM).
-// The fp32 state is rebuilt every step from TMEM plus C_t in the epilogue
-// (one thread per row), which also writes the readout states of the chunks
-// that need this frame's state and re-splits S into the K-major operand image
-// for the next step. M_t's hi/lo images, written by the solve in the operand
-// layout, arrive by one bulk copy per frame, double-buffered; C_t rows are
-// prefetched into registers while the MMAs run.
-// Warp roles: 0 = bulk-copy producer, 1 = TMEM owner + MMA issuer, 2..9 = epilogue
-// (two warps per TMEM lane quadrant, one per column half).
+// S lives in TMEM twice: as the fp32 accumulator (two buffers, alternating by
+// step) and as the bf16 hi/lo A operand of the next step's MMAs. The epilogue
+// (one thread per state row and column group) adds C_t, writes the readout
+// states of the chunks that need this state and the hi/lo operand, 32-column
+// K-chunk by K-chunk, so the next step's MMAs start on the first chunk while
+// the rest are still being written. M_t's hi/lo images (the B operand, in the
+// layout the solve wrote) arrive by bulk copies, double-buffered; C_t rows are
+// prefetched into registers (and into L2 two steps ahead) during the MMAs.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -27,10 +27,13 @@ constexpr int D = 128;
 constexpr int kThreads = 320;  // copy warp, MMA warp, eight epilogue warps
 constexpr int kImg = D * D * 2;           // one bf16 operand image
 constexpr int kMBuf = 2 * kImg;           // hi + lo images of one M_t
-constexpr int kSOff = 2 * kMBuf;          // S image (hi + lo) after two M buffers
-constexpr int kBarOff = kSOff + 2 * kImg;
+constexpr int kBarOff = 2 * kMBuf;        // barriers after the two M buffers
 constexpr int kSmemBytes = kBarOff + 128 + 1024;
-constexpr uint32_t kIdesc = sm100::idesc_bf16_f32(128, 128, false, true);  // A (S) K-major, B (M) MN-major
+// TMEM columns: two fp32 accumulators (step st uses (st & 1) * 128..), then S
+// as the A operand, bf16 hi and lo pairs (state column j in column j / 2).
+constexpr uint32_t kShi = 256, kSlo = 320;
+constexpr uint32_t kIdesc = sm100::idesc_bf16_f32(128, 128, false, true);  // A (S, TMEM) K-major, B (M) MN-major
+
 
 struct ScanArgs {
   int B, H, T, c, J;
@@ -45,11 +48,6 @@ struct ScanArgs {
   unsigned long long wait_ns;
 };
 
-__device__ __forceinline__ uint32_t img_off(int row, int col) {
-  const int atom = col >> 6, cc = col & 63;
-  return (uint32_t)(atom * D * 128 + row * 128 + ((((cc >> 3) ^ (row & 7))) << 4) + (cc & 7) * 2);
-}
-
 __device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
   __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&hi);
   __nv_bfloat162* l = reinterpret_cast<__nv_bfloat162*>(&lo);
@@ -60,6 +58,16 @@ __device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
     h[q] = hh;
     l[q] = __floats2bfloat162_rn(x[2 * q] - hf.x, x[2 * q + 1] - hf.y);
   }
+}
+
+// 16 consecutive values of a state row as 8 hi and 8 lo bf16 pairs (lower
+// column in the low half): the TMEM A-operand layout.
+__device__ __forceinline__ void split16(const float* x, uint32_t (&hi)[8], uint32_t (&lo)[8]) {
+  uint4 h0, l0, h1, l1;
+  split8(x, h0, l0);
+  split8(x + 8, h1, l1);
+  hi[0] = h0.x; hi[1] = h0.y; hi[2] = h0.z; hi[3] = h0.w; hi[4] = h1.x; hi[5] = h1.y; hi[6] = h1.z; hi[7] = h1.w;
+  lo[0] = l0.x; lo[1] = l0.y; lo[2] = l0.z; lo[3] = l0.w; lo[4] = l1.x; lo[5] = l1.y; lo[6] = l1.z; lo[7] = l1.w;
 }
 
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -75,7 +83,6 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = sm100::align_smem_1024(smem_raw);
   uint8_t* sM = smem;           // [2][hi, lo]
-  uint8_t* sS = smem + kSOff;   // [hi, lo]
   uint64_t* mfull = reinterpret_cast<uint64_t*>(smem + kBarOff);
   uint64_t* mempty = mfull + 2;
   uint64_t* tfull = mempty + 2;
@@ -108,13 +115,13 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
       mbar_init(&mempty[s], 1);
     }
     mbar_init(tfull, 1);
-    for (int q = 0; q < 4; ++q) mbar_init(&sready[q], 4);
+    for (int q = 0; q < 4; ++q) mbar_init(&sready[q], 8);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 256);  // two accumulators: step st uses columns (st & 1) * 128..
+    tmem_alloc(tmem_slot, 512);  // two accumulators and the S operand
     tmem_relinquish();
   }
   tc_fence_before();
@@ -146,9 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
         const int s = st & 1;
         const uint32_t acc = tmem + (uint32_t)(st & 1) * 128;
         if (!mbar_wait(&mfull[s], (st >> 1) & 1, abort_flag, a.status, a.wait_ns)) break;
-        const uint32_t sh = smem_u32(sS), sl = sh + kImg;
         const uint32_t mh = smem_u32(sM + s * kMBuf), ml = mh + kImg;
-        const uint32_t as[3] = {sh, sh, sl}, bs[3] = {mh, ml, mh};
+        const uint32_t as[3] = {kShi, kShi, kSlo}, bs[3] = {mh, ml, mh};
         // K-chunk by K-chunk, as soon as the epilogue has written that part of S.
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -161,9 +167,8 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
           for (int kk = 2 * q; kk < 2 * q + 2; ++kk)
 #pragma unroll
             for (int t = 0; t < 3; ++t) {
-              const uint64_t da = smem_desc_sw128(as[t] + (kk / 4) * (D * 128) + (kk % 4) * 32, 16, 1024);
               const uint64_t db = smem_desc_sw128(bs[t] + kk * 2048, D * 128, 1024);
-              mma_f16(acc, da, db, kIdesc, (kk == 0 && t == 0) ? 0u : 1u);
+              mma_f16_ts(acc, tmem + as[t] + kk * 8, db, kIdesc, (kk == 0 && t == 0) ? 0u : 1u);
             }
         }
         if (!run) break;
@@ -173,12 +178,16 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
       mma_commit(drain);
     }
   } else {
-    // Eight epilogue warps: warp w serves TMEM lanes (state rows) 32 (w % 4)..,
-    // columns 64 hf .. 64 hf + 63 (K-chunks 2 hf and 2 hf + 1 of the next image).
+    // Eight epilogue warps: warp w serves TMEM lanes (state rows) 32 (w % 4)..
+    // and the 16-column groups 2 cc + hf (cc = 0..3), so both warps of a lane
+    // quadrant finish each 32-column K-chunk of the next image together and the
+    // chunks reach the MMAs one after the other, as early as possible.
     const int q = warp % 4;
     const int hf = (warp - 2) / 4;
     const int i = q * 32 + lane;  // state row == TMEM lane
     constexpr int kCols = D / 2;
+    auto col_of = [&](int cc) { return 16 * (2 * cc + hf); };
+    const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
     float* out = dir == 0 ? a.Sf : a.Sr;
     auto store_row = [&](int j, const float* x, int col0, int n) {
       float4* d4 = reinterpret_cast<float4*>(out + ((long long)bh * J + j) * D * D);
@@ -189,12 +198,14 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
     // this direction, and the first operand image.
     {
       const float4* st0 = reinterpret_cast<const float4*>(a.C + slots * (long long)D * D);
-      float4 row[kCols / 4];  // the whole half row first: one load latency
+      float4 row[kCols / 4];  // all of this warp's columns first: one load latency
 #pragma unroll
-      for (int t = 0; t < kCols / 4; ++t) row[t] = st0[(hf * kCols / 4 + t) * D + i];
+      for (int cc = 0; cc < kCols / 16; ++cc)
+#pragma unroll
+        for (int t = 0; t < 4; ++t) row[cc * 4 + t] = st0[(col_of(cc) / 4 + t) * D + i];
 #pragma unroll
       for (int c16 = 0; c16 < kCols / 16; ++c16) {
-        const int col = hf * kCols + c16 * 16;
+        const int col = col_of(c16);
         float x[16];
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
@@ -203,32 +214,30 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
         }
         for (int j = 0; j < J; ++j)
           if (dir == 0 ? (c * (j - 1) - 1 <= 0) : (c * (j + 2) >= T - 1)) store_row(j, x, col, 16);
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint4 hi, lo;
-          split8(x + 8 * hh, hi, lo);
-          const uint32_t o = img_off(i, col + 8 * hh);
-          *reinterpret_cast<uint4*>(sS + o) = hi;
-          *reinterpret_cast<uint4*>(sS + kImg + o) = lo;
-        }
+        uint32_t hi[8], lo[8];
+        split16(x, hi, lo);
+        tmem_st8(tl + kShi + col / 2, hi);
+        tmem_st8(tl + kSlo + col / 2, lo);
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&sready[2 * hf]);
-        mbar_arrive(&sready[2 * hf + 1]);
-      }
+      if (lane == 0)
+        for (int q4 = 0; q4 < 4; ++q4) mbar_arrive(&sready[q4]);
     }
     for (int st = 0; st < nsteps; ++st) {
       const int f = dir == 0 ? f_first + st : f_first - st;
-      // Prefetch this warp's half of the injection's row i while the MMAs run.
+      // Prefetch this warp's columns of the injection's row i while the MMAs run.
       float crow[kCols];
       const float4* csrc = reinterpret_cast<const float4*>(step_c(st));
 #pragma unroll
-      for (int t = 0; t < kCols / 4; ++t) {
-        const float4 v = csrc[(hf * kCols / 4 + t) * D + i];
-        crow[4 * t] = v.x; crow[4 * t + 1] = v.y; crow[4 * t + 2] = v.z; crow[4 * t + 3] = v.w;
-      }
+      for (int cc = 0; cc < kCols / 16; ++cc)
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float4 v = csrc[(col_of(cc) / 4 + t) * D + i];
+          crow[16 * cc + 4 * t] = v.x; crow[16 * cc + 4 * t + 1] = v.y;
+          crow[16 * cc + 4 * t + 2] = v.z; crow[16 * cc + 4 * t + 3] = v.w;
+        }
       if (!mbar_wait(tfull, st & 1, abort_flag, a.status, a.wait_ns)) break;
       tc_fence_after();
       int jout = -1;
@@ -242,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
       float xs[kCols];  // the new state's half row, stored once the MMAs have it
 #pragma unroll
       for (int c16 = 0; c16 < kCols / 16; ++c16) {
-        const int col = hf * kCols + c16 * 16;
+        const int col = col_of(c16);
         uint32_t v[16];
         tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(st & 1) * 128 + col, v);
         tmem_ld_wait();
@@ -251,23 +260,19 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
         for (int t = 0; t < 16; ++t) x[t] = __uint_as_float(v[t]) + crow[c16 * 16 + t];
 #pragma unroll
         for (int t = 0; t < 16; ++t) xs[c16 * 16 + t] = x[t];
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint4 hi, lo;
-          split8(x + 8 * hh, hi, lo);
-          const uint32_t o = img_off(i, col + 8 * hh);
-          *reinterpret_cast<uint4*>(sS + o) = hi;
-          *reinterpret_cast<uint4*>(sS + kImg + o) = lo;
-        }
-        if (c16 & 1) {  // K-chunk col / 32 of the next image is complete: release it to the MMAs
-          tc_fence_before();
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sready[col >> 5]);
-        }
+        uint32_t hi[8], lo[8];
+        split16(x, hi, lo);
+        tmem_st8(tl + kShi + col / 2, hi);
+        tmem_st8(tl + kSlo + col / 2, lo);
+        // This warp's part of K-chunk col / 32 of the next operand is in TMEM: release it.
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sready[col >> 5]);
       }
       // The readout state leaves while the next step's MMAs run.
-      if (jout >= 0) store_row(jout, xs, hf * kCols, kCols);
+      if (jout >= 0)
+        for (int cc = 0; cc < kCols / 16; ++cc) store_row(jout, xs + 16 * cc, col_of(cc), 16);
     }
   }
 
@@ -284,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
     if (lane == 0) mbar_wait(drain, 0, nullptr, a.status, a.wait_ns);
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
