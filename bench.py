@@ -83,8 +83,8 @@ def kernel_bytes(name: str, cfg) -> float:
         return BH * ((F * U + L) * (2 * d * esz + 4) + 2 * NS * dd4)
     if name == "solve_simt":
         return BH * (4 * NS * dd4 + F * d * 4)
-    if name in ("solve_tc", "solve_chol_tc"):  # A, B read; M, C (fp32) and M's hi/lo operand images written
-        return BH * (4 * NS * dd4 + F * dd4 + F * d * 4)
+    if name in ("solve_tc", "solve_chol_tc"):  # A, B, alpha read; C (fp32) and M's hi/lo operand images written
+        return BH * (3 * NS * dd4 + F * dd4 + F * d * 4)
     if name == "scan_tc":  # per step: a (chunk) map's hi/lo images + its C; S_T; readout states
         if composed_chunks(cfg):
             steps = 2 * (J - 2)

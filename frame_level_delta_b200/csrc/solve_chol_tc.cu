@@ -368,11 +368,6 @@ __global__ void __launch_bounds__(kThreads, 2) solve_chol_tc_kernel(const SolveA
           *reinterpret_cast<uint4*>(mimg + kImg + o) = lo;
         }
       }
-      if (slot > 0) {
-        float4* md = reinterpret_cast<float4*>(a.M + off);
-#pragma unroll
-        for (int t = 0; t < 4; ++t) md[(j0 / 4 + t) * D + ri] = make_float4(mv[4 * t], mv[4 * t + 1], mv[4 * t + 2], mv[4 * t + 3]);
-      }
     }
   }
   fence_proxy_async_smem();

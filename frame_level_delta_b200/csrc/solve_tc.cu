@@ -15,8 +15,8 @@
 // block barrier per step. The loop over pivots is unrolled by 8, so the
 // pivot's row and column inside a tile are compile-time register indices.
 //
-// Then M = Diag(alpha) P (fp32 and the bf16 hi/lo operand images the
-// tensor-core scan loads as they are) and C = B P on tcgen05 with B_t split
+// Then M = Diag(alpha) P (the bf16 hi/lo operand images the tensor-core scan
+// loads as they are) and C = B P on tcgen05 with B_t split
 // into hi/lo in TMEM as the A operand and P as a hi/lo shared-memory image
 // (three-term split product, ~2^-16 relative, fp32 accumulation). The text
 // slot produces only C = S_T.
@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
     mbar_init(bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.Bm + off), "r"((uint32_t)(D * D * 4)) : "memory");
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, 256);
@@ -170,36 +171,6 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
-
-  // ---------------- B_t (row ri, columns hc*64..) -> TMEM as hi | lo bf16 pairs
-  {
-    const float4* src = reinterpret_cast<const float4*>(a.Bm + off);
-    float4 v[16];
-#pragma unroll
-    for (int t = 0; t < 16; ++t) v[t] = src[(hc * 16 + t) * D + ri];
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      uint32_t ph[16], pl[16];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        const float4 w = v[c * 8 + t];
-        const float xs[4] = {w.x, w.y, w.z, w.w};
-        float hv[4], lv[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          hv[u] = __bfloat162float(__float2bfloat16_rn(xs[u]));
-          lv[u] = xs[u] - hv[u];
-        }
-        ph[2 * t] = pack_bf16(hv[0], hv[1]);
-        ph[2 * t + 1] = pack_bf16(hv[2], hv[3]);
-        pl[2 * t] = pack_bf16(lv[0], lv[1]);
-        pl[2 * t + 1] = pack_bf16(lv[2], lv[3]);
-      }
-      tmem_st16(tl + kTmemB + hc * 32 + c * 16, ph);
-      tmem_st16(tl + kTmemB + 64 + hc * 32 + c * 16, pl);
-    }
-    tmem_st_wait();
-  }
 
   // ---------------- X = I + A into the register tiles; publish pivot 0
   float x[8][8];
@@ -233,7 +204,8 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
     sweep_step<7>(x, pv, K, ti, tj);
   }
 
-  // ---------------- P = -X: the P image for C = B P; M = Diag(alpha) P (fp32 + hi/lo images)
+  // ---------------- P = -X: the P image for C = B P; M = Diag(alpha) P as the hi/lo images
+  // the tensor-core scan reads (no fp32 copy: nothing on this path reads one)
   {
     float al[8];
     if (slot > 0) {
@@ -243,7 +215,6 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
       al[4] = a1.x; al[5] = a1.y; al[6] = a1.z; al[7] = a1.w;
     }
     uint8_t* mimg = a.Msplit + off * 4;  // two D*D bf16 images per slot
-    float4* md = reinterpret_cast<float4*>(a.M + off);
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int i = 8 * ti + r;
@@ -262,11 +233,40 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
         split8(mr, hi, lo);
         *reinterpret_cast<uint4*>(mimg + o) = hi;
         *reinterpret_cast<uint4*>(mimg + kImg + o) = lo;
-        md[(2 * tj) * D + i] = make_float4(mr[0], mr[1], mr[2], mr[3]);
-        md[(2 * tj + 1) * D + i] = make_float4(mr[4], mr[5], mr[6], mr[7]);
       }
     }
   }
+  // ---------------- B_t (row ri, columns hc*64..) -> TMEM as hi | lo bf16 pairs (from L2:
+  // prefetched at the start, needed only by C = B P)
+  {
+    const float4* src = reinterpret_cast<const float4*>(a.Bm + off);
+    float4 v[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) v[t] = src[(hc * 16 + t) * D + ri];
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      uint32_t ph[16], pl[16];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const float4 w = v[c * 8 + t];
+        const float xs[4] = {w.x, w.y, w.z, w.w};
+        float hv[4], lv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          hv[u] = __bfloat162float(__float2bfloat16_rn(xs[u]));
+          lv[u] = xs[u] - hv[u];
+        }
+        ph[2 * t] = pack_bf16(hv[0], hv[1]);
+        ph[2 * t + 1] = pack_bf16(hv[2], hv[3]);
+        pl[2 * t] = pack_bf16(lv[0], lv[1]);
+        pl[2 * t + 1] = pack_bf16(lv[2], lv[3]);
+      }
+      tmem_st16(tl + kTmemB + hc * 32 + c * 16, ph);
+      tmem_st16(tl + kTmemB + 64 + hc * 32 + c * 16, pl);
+    }
+    tmem_st_wait();
+  }
+
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();

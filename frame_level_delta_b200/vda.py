@@ -216,8 +216,10 @@ class VDA:
             return raw.view(torch.int32)
         if name == "chunk_C":
             return _from_quads(raw, (cfg.B, cfg.H, 2, cfg.J), D)
-        if name in ("M_split", "chunk_M"):  # bf16 hi/lo operand images, raw bytes
-            return raw
+        if name == "M_split":  # decoded: float32 [B, H, T-1, 2 (hi, lo), D, D]
+            return _from_images(raw, (cfg.B, cfg.H, cfg.T - 1, 2), D)
+        if name == "chunk_M":
+            return _from_images(raw, (cfg.B, cfg.H, 2, cfg.J, 2), D)
         dt = torch.float32 if cfg.dtype == "f32" else torch.bfloat16
         if name in ("K_prep", "V_prep"):
             return raw.view(dt).view(cfg.B, cfg.H, cfg.T, cfg.U, D)
@@ -248,6 +250,22 @@ def _from_quads(raw: torch.Tensor, lead: tuple, D: int) -> torch.Tensor:
     (element (i, j) at float ((j // 4) * D + i) * 4 + j % 4)."""
     q = raw.view(torch.float32).view(*lead, D // 4, D, 4)
     return q.movedim(-3, -2).reshape(*lead, D, D)
+
+
+def _image_index(D: int) -> torch.Tensor:
+    """Element offset of (i, j) in a bf16 D x D operand image (128-byte rows of
+    64 elements, 16-byte chunks XOR-swizzled by i % 8, 64-column atoms)."""
+    i = torch.arange(D).view(D, 1)
+    j = torch.arange(D).view(1, D)
+    byte = (j // 64) * D * 128 + i * 128 + (((j % 64) // 8) ^ (i % 8)) * 16 + (j % 8) * 2
+    return byte // 2
+
+
+def _from_images(raw: torch.Tensor, lead: tuple, D: int) -> torch.Tensor:
+    """Row-major float32 copies of bf16 operand images."""
+    flat = raw.view(torch.bfloat16).view(*lead, D * D)
+    idx = _image_index(D).to(flat.device).view(-1)
+    return flat.index_select(-1, idx).view(*lead, D, D).float()
 
 
 def run_static_workspace(cfg: VDAConfig, inp: Dict[str, torch.Tensor], O: torch.Tensor, stream=None) -> int:

@@ -166,7 +166,9 @@ typedef enum vda_region {
   VDA_REGION_STATUS = 0, /* uint32 device status word (+ padding) */
   VDA_REGION_A = 1,      /* float32 [B, H, T-1, d_k, d_k]; slot 0 = text, slot t = frame t */
   VDA_REGION_B = 2,      /* float32 [B, H, T-1, d_v, d_k]; same slots */
-  VDA_REGION_M = 3,      /* float32 [B, H, T-1, d_k, d_k]; slot t = M_t (slot 0 unused) */
+  VDA_REGION_M = 3,      /* float32 [B, H, T-1, d_k, d_k]; slot t = M_t (slot 0 unused); written by the
+                            CUDA-core solve only: the tensor-core solves write M_t as the hi/lo images of
+                            VDA_REGION_M_SPLIT, the form their scan reads */
   VDA_REGION_C = 4,      /* float32 [B, H, T-1, d_v, d_k]; slot 0 = S_T, slot t = C_t */
   VDA_REGION_S_FWD = 5,  /* float32 [B, H, J, d_v, d_k]; forward readout state of chunk j */
   VDA_REGION_S_REV = 6,  /* float32 [B, H, J, d_v, d_k]; reverse readout state of chunk j */
@@ -176,7 +178,9 @@ typedef enum vda_region {
   VDA_REGION_VT_PREP = 10, /* storage dtype [B, H, L, d]; prepared V_txt (VDA_PREP_CONV only) */
   VDA_REGION_M_SPLIT = 11, /* bf16 [B, H, T-1, 2, d*d]: M_t as hi + lo parts (M = hi + lo to ~2^-16),
                               each in the swizzled shared-memory operand layout of the tensor-core
-                              scan (used when that scan runs, unused otherwise) */
+                              scan: element (i, j) at byte (j / 64) * d * 128 + i * 128 +
+                              (((j % 64) / 8) XOR (i % 8)) * 16 + (j % 8) * 2 of its image
+                              (written by the tensor-core solves, unused otherwise) */
   VDA_REGION_CHUNK_M = 12, /* bf16 [B, H, 2, J, 2, d*d]: per direction and chunk, the composed transition
                               of the chunk's frames (hi, lo operand images; identity for empty chunks) */
   VDA_REGION_CHUNK_C = 13, /* float32 [B, H, 2, J, d_v, d_k]: the composed injection of those frames */

@@ -39,6 +39,10 @@ def run_gpu(cfg, inp_cpu, force_simt=False, cholesky=False, chunked=False):
     torch.cuda.synchronize()
     assert lib.poll_device_status() == 0
     regions = {k: lib.region(k).detach().cpu().clone() for k in ("A", "B", "M", "C", "S_fwd", "S_rev")}
+    if "solve=tcgen05" in V.describe(lib.c):
+        # The tensor-core solves write M_t only as hi/lo operand images.
+        mi = lib.region("M_split").detach().cpu()
+        regions["M"] = mi[:, :, :, 0] + mi[:, :, :, 1]
     if cfg.prep_conv:
         regions["K_prep"] = lib.region("K_prep").float().cpu()
         regions["V_prep"] = lib.region("V_prep").float().cpu()

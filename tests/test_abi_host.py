@@ -144,3 +144,19 @@ def test_region_view_undoes_column_quad_layout():
         for i in range(D):
             for j in range(D):
                 assert m[s, i, j] == s * D * D + ((j // 4) * D + i) * 4 + j % 4
+
+
+def test_region_view_decodes_operand_images():
+    """M_t's hi/lo images use the swizzled operand layout the header states:
+    element (i, j) at byte (j//64)*D*128 + i*128 + (((j%64)//8) ^ (i%8))*16 + (j%8)*2."""
+    import torch
+    from frame_level_delta_b200.vda import _from_images
+    D = 128
+    vals = torch.randn(D, D)
+    img = torch.zeros(D * D, dtype=torch.bfloat16)
+    for i in range(D):
+        for j in range(D):
+            byte = (j // 64) * D * 128 + i * 128 + (((j % 64) // 8) ^ (i % 8)) * 16 + (j % 8) * 2
+            img[byte // 2] = vals[i, j]
+    out = _from_images(img.view(torch.uint8), (1,), D)[0]
+    assert torch.equal(out, vals.bfloat16().float())
