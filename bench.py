@@ -134,7 +134,22 @@ def kernel_flops(name: str, cfg) -> float:
 
 # Kernels whose time is set by dense contractions and their serial dependencies
 # rather than by HBM streaming: their roofline is the bf16 tensor peak.
-TENSOR_BOUND = ("solve_tc", "solve_chol_tc", "solve_simt")
+TENSOR_BOUND = ("solve_chol_tc", "solve_simt")
+
+# Kernels whose time is set by fp32 FMAs on the CUDA cores. The symmetric sweep
+# applies every pivot's rank-1 update to the whole d x d matrix: d^3 FMAs per
+# slot. Peak: 148 SMs x 128 fp32 lanes x 2 flop per FMA x the SM clock.
+ALU_BOUND = ("solve_tc",)
+
+
+def kernel_alu_flops(name: str, cfg) -> float:
+    if name == "solve_tc":
+        return cfg.B * cfg.H * (cfg.T - 1) * 2 * cfg.d ** 3
+    return 0.0
+
+
+def alu_peak_tflops(sm_mhz: float) -> float:
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
 
 
 def path_bytes(cfg) -> float:
@@ -461,7 +476,14 @@ def main():
     dom_avg_s = dom_ms / dom_n / 1e3
     dom_bytes = kernel_bytes(dom_name, cfg)
     traffic = traffic_for(dom_name, cfg.name)
-    if dom_name in TENSOR_BOUND:
+    if dom_name in ALU_BOUND:
+        bound, unit = "alu", "TFLOP/s"
+        sm_mhz = float(clocks.summary().get("sm_mhz") or 1965.0)
+        achieved = kernel_alu_flops(dom_name, cfg) / dom_avg_s / 1e12
+        peak = alu_peak_tflops(sm_mhz)
+        peak_note = (f"fp32 FMA peak derived: 148 SMs x 128 lanes x 2 flop x {sm_mhz:.0f} MHz "
+                     f"(median SM clock in the timed region)")
+    elif dom_name in TENSOR_BOUND:
         # timed inside a long step: the sustained bf16 figure is the denominator
         bound, unit = "tensor", "TFLOP/s"
         achieved = kernel_flops(dom_name, cfg) / dom_avg_s / 1e12
@@ -495,7 +517,8 @@ def main():
                          "unit": unit, "frac": achieved / peak, "traffic": traffic,
                          "peak_source": peak_note,
                          "algorithmic_bytes_per_launch": dom_bytes,
-                         "algorithmic_flops_per_launch": kernel_flops(dom_name, cfg)},
+                         "algorithmic_flops_per_launch": kernel_flops(dom_name, cfg),
+                         "alu_flops_per_launch": kernel_alu_flops(dom_name, cfg) or None},
             "path_roofline": {"algorithmic_bytes_per_step": path_bytes(cfg),
                               "hbm_GBps": path_bytes(cfg) / step_s / 1e9,
                               "hbm_frac": path_bytes(cfg) / step_s / 1e9 / hbm_peak,
