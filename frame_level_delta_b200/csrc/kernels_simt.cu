@@ -308,78 +308,6 @@ __global__ void zero_anchors_kernel(Problem p, void* O) {
     base[w] = make_uint4(0, 0, 0, 0);
 }
 
-// ---------------------------------------------------------------------------
-// Feature prep (VDA_PREP_CONV). Video: grid (grid_h, T-2, B*H*2), block D
-// threads (one per channel). For grid row y of frame t, each thread slides
-// along x, keeping a 5x5 window of temporally filtered values, applies the
-// spatial filter, then SiLU; K tokens are then divided by sqrt(|k|^2 + eps).
-// Output layout [B, H, T, U, D] (frame-major per head).
-// ---------------------------------------------------------------------------
-__global__ void prep_video_kernel(Problem p, const void* Kraw, const void* Vraw, const float* w) {
-  extern __shared__ float srow[];  // [gw][D]
-  const int D = p.D, gh = p.gh, gw = p.gw, T = p.T, U = p.U, H = p.H;
-  const int y = blockIdx.x, t = blockIdx.y + 1;
-  const int z = blockIdx.z, which = z & 1, bh = z >> 1, b = bh / H, h = bh % H;
-  // blockDim.x = max(D, 32) so that the norm loop below always has >= 1 warp;
-  // threads with ch >= D only take part in the barrier and the norm.
-  const int ch = threadIdx.x;
-  const bool has_ch = ch < D;
-  const void* X = which == 0 ? Kraw : Vraw;
-  const long long hd = (long long)H * D;
-  const int chc = has_ch ? ch : 0;
-  const float* ws = w + (which == 0 ? 0 : hd * 30) + ((long long)h * D + chc) * 25;
-  const float* wt = w + (which == 0 ? hd * 25 : hd * 55) + ((long long)h * D + chc) * 5;
-  float fs[25], ft[5];
-#pragma unroll
-  for (int i = 0; i < 25; ++i) fs[i] = ws[i];
-#pragma unroll
-  for (int i = 0; i < 5; ++i) ft[i] = wt[i];
-  // Temporally filtered value at grid position (yy, xx), zero outside the clip.
-  auto tf = [&](int yy, int xx) -> float {
-    if (yy < 0 || yy >= gh || xx < 0 || xx >= gw) return 0.f;
-    float acc = 0.f;
-#pragma unroll
-    for (int s = 0; s < 5; ++s) {
-      const int tt = t + s - 2;
-      if (tt < 0 || tt >= T) continue;
-      const long long tok = (long long)b * T * U + (long long)tt * U + (long long)yy * gw + xx;
-      acc = fmaf(ft[s], ld_tok(X, (tok * H + h) * D + chc, p.bf16), acc);
-    }
-    return acc;
-  };
-  float win[5][5];  // win[a][q] = tf(y+a-2, x+q-2)
-#pragma unroll
-  for (int a = 0; a < 5; ++a)
-#pragma unroll
-    for (int q = 0; q < 5; ++q) win[a][q] = (q < 2) ? 0.f : tf(y + a - 2, q - 2);
-  for (int x = 0; x < gw && has_ch; ++x) {
-    float acc = 0.f;
-#pragma unroll
-    for (int a = 0; a < 5; ++a)
-#pragma unroll
-      for (int q = 0; q < 5; ++q) acc = fmaf(fs[a * 5 + q], win[a][q], acc);
-    srow[x * D + ch] = silu_f(acc);
-#pragma unroll
-    for (int a = 0; a < 5; ++a) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) win[a][q] = win[a][q + 1];
-      win[a][4] = tf(y + a - 2, x + 3);
-    }
-  }
-  __syncthreads();
-  void* out = which == 0 ? p.Kp : p.Vp;
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, nw = blockDim.x / 32;
-  for (int x = warp; x < gw; x += nw) {
-    float ss = 0.f;
-    for (int k = lane; k < D; k += 32) ss = fmaf(srow[x * D + k], srow[x * D + k], ss);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float sc = which == 0 ? rsqrtf(ss + p.l2_eps) : 1.f;
-    const long long ob = ((((long long)b * H + h) * T + t) * U + (long long)y * gw + x) * D;
-    for (int k = lane; k < D; k += 32) st_tok(out, ob + k, srow[x * D + k] * sc, p.bf16);
-  }
-}
-
 // Text prep: SiLU on K_txt and V_txt, then L2 on K_txt; one warp per token.
 // Output layout [B, H, L, D].
 __global__ void prep_text_kernel(Problem p, const void* Kt, const void* Vt) {
@@ -475,16 +403,6 @@ cudaError_t launch_readout_simt(const Problem& p, const void* gate, void* O, cud
 
 cudaError_t launch_zero_anchors(const Problem& p, void* O, cudaStream_t s) {
   zero_anchors_kernel<<<dim3(148, 2 * p.B), 256, 0, s>>>(p, O);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_prep_video(const Problem& p, const void* K, const void* V, const float* conv_w,
-                              cudaStream_t s) {
-  dim3 grid(p.gh, p.T - 2, p.B * p.H * 2);
-  const size_t smem = (size_t)p.gw * p.D * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(prep_video_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  prep_video_kernel<<<grid, p.D < 32 ? 32 : p.D, smem, s>>>(p, K, V, conv_w);
   return cudaGetLastError();
 }
 

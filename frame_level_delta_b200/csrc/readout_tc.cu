@@ -40,14 +40,17 @@ struct RoCfg {
   static constexpr int kTileBytes = kTileM * D * 2;       // one bf16 token tile
   static constexpr int kSAtomBytes = D * 128;             // one K-atom (64 k) of S: D rows x 128 B
   static constexpr int kSBytes = kBoxes * kSAtomBytes;    // one bf16 copy of S
-  static constexpr int kTmemCols = 2 * D;                 // two accumulators
+  // TMEM: two accumulators of D columns, then 4 columns for the row halves' partial sums.
+  static constexpr uint32_t kXchgCol = 2 * D;
+  static constexpr int kTmemAlloc = D == 128 ? 512 : 256;
   static constexpr uint32_t kIdesc = sm100::idesc_bf16_f32(128, D, false, false);
   // Q tiles are the only stream without the gate: four stages deep. With the
   // gate, a stage holds a Q tile and a gate tile: two stages.
   static constexpr int kStages = GATE ? 2 : (D == 128 ? 4 : 6);
   static constexpr int kStageBytes = kTileBytes * (GATE ? 2 : 1);
-  // layout: S_hi | S_lo | stages | output staging tile | barriers | RMS partial sums
-  static constexpr int kSmemBytes = 2 * kSBytes + kStages * kStageBytes + kTileBytes + 1024 + 256 + 1024;
+  // layout: S_hi | S_lo | stages | output staging tile | barriers
+  static constexpr int kSmemBytes = 2 * kSBytes + kStages * kStageBytes + kTileBytes + 1024 + 256;
+  static_assert((232448 / kSmemBytes) * kTmemAlloc <= 512, "CTAs that fit on an SM must fit in its TMEM");
   static_assert((2 * kStages + 7) * 8 + 16 <= 256, "barrier block overflows its allowance");
   static_assert(kSmemBytes <= 232448, "more shared memory than a CTA may use");
 };
@@ -114,7 +117,8 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-__device__ __forceinline__ float sigmoid_f(float x) { return 1.0f / (1.0f + __expf(-x)); }
+// Fast division intrinsic: a few ulp, far below the bf16 rounding of the output.
+__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
 
 template <int D, bool GATE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -138,7 +142,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* epibar = drain + 1;  // bounded barrier of the 128 epilogue threads
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epibar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* ss_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + 256);  // [2][128]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   constexpr bool gate = GATE;
@@ -173,7 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (gate) prefetch_tmap(&mG);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_alloc(tmem_slot, C::kTmemAlloc);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -319,14 +322,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (stage_read && !mbar_wait(&full[s], ph, abort_flag, a.status, a.wait_ns)) { ok = false; break; }
       const uint8_t* qrow = sQ + s * C::kStageBytes + r * 128;
       const uint8_t* grow = qrow + C::kTileBytes;
-      float scale = 1.f;
-      if (qnorm) {
-        float qq = 0.f;
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + tb * D;
+      constexpr int kHalf = D / 2;  // output columns of this warp: col0 .. col0 + kHalf - 1
+      const int col0 = hf * kHalf;
+      // Sums over the whole row: each half adds its channels (|q|^2) and its
+      // accumulator columns (|o|^2 before the 1/|q| scale, for the RMS norm); the
+      // two halves of a row swap their partial sums through two spare TMEM columns.
+      float av[GATE ? kHalf : 1];
+      uint4 gr[GATE ? kHalf / 8 : 1];
+      float scale = 1.f, rn = 1.f;
+      if (qnorm || GATE) {
+        float qq = 0.f, ss = 0.f;
+        if (qnorm) {
+          constexpr int kChunks = D / 16;  // 16-byte chunks of this half of the q row
 #pragma unroll
-        for (int box = 0; box < C::kBoxes; ++box)
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 v = *reinterpret_cast<const uint4*>(qrow + box * (kTileM * 128) + c * 16);
+          for (int c = 0; c < kChunks; ++c) {
+            const int gc = hf * kChunks + c;  // chunk of the whole row (swizzled order: the sum needs none)
+            const uint4 v = *reinterpret_cast<const uint4*>(qrow + (gc / 8) * (kTileM * 128) + (gc % 8) * 16);
             const __nv_bfloat162* e = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
             for (int k2 = 0; k2 < 4; ++k2) {
@@ -334,45 +346,65 @@ __global__ void __launch_bounds__(kThreads, 1)
               qq = fmaf(f.x, f.x, fmaf(f.y, f.y, qq));
             }
           }
-        scale = rsqrtf(qq + a.l2_eps);
-      }
-      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + tb * D;
-      constexpr int kHalf = D / 2;  // output columns of this warp: col0 .. col0 + kHalf - 1
-      const int col0 = hf * kHalf;
-      float rn = 1.f;
-      if constexpr (GATE) {
-        // RMS over the whole row: each half sums its columns, the halves meet in shared memory.
-        float ss = 0.f;
-#pragma unroll 1
-        for (int cc = 0; cc < kHalf / 16; ++cc) {
-          uint32_t v[16];
-          tmem_ld16(taddr + col0 + cc * 16, v);
-          tmem_ld_wait();
+        }
+        if constexpr (GATE) {
+          // This half row of the gate into registers, so the stage can go back at once.
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const float x = __uint_as_float(v[k]) * scale;
-            ss = fmaf(x, x, ss);
+          for (int c = 0; c < kHalf / 8; ++c) {
+            const int gcc = col0 / 8 + c;  // 8-column chunk of the whole row
+            gr[c] = *reinterpret_cast<const uint4*>(grow + (gcc / 8) * (kTileM * 128) + (((gcc % 8) ^ (r & 7)) * 16));
           }
         }
-        ss_part[hf * kTileM + r] = ss;
+        __syncwarp();
+        if (lane == 0 && stage_read) mbar_arrive(&empty[s]);  // Q (and gate) tile read: release the stage
+        if constexpr (GATE) {
+#pragma unroll
+          for (int cc = 0; cc < kHalf / 16; ++cc) {
+            uint32_t v[16];
+            tmem_ld16(taddr + col0 + cc * 16, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              av[cc * 16 + k] = __uint_as_float(v[k]);
+              ss = fmaf(av[cc * 16 + k], av[cc * 16 + k], ss);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[tb]);  // accumulator read: the MMAs may reuse it
+        }
+        const uint32_t xaddr = tmem + ((uint32_t)(q * 32) << 16) + C::kXchgCol;
+        tmem_st2(xaddr + 2 * hf, __float_as_uint(qq), __float_as_uint(ss));
+        tmem_st_wait();
+        tc_fence_before();
         if (!epi_sync()) { ok = false; break; }
-        rn = rsqrtf((ss_part[r] + ss_part[kTileM + r]) / D + a.rms_eps);
+        tc_fence_after();
+        uint32_t pq, ps;
+        tmem_ld2(xaddr + 2 * (1 - hf), pq, ps);
+        tmem_ld_wait();
+        if (qnorm) scale = rsqrtf(qq + __uint_as_float(pq) + a.l2_eps);
+        if constexpr (GATE) rn = rsqrtf(scale * scale * (ss + __uint_as_float(ps)) / D + a.rms_eps);
       }
       // Output half row into registers: 16-byte chunk pair (2cc, 2cc+1) holds columns col0+16cc..+15.
       uint4 outs[kHalf / 8];
 #pragma unroll
       for (int cc = 0; cc < kHalf / 16; ++cc) {
-        uint32_t v[16];
-        tmem_ld16(taddr + col0 + cc * 16, v);
-        tmem_ld_wait();
-        const int gc = col0 / 16 + cc;  // 16-column group of the whole row
-        const int box = gc / 4, c16 = (gc % 4) * 2;
+        float vf[16];
+        if constexpr (GATE) {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) vf[k] = av[cc * 16 + k];
+        } else {
+          uint32_t v[16];
+          tmem_ld16(taddr + col0 + cc * 16, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 16; ++k) vf[k] = __uint_as_float(v[k]);
+        }
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           float g8[8];
           if constexpr (GATE) {
-            const int pc = (c16 + half) ^ (r & 7);
-            const uint4 gv = *reinterpret_cast<const uint4*>(grow + box * (kTileM * 128) + pc * 16);
+            const uint4 gv = gr[2 * cc + half];
             const __nv_bfloat162* ge = reinterpret_cast<const __nv_bfloat162*>(&gv);
 #pragma unroll
             for (int k2 = 0; k2 < 4; ++k2) {
@@ -387,15 +419,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           __nv_bfloat162* op = reinterpret_cast<__nv_bfloat162*>(&outs[2 * cc + half]);
 #pragma unroll
           for (int k2 = 0; k2 < 4; ++k2)
-            op[k2] = __floats2bfloat162_rn(__uint_as_float(v[half * 8 + 2 * k2]) * scale * g8[2 * k2],
-                                           __uint_as_float(v[half * 8 + 2 * k2 + 1]) * scale * g8[2 * k2 + 1]);
+            op[k2] = __floats2bfloat162_rn(vf[half * 8 + 2 * k2] * scale * g8[2 * k2],
+                                           vf[half * 8 + 2 * k2 + 1] * scale * g8[2 * k2 + 1]);
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&tempty[tb]);
-        if (stage_read) mbar_arrive(&empty[s]);
+      if constexpr (!GATE) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[tb]);
       }
       // The staging buffer must have been read by the previous tile's TMA store.
       if (et == 0) bulk_wait_read0();
@@ -441,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) mbar_wait(drain, 0, nullptr, a.status, a.wait_ns);  // all MMAs retired
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
+    tmem_dealloc(tmem, C::kTmemAlloc);
   }
 }
 

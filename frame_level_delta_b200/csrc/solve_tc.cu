@@ -115,10 +115,17 @@ __device__ __forceinline__ void sweep_step(float (&x)[8][8], float* pv_all, int 
   float ur[8];
 #pragma unroll
   for (int r = 0; r < 8; ++r) ur[r] = vr[r] * inv;  // x_ik / x_kk
+  // The rank-1 update as packed fp32x2 FMAs (each lane rounds exactly as fmaf).
 #pragma unroll
-  for (int r = 0; r < 8; ++r)
+  for (int r = 0; r < 8; ++r) {
+    const float2 nu = make_float2(-ur[r], -ur[r]);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) x[r][c] = fmaf(-ur[r], vc[c], x[r][c]);
+    for (int c = 0; c < 8; c += 2) {
+      const float2 xv = __ffma2_rn(nu, make_float2(vc[c], vc[c + 1]), make_float2(x[r][c], x[r][c + 1]));
+      x[r][c] = xv.x;
+      x[r][c + 1] = xv.y;
+    }
+  }
   if (tj == K) {  // column k
 #pragma unroll
     for (int r = 0; r < 8; ++r) x[r][s] = ur[r];

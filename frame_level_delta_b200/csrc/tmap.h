@@ -37,4 +37,18 @@ inline cudaError_t make_tmap_bf16(CUtensorMap* m, const void* base, int rank, co
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// Same for any element type, without swizzle unless asked (plain row-major boxes).
+inline cudaError_t make_tmap_typed(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int rank,
+                                   const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                                   CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_NONE) {
+  auto fn = tmap_encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint32_t estride[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(m, dt, (cuuint32_t)rank, const_cast<void*>(base), reinterpret_cast<const cuuint64_t*>(dims),
+                  reinterpret_cast<const cuuint64_t*>(strides_bytes), reinterpret_cast<const cuuint32_t*>(box),
+                  estride, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace vda
