@@ -87,25 +87,41 @@ struct TileInfo {
   int nvalid;        // rows of the tile inside the chunk
 };
 
-__device__ __forceinline__ TileInfo tile_info(const RoArgs& a, int bh, int local) {
-  TileInfo ti;
-  ti.bh = bh;
-  int j = 0;
-  for (;; ++j) {
-    const int n = chunk_tiles(a, j);
-    if (local < n) break;
-    local -= n;
+
+// The tiles of one (b, h) in order, one step at a time: chunk j and tile
+// `local` within it (the direct lookup walks every earlier chunk).
+struct TileIter {
+  int j, local, n;  // chunk, tile within the chunk, tiles in the chunk
+  __device__ __forceinline__ void start(const RoArgs& a, int t) {
+    j = 0;
+    for (;; ++j) {
+      n = chunk_tiles(a, j);
+      if (t < n) break;
+      t -= n;
+    }
+    local = t;
   }
-  ti.j = j;
-  int lo, hi;
-  chunk_frames(a, j, lo, hi);
-  const long long first = (long long)lo * a.U + (long long)local * kTileM;
-  const long long end = (long long)hi * a.U;
-  ti.nvalid = (int)min((long long)kTileM, end - first);
-  const int b = ti.bh / a.H;
-  ti.tok0 = (long long)b * a.T * a.U + first;
-  return ti;
-}
+  // Valid only while tiles remain.
+  __device__ __forceinline__ void next(const RoArgs& a) {
+    if (++local < n) return;
+    local = 0;
+    do {
+      n = chunk_tiles(a, ++j);
+    } while (n == 0);
+  }
+  __device__ __forceinline__ TileInfo info(const RoArgs& a, int bh) const {
+    TileInfo ti;
+    ti.bh = bh;
+    ti.j = j;
+    int lo, hi;
+    chunk_frames(a, j, lo, hi);
+    const long long first = (long long)lo * a.U + (long long)local * kTileM;
+    const long long end = (long long)hi * a.U;
+    ti.nvalid = (int)min((long long)kTileM, end - first);
+    ti.tok0 = (long long)(bh / a.H) * a.T * a.U + first;
+    return ti;
+  }
+};
 
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
   asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
@@ -189,11 +205,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- TMA producer: Q tile (+ gate tile) per stage
     if (lane == 0) {
       const uint32_t bytes = C::kTileBytes * (gate ? 2 : 1);
+      TileIter tit;
+      if (ntiles > 0) tit.start(a, t_begin);
       for (int it = 0; it < ntiles; ++it) {
+        if (it > 0) tit.next(a);
         const int s = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
         if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, a.status, a.wait_ns)) break;
-        const TileInfo ti = tile_info(a, my_bh, t_begin + it);
+        const TileInfo ti = tit.info(a, my_bh);
         const int h = ti.bh % a.H;
         mbar_arrive_expect_tx(&full[s], bytes);
 #pragma unroll
@@ -210,8 +229,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- MMA issuer
     if (lane == 0) {
       int g_prev = -1, gi = 0;
+      TileIter tit;
+      if (ntiles > 0) tit.start(a, t_begin);
       for (int it = 0; it < ntiles; ++it) {
-        const TileInfo ti = tile_info(a, my_bh, t_begin + it);
+        if (it > 0) tit.next(a);
+        const TileInfo ti = tit.info(a, my_bh);
         const int g = ti.bh * a.J + ti.j;
         if (g != g_prev) {
           if (!mbar_wait(sready, gi & 1, abort_flag, a.status, a.wait_ns)) break;
@@ -275,8 +297,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       epi_phase ^= 1;
       return r;
     };
+    TileIter tit;
+    if (ntiles > 0) tit.start(a, t_begin);
     for (int it = 0; it < ntiles && ok; ++it) {
-      const TileInfo ti = tile_info(a, my_bh, t_begin + it);
+      if (it > 0) tit.next(a);
+      const TileInfo ti = tit.info(a, my_bh);
       const int g = ti.bh * a.J + ti.j;
       if (g != g_prev) {
         // The MMAs of the previous tile are complete (its accumulator was read
