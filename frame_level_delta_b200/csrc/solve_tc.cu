@@ -91,12 +91,15 @@ __device__ __forceinline__ float recip(float d) {
 }
 
 // Publish row `row` of this thread's tile (global row 8 ti + row) as the next
-// pivot vector, and, from the tile on the diagonal, the pivot's reciprocal.
+// pivot vector, and, from the tile on the diagonal, the pivot's reciprocal. The
+// vector is stored in two halves: entries 8t..8t+3 of tile t at float4 t, entries
+// 8t+4..8t+7 at float4 D/8 + t, so that a warp's float4 reads of the 16 tiles'
+// entries fall on distinct banks (consecutive 16-byte words) rather than on every
+// other group of four banks.
 template <int row>
 __device__ __forceinline__ void publish(float* pv, const float (&x)[8][8], int ti, int tj) {
-  float4* dst = reinterpret_cast<float4*>(pv + 8 * tj);
-  dst[0] = make_float4(x[row][0], x[row][1], x[row][2], x[row][3]);
-  dst[1] = make_float4(x[row][4], x[row][5], x[row][6], x[row][7]);
+  reinterpret_cast<float4*>(pv)[tj] = make_float4(x[row][0], x[row][1], x[row][2], x[row][3]);
+  reinterpret_cast<float4*>(pv + D / 2)[tj] = make_float4(x[row][4], x[row][5], x[row][6], x[row][7]);
   if (ti == tj) pv[D] = recip(x[row][row]);
 }
 
@@ -105,10 +108,10 @@ template <int s>
 __device__ __forceinline__ void sweep_step(float (&x)[8][8], float* pv_all, int K, int ti, int tj) {
   const float* v = pv_all + (s & 1) * kPvStride;
   float* vn = pv_all + ((s + 1) & 1) * kPvStride;
-  const float4 r0 = reinterpret_cast<const float4*>(v + 8 * ti)[0];
-  const float4 r1 = reinterpret_cast<const float4*>(v + 8 * ti)[1];
-  const float4 c0 = reinterpret_cast<const float4*>(v + 8 * tj)[0];
-  const float4 c1 = reinterpret_cast<const float4*>(v + 8 * tj)[1];
+  const float4 r0 = reinterpret_cast<const float4*>(v)[ti];
+  const float4 r1 = reinterpret_cast<const float4*>(v + D / 2)[ti];
+  const float4 c0 = reinterpret_cast<const float4*>(v)[tj];
+  const float4 c1 = reinterpret_cast<const float4*>(v + D / 2)[tj];
   const float inv = v[D];
   const float vr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
   const float vc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
@@ -167,7 +170,6 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
     mbar_init(bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.Bm + off), "r"((uint32_t)(D * D * 4)) : "memory");
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, 256);
@@ -201,6 +203,10 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
   // ---------------- the sweep: pivots k = 8 K + s
 #pragma unroll 1
   for (int K = 0; K < D / 8; ++K) {
+    // B_t is needed only after the sweep: fetch it into L2 in the middle of the
+    // sweep, not while the slot's A is being loaded.
+    if (K == 6 && tid == 0)
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.Bm + off), "r"((uint32_t)(D * D * 4)) : "memory");
     sweep_step<0>(x, pv, K, ti, tj);
     sweep_step<1>(x, pv, K, ti, tj);
     sweep_step<2>(x, pv, K, ti, tj);
@@ -244,7 +250,7 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
     }
   }
   // ---------------- B_t (row ri, columns hc*64..) -> TMEM as hi | lo bf16 pairs (from L2:
-  // prefetched at the start, needed only by C = B P)
+  // prefetched during the sweep, needed only by C = B P)
   {
     const float4* src = reinterpret_cast<const float4*>(a.Bm + off);
     float4 v[16];
