@@ -44,6 +44,12 @@ struct Problem {
   void* Msplit;  // [B,H,T-1] x 2 bf16 d*d images of M_t (hi, lo) for the tensor-core scan
   void* CMi;     // [B,H,2,J] x 2 bf16 d*d images: composed chunk transitions per direction
   float* CC;     // [B,H,2,J,D,D]: composed chunk injections per direction
+  // [B,H,T-1] slot-ready words (zeroed at the start of every prepare): the
+  // tensor-core sweep solve sets word (b,h,s) to 1 once slot s's C_t and M_t
+  // images are written, and the frame scan, launched to overlap the solve's
+  // last CTAs, acquires each word before it reads that slot. nullptr when the
+  // solve that ran does not publish them (the scan then waits for nothing).
+  uint32_t* ready;
   unsigned long long spin_limit;  // wall-time bound (ns) of every device-side wait
 };
 

@@ -14,6 +14,12 @@
 // the rest are still being written. M_t's hi/lo images (the B operand, in the
 // layout the solve wrote) arrive by bulk copies, double-buffered; C_t rows are
 // prefetched into registers (and into L2 two steps ahead) during the MMAs.
+//
+// In frame mode the kernel may be launched while the solve's last CTAs still
+// run (programmatic dependent launch): the copy thread then acquires each
+// slot's ready word before it copies that slot's M_t or lets the epilogue read
+// its C_t (through a counter in shared memory), so the scan advances through
+// every frame the solve has finished.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -42,6 +48,7 @@ struct ScanArgs {
   const uint8_t* Mi;  // [B,H,T-1] x (hi, lo) operand images
   const uint8_t* CMi; // [B,H,2,J] x (hi, lo) composed chunk transitions
   const float* CC;    // [B,H,2,J,D,D] composed chunk injections
+  const uint32_t* ready;  // [B,H,T-1] slot-ready words to acquire first, or nullptr
   float* Sf;
   float* Sr;
   uint32_t* status;
@@ -90,6 +97,9 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
   uint64_t* drain = sready + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // Slots whose ready word the copy thread has acquired: 1 = slot 0 (S_T), then
+  // st + 2 once step st's slot is.
+  uint32_t* cgot = reinterpret_cast<uint32_t*>(tmem_slot + 2);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int bh = blockIdx.x, dir = blockIdx.y;
@@ -118,6 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
     for (int q = 0; q < 4; ++q) mbar_init(&sready[q], 8);
     mbar_init(drain, 1);
     *abort_flag = 0;
+    *cgot = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -132,8 +143,18 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int st = 0; st < nsteps; ++st) {
+      bool go = a.ready == nullptr || flag_wait_gpu(a.ready + slots, 1u, abort_flag, a.status, a.wait_ns);
+      if (go) smem_release_u32(cgot, 1u);
+      for (int st = 0; go && st < nsteps; ++st) {
         const int s = st & 1;
+        // Acquire the slot before anything reads it: ahead of the wait for the
+        // buffer, so the epilogue's C_t loads find it already acquired.
+        if (a.ready != nullptr) {
+          const int f = dir == 0 ? f_first + st : f_first - st;
+          if (!flag_wait_gpu(a.ready + slots + f, 1u, abort_flag, a.status, a.wait_ns)) break;
+          fence_proxy_async_global();
+        }
+        smem_release_u32(cgot, (uint32_t)st + 2u);
         if (!mbar_wait(&mempty[s], ((st >> 1) & 1) ^ 1, abort_flag, a.status, a.wait_ns)) break;
         mbar_arrive_expect_tx(&mfull[s], kMBuf);
         const uint8_t* src = step_img(st);
@@ -196,7 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
     };
     // Initial state S_T / 2: readout states of the chunks that see no frame of
     // this direction, and the first operand image.
-    {
+    const bool live = smem_wait_geq(cgot, 1u, abort_flag, a.status, a.wait_ns);
+    if (live) {
       const float4* st0 = reinterpret_cast<const float4*>(a.C + slots * (long long)D * D);
       float4 row[kCols / 4];  // all of this warp's columns first: one load latency
 #pragma unroll
@@ -225,8 +247,9 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
       if (lane == 0)
         for (int q4 = 0; q4 < 4; ++q4) mbar_arrive(&sready[q4]);
     }
-    for (int st = 0; st < nsteps; ++st) {
+    for (int st = 0; live && st < nsteps; ++st) {
       const int f = dir == 0 ? f_first + st : f_first - st;
+      if (!smem_wait_geq(cgot, (uint32_t)st + 2u, abort_flag, a.status, a.wait_ns)) break;
       // Prefetch this warp's columns of the injection's row i while the MMAs run.
       float crow[kCols];
       const float4* csrc = reinterpret_cast<const float4*>(step_c(st));
@@ -304,11 +327,23 @@ cudaError_t launch_scan_tc(const Problem& p, cudaStream_t s, bool chunked) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
+  // Composed chunks come from a kernel that ran after the whole solve: only the
+  // frame scan waits on the slot-ready words, and only it overlaps the solve.
+  const bool overlap = !chunked && p.ready != nullptr;
   ScanArgs a{p.B, p.H, p.T, p.c, p.J, chunked ? 1 : 0, p.C, static_cast<const uint8_t*>(p.Msplit),
-             static_cast<const uint8_t*>(p.CMi), p.CC, p.Sf, p.Sr, p.status, p.spin_limit};
-  dim3 grid(p.B * p.H, 2);
-  scan_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(a);
-  return cudaGetLastError();
+             static_cast<const uint8_t*>(p.CMi), p.CC, overlap ? p.ready : nullptr, p.Sf, p.Sr, p.status,
+             p.spin_limit};
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(p.B * p.H, 2);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = overlap ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, scan_tc_kernel, a);
 }
 
 }  // namespace vda

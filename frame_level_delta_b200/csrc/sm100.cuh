@@ -79,6 +79,67 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Flags shared between the CTAs of two kernels that run at the same time (the
+// writer releases at GPU scope after its data; the reader acquires before it
+// reads the data).
+__device__ __forceinline__ void flag_release_gpu(uint32_t* f, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t flag_acquire_gpu(const uint32_t* f) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+  return v;
+}
+// Bounded wait until *f == v, with the timeout and abort rules of mbar_wait.
+__device__ __forceinline__ bool flag_wait_gpu(const uint32_t* f, uint32_t v, volatile int* abort, uint32_t* status,
+                                              uint64_t limit_ns) {
+  if (flag_acquire_gpu(f) == v) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    __nanosleep(64);
+    if (flag_acquire_gpu(f) == v) return true;
+    if ((n & 7) == 0) {
+      if (abort != nullptr && *abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        if (abort != nullptr) *abort = 1;
+        atomicExch(status, (uint32_t)VDA_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+// A counter in shared memory that one thread raises and others wait on.
+__device__ __forceinline__ void smem_release_u32(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t smem_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+// Bounded wait until the counter reaches at least v.
+__device__ __forceinline__ bool smem_wait_geq(const uint32_t* p, uint32_t v, volatile int* abort, uint32_t* status,
+                                              uint64_t limit_ns) {
+  if (smem_acquire_u32(p) >= v) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (smem_acquire_u32(p) >= v) return true;
+    if ((n & 31) == 0) {
+      if (abort != nullptr && *abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        if (abort != nullptr) *abort = 1;
+        atomicExch(status, (uint32_t)VDA_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+// Orders this thread's earlier generic-proxy accesses (here: a flag acquire)
+// before its later async-proxy (bulk copy) accesses of global memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // 4-byte asynchronous global -> shared copy; copies `src_bytes` (0 or 4) and
 // zero-fills the rest, so src_bytes = 0 reads nothing and stores a zero.
 __device__ __forceinline__ void cp_async_4(void* dst, const void* src, uint32_t src_bytes) {

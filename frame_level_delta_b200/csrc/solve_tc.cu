@@ -46,6 +46,7 @@ constexpr uint32_t kAccC = 0, kTmemB = 128;  // TMEM columns: C accumulator, B_t
 
 struct SolveArgs {
   int B, H, T;
+  uint32_t* ready;  // [B,H,T-1] slot-ready words, or nullptr
   const float* A;
   const float* Bm;
   const float* alpha;
@@ -147,6 +148,29 @@ __device__ __forceinline__ void sweep_step(float (&x)[8][8], float* pv_all, int 
   __syncthreads();
 }
 
+// CTA order over the n = T-1 slots of all BH heads, in the order the scans need
+// them: first every head's slot 0 (S_T, read by both directions at the start),
+// then key k = 1, 2, ...: slots k (forward step k-1) and n-k (reverse step k-1)
+// of every head, and for even n the middle slot n/2 last. CTAs start in about
+// this order, so the last wave holds the frames both scans reach last and the
+// scans, launched while that wave runs, advance on everything before them.
+__device__ __forceinline__ void order_slot(int cta, int BH, int n, int& bh, int& slot) {
+  if (cta < BH) {
+    bh = cta;
+    slot = 0;
+    return;
+  }
+  const int l = cta - BH, npairs = (n - 1) / 2;
+  if (l < npairs * 2 * BH) {
+    const int k = 1 + l / (2 * BH), w = l % (2 * BH);
+    bh = w >> 1;
+    slot = (w & 1) ? n - k : k;
+  } else {
+    bh = l - npairs * 2 * BH;
+    slot = n / 2;
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
@@ -158,8 +182,13 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int slot = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const long long off = (((long long)b * a.H + h) * (a.T - 1) + slot) * (long long)D * D;
+  // Let the scan kernel launch as soon as every solve CTA has started (it then
+  // waits on the slot-ready words, not on the end of this grid).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  int bh, slot;
+  order_slot(blockIdx.x, a.B * a.H, a.T - 1, bh, slot);
+  const int b = bh / a.H, h = bh % a.H;
+  const long long off = ((long long)bh * (a.T - 1) + slot) * (long long)D * D;
   // TMEM-side roles: matrix row ri == TMEM lane, column half hc.
   const int q = warp % 4, hc = warp / 4;
   const int ri = q * 32 + lane;
@@ -320,6 +349,11 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
   tc_fence_before();
   __syncthreads();
   if (tid == 0 && *abort_flag) mbar_wait(bar, 0, nullptr, a.status, a.wait_ns);
+  // Every thread's C_t and M_t stores precede the barrier above: publish the slot.
+  if (tid == 0 && ok && a.ready != nullptr) {
+    __threadfence();
+    flag_release_gpu(a.ready + (long long)bh * (a.T - 1) + slot, 1u);
+  }
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
@@ -338,10 +372,10 @@ cudaError_t launch_solve_tc(const Problem& p, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  SolveArgs a{p.B, p.H, p.T, p.A, p.Bm, p.alpha, p.M, p.C, static_cast<uint8_t*>(p.Msplit), p.status,
+  SolveArgs a{p.B, p.H, p.T, p.ready, p.A, p.Bm, p.alpha, p.M, p.C, static_cast<uint8_t*>(p.Msplit), p.status,
               p.spin_limit};
-  dim3 grid(p.T - 1, p.H, p.B);
-  solve_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(a);
+  const long long n = (long long)p.B * p.H * (p.T - 1);
+  solve_tc_kernel<<<(unsigned)n, kThreads, kSmemBytes, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -95,7 +95,8 @@ Layout make_layout(const vda_config& c) {
   const size_t d = (size_t)d_of(c), BH = (size_t)c.B * c.H;
   const size_t esz = c.dtype == VDA_BF16 ? 2 : 4;
   const bool prep = (c.flags & VDA_PREP_CONV) != 0;
-  L.bytes[VDA_REGION_STATUS] = 256;
+  // Status word (+ padding), then the [B,H,T-1] uint32 slot-ready words at byte 256.
+  L.bytes[VDA_REGION_STATUS] = 256 + align_up(BH * (c.T - 1) * 4, 256);
   L.bytes[VDA_REGION_A] = BH * (c.T - 1) * d * d * 4;
   L.bytes[VDA_REGION_B] = BH * (c.T - 1) * d * d * 4;
   L.bytes[VDA_REGION_M] = BH * (c.T - 1) * d * d * 4;
@@ -316,7 +317,8 @@ vda_status vda_prepare(vda_ctx* ctx, const void* Q, const void* K, const void* V
     p.Vt = TokView{V_txt, Lt * H * D, D, 0, H * D};
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(p.status, 0, 256, s);
+  // Clears the status word and the slot-ready words the solve raises.
+  cudaError_t e = cudaMemsetAsync(p.status, 0, L.bytes[VDA_REGION_STATUS], s);
   if (e != cudaSuccess) return cuda_fail(ctx, e, "status reset");
   vda_status st;
   if (prep) {
@@ -332,8 +334,12 @@ vda_status vda_prepare(vda_ctx* ctx, const void* Q, const void* K, const void* V
   if (st != VDA_OK) return st;
   if (!use_simt_only(c) && solve_tc_supported(p) && (c.flags & VDA_SOLVE_CHOLESKY))
     st = run_kernel(ctx, K_SOLVE_CHOL_TC, s, [&] { return launch_solve_chol_tc(p, s); });
-  else if (!use_simt_only(c) && solve_tc_supported(p))
+  else if (!use_simt_only(c) && solve_tc_supported(p)) {
+    // The sweep solve publishes per-slot ready words, so the frame scan may
+    // start on the slots finished while its last CTAs still run.
+    p.ready = p.status + 64;
     st = run_kernel(ctx, K_SOLVE_TC, s, [&] { return launch_solve_tc(p, s); });
+  }
   else
     st = run_kernel(ctx, K_SOLVE_SIMT, s, [&] { return launch_solve_simt(p, s); });
   if (st != VDA_OK) return st;

@@ -134,6 +134,10 @@ vda_status vda_prepare(vda_ctx* ctx, const void* Q, const void* K, const void* V
  * for t = 1 ..; reverse R(T-1) = S_T/2, R(t) = R(t+1) M_t + C_t for t = T-2 ..
  * down. Writes, for every chunk j, its forward and reverse readout states into
  * the workspace. VDA_ERR_STATE unless vda_prepare succeeded on this context.
+ * Queued on the stream of the vda_prepare call, the tensor-core frame scan is
+ * launched as a programmatic dependent of the solve and starts while the
+ * solve's last CTAs still run, reading each slot once its ready word is set
+ * (see VDA_REGION_STATUS); results do not depend on the overlap.
  */
 vda_status vda_scan_bidir(vda_ctx* ctx, void* stream);
 
@@ -163,7 +167,11 @@ vda_status vda_poll_device_status(vda_ctx* ctx, void* stream);
  * memory. The shapes name the logical indices, outermost first.
  */
 typedef enum vda_region {
-  VDA_REGION_STATUS = 0, /* uint32 device status word (+ padding) */
+  VDA_REGION_STATUS = 0, /* uint32 device status word (+ padding to byte 256), then uint32 [B, H, T-1]
+                            slot-ready words: vda_prepare clears the region, the tensor-core sweep
+                            solve sets word (b, h, s) to 1 once slot s's C_t and M_t are written, and
+                            the tensor-core frame scan (which may start while the solve's last CTAs
+                            run) reads a slot only after its word is 1 */
   VDA_REGION_A = 1,      /* float32 [B, H, T-1, d_k, d_k]; slot 0 = text, slot t = frame t */
   VDA_REGION_B = 2,      /* float32 [B, H, T-1, d_v, d_k]; same slots */
   VDA_REGION_M = 3,      /* float32 [B, H, T-1, d_k, d_k]; slot t = M_t (slot 0 unused); written by the
