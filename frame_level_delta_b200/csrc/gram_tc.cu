@@ -55,20 +55,23 @@ struct GramArgs {
   float* A;
   float* Bm;
   uint32_t* status;
+  uint32_t* gready;  // [B,H,T-1] per-slot counts raised after the stores, or nullptr
   unsigned long long wait_ns;
 };
 
-// Unit u = (b, h, slot) with heads fastest, so the CTAs working at any moment
-// cover all heads of neighbouring frames (one 6 KB token row holds every head).
+// Unit u = (b, h, slot) in the key order the solve consumes slots in (slot 0,
+// then slots k and T-1-k for k = 1, 2, ...), heads fastest within a slot, so
+// the CTAs working at any moment cover all heads of the same frames (one 6 KB
+// token row holds every head).
 struct Unit {
   int b, h, slot, n;
 };
 __device__ __forceinline__ Unit unit_of(const GramArgs& a, int u) {
   Unit x;
-  x.h = u % a.H;
-  const int r = u / a.H;
-  x.slot = r % (a.T - 1);
-  x.b = r / (a.T - 1);
+  int bh;
+  key_slot(u, a.B * a.H, a.T - 1, bh, x.slot);
+  x.b = bh / a.H;
+  x.h = bh % a.H;
   x.n = x.slot == 0 ? a.L : a.U;
   return x;
 }
@@ -101,6 +104,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int nunits = a.B * a.H * (a.T - 1);
   const int G = gridDim.x;
+  // The solve may launch now: its CTAs take the SMs this grid leaves and wait
+  // for their slot's count.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -319,7 +325,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[ub]);
+      if (lane == 0) {
+        mbar_arrive(&tempty[ub]);
+        // This warp's rows of A_t and B_t are stored (the warp barrier orders the
+        // other lanes' stores before this fence): count them for the solve.
+        if (a.gready != nullptr) {
+          __threadfence();
+          flag_add_release_gpu(a.gready + ((long long)x.b * a.H + x.h) * (a.T - 1) + x.slot, 1u);
+        }
+      }
     }
   }
 
@@ -381,7 +395,7 @@ template <int D>
 cudaError_t launch_d(const Problem& p, cudaStream_t s) {
   using C = GramCfg<D>;
   CUtensorMap mK, mV, mKt, mVt;
-  GramArgs a{p.B, p.H, p.T, p.U, p.L, 0, p.beta, p.beta_txt, p.A, p.Bm, p.status, p.spin_limit};
+  GramArgs a{p.B, p.H, p.T, p.U, p.L, 0, p.beta, p.beta_txt, p.A, p.Bm, p.status, p.gready, p.spin_limit};
   cudaError_t e = encode_maps(p, &mK, &mV, &mKt, &mVt, &a.layout);
   if (e != cudaSuccess) return e;
   static bool attr_set = false;

@@ -50,8 +50,37 @@ struct Problem {
   // last CTAs, acquires each word before it reads that slot. nullptr when the
   // solve that ran does not publish them (the scan then waits for nothing).
   uint32_t* ready;
+  // [B,H,T-1] words the tensor-core statistics kernel raises (one count per
+  // epilogue warp, kGramReadyCount in all) once slot s's A_t and B_t are written,
+  // for the sweep solve, launched to overlap that kernel's last units. nullptr
+  // when the statistics kernel that ran does not raise them.
+  uint32_t* gready;
   unsigned long long spin_limit;  // wall-time bound (ns) of every device-side wait
 };
+
+constexpr uint32_t kGramReadyCount = 4;
+
+// The order in which the statistics kernel, the solve and the frame scan treat
+// the n = T-1 slots of the BH heads: every head's slot 0 (S_T, read by both
+// scan directions first), then for key k = 1, 2, ...: slot k of every head
+// (forward step k-1), slot n-k of every head (reverse step k-1), and for even n
+// the middle slot n/2 last. Position idx in 0 .. BH*n-1 maps to (bh, slot).
+inline __host__ __device__ void key_slot(int idx, int BH, int n, int& bh, int& slot) {
+  if (idx < BH) {
+    bh = idx;
+    slot = 0;
+    return;
+  }
+  const int l = idx - BH, npairs = (n - 1) / 2;
+  if (l < npairs * 2 * BH) {
+    const int k = 1 + l / (2 * BH), w = l % (2 * BH);
+    bh = w % BH;
+    slot = w >= BH ? n - k : k;
+  } else {
+    bh = l - npairs * 2 * BH;
+    slot = n / 2;
+  }
+}
 
 // Slot s of the statistics / solve arrays: 0 = text, t = frame t (1..T-2).
 inline __host__ __device__ long long slot_off(const Problem& p, int b, int h, int s) {

@@ -34,7 +34,11 @@ constexpr int kThreads = 320;  // copy warp, MMA warp, eight epilogue warps
 constexpr int kImg = D * D * 2;           // one bf16 operand image
 constexpr int kMBuf = 2 * kImg;           // hi + lo images of one M_t
 constexpr int kBarOff = 2 * kMBuf;        // barriers after the two M buffers
-constexpr int kSmemBytes = kBarOff + 128 + 1024;
+constexpr int kSmemUsed = kBarOff + 128 + 1024;
+// Launched while the solve's last CTAs run, a scan CTA must not share an SM
+// with one (67 KB of shared memory each): it would wait in tcgen05.alloc for
+// the solve CTA's TMEM columns instead of starting on a free SM.
+constexpr int kSmemBytes = kSmemUsed > 164 * 1024 ? kSmemUsed : 164 * 1024;
 // TMEM columns: two fp32 accumulators (step st uses (st & 1) * 128..), then S
 // as the A operand, bf16 hi and lo pairs (state column j in column j / 2).
 constexpr uint32_t kShi = 256, kSlo = 320;

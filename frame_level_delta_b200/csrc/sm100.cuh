@@ -85,6 +85,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 __device__ __forceinline__ void flag_release_gpu(uint32_t* f, uint32_t v) {
   asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
 }
+__device__ __forceinline__ void flag_add_release_gpu(uint32_t* f, uint32_t v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+}
 __device__ __forceinline__ uint32_t flag_acquire_gpu(const uint32_t* f) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");

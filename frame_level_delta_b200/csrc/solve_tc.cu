@@ -2,24 +2,27 @@
 // S_t (I + A_t) = Sbar_t + B_t, transition M_t = Diag(alpha_t)(I + A_t)^-1, with
 // the inverse taken in the d_k x d_k key space; the injection is C_t = B_t (I + A_t)^-1).
 //
-// Per (b, h, slot), d = 128, one CTA of 256 threads, two CTAs per SM.
+// Per (b, h, slot), d = 128, one CTA of 160 threads, three CTAs per SM.
 //
 // The inverse P = (I + A)^-1 comes from the symmetric sweep (Gauss-Jordan
 // elimination without pivoting, safe here because I + A is symmetric positive
 // definite with every eigenvalue >= 1). Sweeping pivot k of a symmetric X:
 //   x_ij -= x_ik x_kj / x_kk  (i, j != k),  x_ik /= x_kk,  x_kj /= x_kk,  x_kk = -1 / x_kk,
-// and after all 128 pivots X = -P. Each thread keeps an 8 x 8 tile of X in
-// registers and applies the rank-1 update of every step to it (64 FMAs); the
-// pivot row (= column, by symmetry) and its reciprocal are published through
-// a double-buffered shared-memory vector by the threads that own it, with one
-// block barrier per step. The loop over pivots is unrolled by 8, so the
-// pivot's row and column inside a tile are compile-time register indices.
+// keeps X symmetric, and after all 128 pivots X = -P. Only the upper triangle
+// is kept: its 136 8 x 8 tiles (ti <= tj) live in the registers of threads
+// 0..135, which apply every step's rank-1 update to them (64 FMAs, as packed
+// fp32x2 FMAs). Pivot row k (= column k) is published through a double-buffered
+// shared-memory vector: its entries left of the diagonal tile come from column
+// k of the tiles above it, the rest from row k of the tiles right of it, and
+// the reciprocal from the diagonal tile; one block barrier per step. Half the
+// registers of a full-matrix sweep let three slots share an SM, whose steps
+// (each bound by the barrier -> load -> update -> publish latency) then overlap.
 //
 // Then M = Diag(alpha) P (the bf16 hi/lo operand images the tensor-core scan
-// loads as they are) and C = B P on tcgen05 with B_t split
-// into hi/lo in TMEM as the A operand and P as a hi/lo shared-memory image
-// (three-term split product, ~2^-16 relative, fp32 accumulation). The text
-// slot produces only C = S_T.
+// loads as they are), and C = B P on tcgen05 in two halves of the contraction
+// index: B_t (hi/lo, K-major) and 64 rows of P (hi/lo, N-major) as shared-memory
+// images, three-term split product (~2^-16 relative), fp32 accumulation in 128
+// TMEM columns. The text slot produces only C = S_T.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -30,23 +33,23 @@ namespace vda {
 namespace {
 
 constexpr int D = 128;
-constexpr int kThreads = 256;
-constexpr int kImg = D * D * 2;            // one bf16 operand image (two 64-column atoms of D rows)
-constexpr int kPOff = 0;                   // P image (hi, lo)
-constexpr int kPvOff = 2 * kImg;           // pivot vectors: 2 x (D values + reciprocal), 16-byte aligned
-constexpr int kPvStride = D + 4;           // floats per pivot buffer
-constexpr int kBarOff = kPvOff + 2 * kPvStride * 4 + 64;
-// More shared memory than the kernel uses, so that at most two CTAs share an
-// SM: each holds 256 of the SM's 512 TMEM columns.
-constexpr int kSmemBytes = 80 * 1024;
-static_assert(kBarOff + 64 + 1024 <= kSmemBytes, "shared memory layout");
-static_assert(3 * kSmemBytes > 227 * 1024, "at most two CTAs per SM");
+constexpr int kThreads = 160;               // five warps
+constexpr int kTiles = 136;                 // 8 x 8 tiles with ti <= tj
+constexpr int kHalf = 64 * D * 2;           // one bf16 image of 64 x 128 values (16 KB)
+constexpr int kPOff = 0;                    // P rows of one half: hi, lo (N-major, two 64-column atoms)
+constexpr int kBOff = 2 * kHalf;            // B_t columns of one half: hi, lo (K-major, one atom)
+constexpr int kPvOff = 4 * kHalf;           // pivot vectors: 2 x (D values + reciprocal)
+constexpr int kPvStride = D + 4;            // floats per pivot buffer (16-byte aligned)
+constexpr int kBarOff = kPvOff + 2 * kPvStride * 4;
+constexpr int kSmemBytes = kBarOff + 64 + 1024;  // + room to align the base to 1024 bytes
+static_assert(3 * (kSmemBytes + 1024) <= 228 * 1024, "three CTAs per SM");
+constexpr uint32_t kTmemCols = 128;         // the C accumulator; three CTAs use 384 of 512
 constexpr uint32_t kIdKM = sm100::idesc_bf16_f32(128, 128, false, true);  // A K-major, B MN-major
-constexpr uint32_t kAccC = 0, kTmemB = 128;  // TMEM columns: C accumulator, B_t hi (+64: lo)
 
 struct SolveArgs {
   int B, H, T;
-  uint32_t* ready;  // [B,H,T-1] slot-ready words, or nullptr
+  uint32_t* ready;         // [B,H,T-1] slot-ready words to raise, or nullptr
+  const uint32_t* gready;  // [B,H,T-1] statistics counts to wait for, or nullptr
   const float* A;
   const float* Bm;
   const float* alpha;
@@ -57,12 +60,12 @@ struct SolveArgs {
   unsigned long long wait_ns;
 };
 
-// Byte offset of element (row, col) in a bf16 operand image with 128-byte rows of
-// 64 elements, 16-byte chunks XOR-swizzled by (row % 8) and 64-column atoms of D
-// rows one after the other (the 128-byte-swizzle canonical layout).
-__device__ __forceinline__ uint32_t img_off(int row, int col) {
+// Byte offset of element (row, col) in a bf16 image with 128-byte rows of 64
+// elements, 16-byte chunks XOR-swizzled by (row % 8), and 64-column atoms of
+// `rows` rows one after the other (the 128-byte-swizzle canonical layout).
+__device__ __forceinline__ uint32_t img_off(int rows, int row, int col) {
   const int atom = col >> 6, cc = col & 63;
-  return (uint32_t)(atom * D * 128 + row * 128 + ((((cc >> 3) ^ (row & 7))) << 4) + (cc & 7) * 2);
+  return (uint32_t)(atom * rows * 128 + row * 128 + ((((cc >> 3) ^ (row & 7))) << 4) + (cc & 7) * 2);
 }
 
 __device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
@@ -91,128 +94,133 @@ __device__ __forceinline__ float recip(float d) {
   return fmaf(r, fmaf(-d, r, 1.f), r);
 }
 
-// Publish row `row` of this thread's tile (global row 8 ti + row) as the next
-// pivot vector, and, from the tile on the diagonal, the pivot's reciprocal. The
-// vector is stored in two halves: entries 8t..8t+3 of tile t at float4 t, entries
-// 8t+4..8t+7 at float4 D/8 + t, so that a warp's float4 reads of the 16 tiles'
-// entries fall on distinct banks (consecutive 16-byte words) rather than on every
-// other group of four banks.
+// The pivot vector is stored in two halves: entries 8t..8t+3 of tile t at
+// float4 t, entries 8t+4..8t+7 at float4 D/8 + t, so that a warp's float4 reads
+// of different tiles' entries fall on consecutive 16-byte words.
+__device__ __forceinline__ void put8(float* pv, int t, float a0, float a1, float a2, float a3, float a4, float a5,
+                                     float a6, float a7) {
+  reinterpret_cast<float4*>(pv)[t] = make_float4(a0, a1, a2, a3);
+  reinterpret_cast<float4*>(pv + D / 2)[t] = make_float4(a4, a5, a6, a7);
+}
+// Row `row` of tile (ti, tj) as entries 8 tj.. of the pivot vector; the
+// diagonal tile adds the pivot's reciprocal.
 template <int row>
-__device__ __forceinline__ void publish(float* pv, const float (&x)[8][8], int ti, int tj) {
-  reinterpret_cast<float4*>(pv)[tj] = make_float4(x[row][0], x[row][1], x[row][2], x[row][3]);
-  reinterpret_cast<float4*>(pv + D / 2)[tj] = make_float4(x[row][4], x[row][5], x[row][6], x[row][7]);
+__device__ __forceinline__ void publish_row(float* pv, const float (&x)[8][8], int ti, int tj) {
+  put8(pv, tj, x[row][0], x[row][1], x[row][2], x[row][3], x[row][4], x[row][5], x[row][6], x[row][7]);
   if (ti == tj) pv[D] = recip(x[row][row]);
+}
+// Column `col` of tile (ti, tj) above the diagonal as entries 8 ti.. (symmetry).
+template <int col>
+__device__ __forceinline__ void publish_col(float* pv, const float (&x)[8][8], int ti) {
+  put8(pv, ti, x[0][col], x[1][col], x[2][col], x[3][col], x[4][col], x[5][col], x[6][col], x[7][col]);
 }
 
 // One sweep step, pivot k = 8 K + s (s is a compile-time constant).
 template <int s>
-__device__ __forceinline__ void sweep_step(float (&x)[8][8], float* pv_all, int K, int ti, int tj) {
-  const float* v = pv_all + (s & 1) * kPvStride;
-  float* vn = pv_all + ((s + 1) & 1) * kPvStride;
-  const float4 r0 = reinterpret_cast<const float4*>(v)[ti];
-  const float4 r1 = reinterpret_cast<const float4*>(v + D / 2)[ti];
-  const float4 c0 = reinterpret_cast<const float4*>(v)[tj];
-  const float4 c1 = reinterpret_cast<const float4*>(v + D / 2)[tj];
-  const float inv = v[D];
-  const float vr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
-  const float vc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-  float ur[8];
+__device__ __forceinline__ void sweep_step(float (&x)[8][8], float* pv_all, int K, int ti, int tj, bool active) {
+  if (active) {
+    const float* v = pv_all + (s & 1) * kPvStride;
+    float* vn = pv_all + ((s + 1) & 1) * kPvStride;
+    const float4 r0 = reinterpret_cast<const float4*>(v)[ti];
+    const float4 r1 = reinterpret_cast<const float4*>(v + D / 2)[ti];
+    const float4 c0 = reinterpret_cast<const float4*>(v)[tj];
+    const float4 c1 = reinterpret_cast<const float4*>(v + D / 2)[tj];
+    const float inv = v[D];
+    const float vr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+    const float vc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+    float ur[8];
 #pragma unroll
-  for (int r = 0; r < 8; ++r) ur[r] = vr[r] * inv;  // x_ik / x_kk
-  // The rank-1 update as packed fp32x2 FMAs (each lane rounds exactly as fmaf).
+    for (int r = 0; r < 8; ++r) ur[r] = vr[r] * inv;  // x_ik / x_kk
+    // The rank-1 update as packed fp32x2 FMAs (each lane rounds exactly as fmaf).
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    const float2 nu = make_float2(-ur[r], -ur[r]);
+    for (int r = 0; r < 8; ++r) {
+      const float2 nu = make_float2(-ur[r], -ur[r]);
 #pragma unroll
-    for (int c = 0; c < 8; c += 2) {
-      const float2 xv = __ffma2_rn(nu, make_float2(vc[c], vc[c + 1]), make_float2(x[r][c], x[r][c + 1]));
-      x[r][c] = xv.x;
-      x[r][c + 1] = xv.y;
+      for (int c = 0; c < 8; c += 2) {
+        const float2 xv = __ffma2_rn(nu, make_float2(vc[c], vc[c + 1]), make_float2(x[r][c], x[r][c + 1]));
+        x[r][c] = xv.x;
+        x[r][c + 1] = xv.y;
+      }
     }
-  }
-  if (tj == K) {  // column k
+    if (tj == K) {  // column k (the tiles above and on the diagonal)
 #pragma unroll
-    for (int r = 0; r < 8; ++r) x[r][s] = ur[r];
-  }
-  if (ti == K) {  // row k
+      for (int r = 0; r < 8; ++r) x[r][s] = ur[r];
+    }
+    if (ti == K) {  // row k (the tiles on and right of the diagonal)
 #pragma unroll
-    for (int c = 0; c < 8; ++c) x[s][c] = vc[c] * inv;
-    if (tj == K) x[s][s] = -inv;
-  }
-  // The next pivot, k + 1, is row s + 1 of tile row K, or row 0 of tile row K + 1.
-  if (s < 7) {
-    if (ti == K) publish<(s + 1) & 7>(vn, x, ti, tj);
-  } else {
-    if (ti == K + 1) publish<0>(vn, x, ti, tj);
+      for (int c = 0; c < 8; ++c) x[s][c] = vc[c] * inv;
+      if (tj == K) x[s][s] = -inv;
+    }
+    // The next pivot, k + 1, is row/column n of tile row/column Kn.
+    constexpr int n = (s + 1) & 7;
+    const int Kn = s < 7 ? K : K + 1;
+    if (tj == Kn && ti < Kn) publish_col<n>(vn, x, ti);
+    if (ti == Kn) publish_row<n>(vn, x, ti, tj);
   }
   __syncthreads();
 }
 
-// CTA order over the n = T-1 slots of all BH heads, in the order the scans need
-// them: first every head's slot 0 (S_T, read by both directions at the start),
-// then key k = 1, 2, ...: slots k (forward step k-1) and n-k (reverse step k-1)
-// of every head, and for even n the middle slot n/2 last. CTAs start in about
-// this order, so the last wave holds the frames both scans reach last and the
-// scans, launched while that wave runs, advance on everything before them.
-__device__ __forceinline__ void order_slot(int cta, int BH, int n, int& bh, int& slot) {
-  if (cta < BH) {
-    bh = cta;
-    slot = 0;
-    return;
+// Tile t of the upper triangle, row-major: (0,0..15), (1,1..15), ...
+__device__ __forceinline__ void tile_of(int t, int& ti, int& tj) {
+  int r = 0, n = D / 8;
+  while (t >= n) {
+    t -= n;
+    ++r;
+    --n;
   }
-  const int l = cta - BH, npairs = (n - 1) / 2;
-  if (l < npairs * 2 * BH) {
-    const int k = 1 + l / (2 * BH), w = l % (2 * BH);
-    bh = w >> 1;
-    slot = (w & 1) ? n - k : k;
-  } else {
-    bh = l - npairs * 2 * BH;
-    slot = n / 2;
-  }
+  ti = r;
+  tj = r + t;
 }
 
-__global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a) {
+__global__ void __launch_bounds__(kThreads, 3) solve_tc_kernel(const SolveArgs a) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = sm100::align_smem_1024(smem_raw);
   uint8_t* pimg = smem + kPOff;
+  uint8_t* bimg = smem + kBOff;
   float* pv = reinterpret_cast<float*>(smem + kPvOff);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kBarOff);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kBarOff);  // [2]: the two halves' MMAs
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  // Let the scan kernel launch as soon as every solve CTA has started (it then
-  // waits on the slot-ready words, not on the end of this grid).
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // CTAs start in about key order, so the last wave holds the frames both
+  // scans reach last, and the scans, launched while that wave runs, advance on
+  // everything before them.
   int bh, slot;
-  order_slot(blockIdx.x, a.B * a.H, a.T - 1, bh, slot);
-  const int b = bh / a.H, h = bh % a.H;
+  key_slot(blockIdx.x, a.B * a.H, a.T - 1, bh, slot);
   const long long off = ((long long)bh * (a.T - 1) + slot) * (long long)D * D;
-  // TMEM-side roles: matrix row ri == TMEM lane, column half hc.
-  const int q = warp % 4, hc = warp / 4;
-  const int ri = q * 32 + lane;
-  // Sweep roles: the 8 x 8 tile (ti, tj) of X, rows 8 ti.., columns 8 tj..
-  const int ti = tid / 16, tj = tid % 16;
+  const bool active = tid < kTiles;
+  int ti = -1, tj = -1;
+  if (active) tile_of(tid, ti, tj);
 
   if (tid == 0) {
-    mbar_init(bar, 1);
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
+    // Launched while the statistics kernel finishes: wait until its four
+    // epilogue warps have stored this slot's A_t and B_t (the block barrier
+    // below orders every thread's loads after this acquire).
+    if (a.gready != nullptr)
+      flag_wait_gpu(a.gready + (long long)bh * (a.T - 1) + slot, kGramReadyCount, abort_flag, a.status, a.wait_ns);
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tl = tmem + ((uint32_t)(q * 32) << 16);
+  // Let the scan kernel launch once every solve CTA holds its TMEM (the scan
+  // then waits on the slot-ready words, not on the end of this grid, and never
+  // competes with a solve CTA for TMEM columns).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  // ---------------- X = I + A into the register tiles; publish pivot 0
+  // ---------------- X = I + A (upper tiles) into registers; publish pivot 0
   float x[8][8];
-  {
+  if (active) {
     const float4* src = reinterpret_cast<const float4*>(a.A + off);
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
@@ -225,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
 #pragma unroll
       for (int r = 0; r < 8; ++r) x[r][r] += 1.f;
     }
-    if (ti == 0) publish<0>(pv, x, ti, tj);
+    if (ti == 0) publish_row<0>(pv, x, ti, tj);
   }
   __syncthreads();
 
@@ -236,61 +244,108 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
     // sweep, not while the slot's A is being loaded.
     if (K == 6 && tid == 0)
       asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(a.Bm + off), "r"((uint32_t)(D * D * 4)) : "memory");
-    sweep_step<0>(x, pv, K, ti, tj);
-    sweep_step<1>(x, pv, K, ti, tj);
-    sweep_step<2>(x, pv, K, ti, tj);
-    sweep_step<3>(x, pv, K, ti, tj);
-    sweep_step<4>(x, pv, K, ti, tj);
-    sweep_step<5>(x, pv, K, ti, tj);
-    sweep_step<6>(x, pv, K, ti, tj);
-    sweep_step<7>(x, pv, K, ti, tj);
+    sweep_step<0>(x, pv, K, ti, tj, active);
+    sweep_step<1>(x, pv, K, ti, tj, active);
+    sweep_step<2>(x, pv, K, ti, tj, active);
+    sweep_step<3>(x, pv, K, ti, tj, active);
+    sweep_step<4>(x, pv, K, ti, tj, active);
+    sweep_step<5>(x, pv, K, ti, tj, active);
+    sweep_step<6>(x, pv, K, ti, tj, active);
+    sweep_step<7>(x, pv, K, ti, tj, active);
   }
 
-  // ---------------- P = -X: the P image for C = B P; M = Diag(alpha) P as the hi/lo images
-  // the tensor-core scan reads (no fp32 copy: nothing on this path reads one)
-  {
-    float al[8];
+  // ---------------- P = -X; M = Diag(alpha) P as the hi/lo images the scan reads
+  // (the tile and, off the diagonal, its mirror; no fp32 copy: nothing on this
+  // path reads one)
+  if (active) {
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) x[r][c] = -x[r][c];
     if (slot > 0) {
-      const float4* ap = reinterpret_cast<const float4*>(a.alpha + (((long long)b * a.H + h) * a.T + slot) * D + 8 * ti);
-      const float4 a0 = ap[0], a1 = ap[1];
-      al[0] = a0.x; al[1] = a0.y; al[2] = a0.z; al[3] = a0.w;
-      al[4] = a1.x; al[5] = a1.y; al[6] = a1.z; al[7] = a1.w;
-    }
-    uint8_t* mimg = a.Msplit + off * 4;  // two D*D bf16 images per slot
+      const float* al = a.alpha + ((long long)bh * a.T + slot) * D;
+      float ar[8], ac[8];
+      {
+        const float4 p0 = reinterpret_cast<const float4*>(al + 8 * ti)[0];
+        const float4 p1 = reinterpret_cast<const float4*>(al + 8 * ti)[1];
+        const float4 q0 = reinterpret_cast<const float4*>(al + 8 * tj)[0];
+        const float4 q1 = reinterpret_cast<const float4*>(al + 8 * tj)[1];
+        ar[0] = p0.x; ar[1] = p0.y; ar[2] = p0.z; ar[3] = p0.w; ar[4] = p1.x; ar[5] = p1.y; ar[6] = p1.z; ar[7] = p1.w;
+        ac[0] = q0.x; ac[1] = q0.y; ac[2] = q0.z; ac[3] = q0.w; ac[4] = q1.x; ac[5] = q1.y; ac[6] = q1.z; ac[7] = q1.w;
+      }
+      uint8_t* mimg = a.Msplit + off * 4;  // two D*D bf16 images per slot
+      constexpr int kImg = D * D * 2;
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int i = 8 * ti + r;
-      float pr[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) pr[c] = -x[r][c];
-      const uint32_t o = img_off(i, 8 * tj);
-      uint4 hi, lo;
-      split8(pr, hi, lo);
-      *reinterpret_cast<uint4*>(pimg + o) = hi;
-      *reinterpret_cast<uint4*>(pimg + kImg + o) = lo;
-      if (slot > 0) {
+      for (int r = 0; r < 8; ++r) {
         float mr[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) mr[c] = al[r] * pr[c];
+        for (int c = 0; c < 8; ++c) mr[c] = ar[r] * x[r][c];
+        uint4 hi, lo;
         split8(mr, hi, lo);
+        const uint32_t o = img_off(D, 8 * ti + r, 8 * tj);
         *reinterpret_cast<uint4*>(mimg + o) = hi;
         *reinterpret_cast<uint4*>(mimg + kImg + o) = lo;
       }
+      if (ti != tj) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          float mr[8];
+#pragma unroll
+          for (int r = 0; r < 8; ++r) mr[r] = ac[c] * x[r][c];
+          uint4 hi, lo;
+          split8(mr, hi, lo);
+          const uint32_t o = img_off(D, 8 * tj + c, 8 * ti);
+          *reinterpret_cast<uint4*>(mimg + o) = hi;
+          *reinterpret_cast<uint4*>(mimg + kImg + o) = lo;
+        }
+      }
     }
   }
-  // ---------------- B_t (row ri, columns hc*64..) -> TMEM as hi | lo bf16 pairs (from L2:
-  // prefetched during the sweep, needed only by C = B P)
-  {
-    const float4* src = reinterpret_cast<const float4*>(a.Bm + off);
-    float4 v[16];
+
+  // ---------------- C = B P in two halves of the contraction index k
+  bool ok = true;
 #pragma unroll
-    for (int t = 0; t < 16; ++t) v[t] = src[(hc * 16 + t) * D + ri];
+  for (int h = 0; h < 2; ++h) {
+    if (h == 1) {
+      // The first half's MMAs must have read the images before they are rewritten.
+      ok = mbar_wait(&bar[0], 0, abort_flag, a.status, a.wait_ns) && ok;
+      tc_fence_after();
+    }
+    // Rows 64 h.. of P: this tile's rows if its tile row is in the half, its
+    // mirrored rows if its tile column is.
+    if (active) {
+      if ((ti >> 3) == h) {
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      uint32_t ph[16], pl[16];
+        for (int r = 0; r < 8; ++r) {
+          uint4 hi, lo;
+          split8(x[r], hi, lo);
+          const uint32_t o = img_off(64, 8 * ti + r - 64 * h, 8 * tj);
+          *reinterpret_cast<uint4*>(pimg + o) = hi;
+          *reinterpret_cast<uint4*>(pimg + kHalf + o) = lo;
+        }
+      }
+      if (ti != tj && (tj >> 3) == h) {
 #pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        const float4 w = v[c * 8 + t];
+        for (int c = 0; c < 8; ++c) {
+          float pc[8];
+#pragma unroll
+          for (int r = 0; r < 8; ++r) pc[r] = x[r][c];
+          uint4 hi, lo;
+          split8(pc, hi, lo);
+          const uint32_t o = img_off(64, 8 * tj + c - 64 * h, 8 * ti);
+          *reinterpret_cast<uint4*>(pimg + o) = hi;
+          *reinterpret_cast<uint4*>(pimg + kHalf + o) = lo;
+        }
+      }
+    }
+    // Columns 64 h.. of B_t (from L2: prefetched during the sweep) as K-major
+    // hi/lo images: float4 f = (column quad 16 h + f / D, row f % D).
+    {
+      const float4* src = reinterpret_cast<const float4*>(a.Bm + off) + (long long)(16 * h) * D;
+#pragma unroll 4
+      for (int f = tid; f < 16 * D; f += kThreads) {
+        const float4 w = src[f];
+        const int i = f % D, kq = f / D;  // row, column quad within the half
         const float xs[4] = {w.x, w.y, w.z, w.w};
         float hv[4], lv[4];
 #pragma unroll
@@ -298,66 +353,66 @@ __global__ void __launch_bounds__(kThreads, 2) solve_tc_kernel(const SolveArgs a
           hv[u] = __bfloat162float(__float2bfloat16_rn(xs[u]));
           lv[u] = xs[u] - hv[u];
         }
-        ph[2 * t] = pack_bf16(hv[0], hv[1]);
-        ph[2 * t + 1] = pack_bf16(hv[2], hv[3]);
-        pl[2 * t] = pack_bf16(lv[0], lv[1]);
-        pl[2 * t + 1] = pack_bf16(lv[2], lv[3]);
+        const uint32_t o = img_off(D, i, 4 * kq);
+        *reinterpret_cast<uint2*>(bimg + o) = make_uint2(pack_bf16(hv[0], hv[1]), pack_bf16(hv[2], hv[3]));
+        *reinterpret_cast<uint2*>(bimg + kHalf + o) = make_uint2(pack_bf16(lv[0], lv[1]), pack_bf16(lv[2], lv[3]));
       }
-      tmem_st16(tl + kTmemB + hc * 32 + c * 16, ph);
-      tmem_st16(tl + kTmemB + 64 + hc * 32 + c * 16, pl);
     }
-    tmem_st_wait();
-  }
-
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-
-  // ---------------- C = B P (A operand B_t from TMEM, B operand the P image)
-  if (tid == 0) {
-    tc_fence_after();
-    const uint32_t pb = smem_u32(pimg);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t pb = smem_u32(pimg), bb = smem_u32(bimg);
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint64_t ph = smem_desc_sw128(pb + kk * 2048, D * 128, 1024);
-      const uint64_t pl = smem_desc_sw128(pb + kImg + kk * 2048, D * 128, 1024);
-      const uint32_t bh = tmem + kTmemB + kk * 8, bl = tmem + kTmemB + 64 + kk * 8;
-      mma_f16_ts(tmem + kAccC, bh, ph, kIdKM, kk > 0 ? 1u : 0u);
-      mma_f16_ts(tmem + kAccC, bh, pl, kIdKM, 1u);
-      mma_f16_ts(tmem + kAccC, bl, ph, kIdKM, 1u);
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t ph = smem_desc_sw128(pb + kk * 2048, 64 * 128, 1024);
+        const uint64_t pl = smem_desc_sw128(pb + kHalf + kk * 2048, 64 * 128, 1024);
+        const uint64_t dbh = smem_desc_sw128(bb + kk * 32, 16, 1024);
+        const uint64_t dbl = smem_desc_sw128(bb + kHalf + kk * 32, 16, 1024);
+        mma_f16(tmem, dbh, ph, kIdKM, (h > 0 || kk > 0) ? 1u : 0u);
+        mma_f16(tmem, dbh, pl, kIdKM, 1u);
+        mma_f16(tmem, dbl, ph, kIdKM, 1u);
+      }
+      mma_commit(&bar[h]);
     }
-    mma_commit(bar);
   }
-  const bool ok = mbar_wait(bar, 0, abort_flag, a.status, a.wait_ns);
+  ok = mbar_wait(&bar[1], 0, abort_flag, a.status, a.wait_ns) && ok;
   tc_fence_after();
-  if (ok) {
+
+  // ---------------- C out: warp q < 4 reads TMEM lanes (rows of C) 32 q..
+  if (ok && warp < 4) {
+    const int i = warp * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
     float4* cd = reinterpret_cast<float4*>(a.C + off);
 #pragma unroll 1
-    for (int cc = 0; cc < 4; ++cc) {
-      const int j0 = hc * 64 + cc * 16;
+    for (int j0 = 0; j0 < D; j0 += 16) {
       uint32_t v[16];
-      tmem_ld16(tl + kAccC + j0, v);
+      tmem_ld16(tl + j0, v);
       tmem_ld_wait();
 #pragma unroll
       for (int t = 0; t < 4; ++t)
-        cd[(j0 / 4 + t) * D + ri] = make_float4(__uint_as_float(v[4 * t]), __uint_as_float(v[4 * t + 1]),
-                                                __uint_as_float(v[4 * t + 2]), __uint_as_float(v[4 * t + 3]));
+        cd[(j0 / 4 + t) * D + i] = make_float4(__uint_as_float(v[4 * t]), __uint_as_float(v[4 * t + 1]),
+                                               __uint_as_float(v[4 * t + 2]), __uint_as_float(v[4 * t + 3]));
     }
   }
 
-  // ---------------- teardown: the MMA must be complete before TMEM is freed
+  // ---------------- teardown: the MMAs must be complete before TMEM is freed
   tc_fence_before();
   __syncthreads();
-  if (tid == 0 && *abort_flag) mbar_wait(bar, 0, nullptr, a.status, a.wait_ns);
+  if (tid == 0 && *abort_flag) {
+    mbar_wait(&bar[0], 0, nullptr, a.status, a.wait_ns);
+    mbar_wait(&bar[1], 0, nullptr, a.status, a.wait_ns);
+  }
   // Every thread's C_t and M_t stores precede the barrier above: publish the slot.
-  if (tid == 0 && ok && a.ready != nullptr) {
+  if (tid == 0 && ok && !*abort_flag && a.ready != nullptr) {
     __threadfence();
     flag_release_gpu(a.ready + (long long)bh * (a.T - 1) + slot, 1u);
   }
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -372,11 +427,22 @@ cudaError_t launch_solve_tc(const Problem& p, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  SolveArgs a{p.B, p.H, p.T, p.ready, p.A, p.Bm, p.alpha, p.M, p.C, static_cast<uint8_t*>(p.Msplit), p.status,
-              p.spin_limit};
+  SolveArgs a{p.B, p.H, p.T, p.ready, p.gready, p.A, p.Bm, p.alpha, p.M, p.C, static_cast<uint8_t*>(p.Msplit),
+              p.status, p.spin_limit};
   const long long n = (long long)p.B * p.H * (p.T - 1);
-  solve_tc_kernel<<<(unsigned)n, kThreads, kSmemBytes, s>>>(a);
-  return cudaGetLastError();
+  // After the tensor-core statistics kernel, launch as its programmatic
+  // dependent: CTAs start on the SMs its finished CTAs leave.
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3((unsigned)n);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.gready != nullptr ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, solve_tc_kernel, a);
 }
 
 }  // namespace vda

@@ -95,8 +95,9 @@ Layout make_layout(const vda_config& c) {
   const size_t d = (size_t)d_of(c), BH = (size_t)c.B * c.H;
   const size_t esz = c.dtype == VDA_BF16 ? 2 : 4;
   const bool prep = (c.flags & VDA_PREP_CONV) != 0;
-  // Status word (+ padding), then the [B,H,T-1] uint32 slot-ready words at byte 256.
-  L.bytes[VDA_REGION_STATUS] = 256 + align_up(BH * (c.T - 1) * 4, 256);
+  // Status word (+ padding), then at byte 256 the [B,H,T-1] uint32 slot-ready
+  // words of the solve, then those of the statistics kernel.
+  L.bytes[VDA_REGION_STATUS] = 256 + 2 * align_up(BH * (c.T - 1) * 4, 256);
   L.bytes[VDA_REGION_A] = BH * (c.T - 1) * d * d * 4;
   L.bytes[VDA_REGION_B] = BH * (c.T - 1) * d * d * 4;
   L.bytes[VDA_REGION_M] = BH * (c.T - 1) * d * d * 4;
@@ -327,16 +328,20 @@ vda_status vda_prepare(vda_ctx* ctx, const void* Q, const void* K, const void* V
     st = run_kernel(ctx, K_PREP_TEXT, s, [&] { return launch_prep_text(p, K_txt, V_txt, s); });
     if (st != VDA_OK) return st;
   }
-  if (!use_simt_only(c) && gram_tc_supported(p))
+  const bool gram_tc = !use_simt_only(c) && gram_tc_supported(p);
+  const bool sweep_tc = !use_simt_only(c) && solve_tc_supported(p) && !(c.flags & VDA_SOLVE_CHOLESKY);
+  // Per-slot ready words let the sweep solve overlap the statistics kernel's
+  // last units, and the frame scan the solve's last CTAs.
+  const size_t words = align_up((size_t)p.B * p.H * (p.T - 1) * 4, 256) / 4;
+  if (gram_tc && sweep_tc) p.gready = p.status + 64 + words;
+  if (gram_tc)
     st = run_kernel(ctx, K_GRAM_TC, s, [&] { return launch_gram_tc(p, s); });
   else
     st = run_kernel(ctx, K_GRAM_SIMT, s, [&] { return launch_gram_simt(p, s); });
   if (st != VDA_OK) return st;
   if (!use_simt_only(c) && solve_tc_supported(p) && (c.flags & VDA_SOLVE_CHOLESKY))
     st = run_kernel(ctx, K_SOLVE_CHOL_TC, s, [&] { return launch_solve_chol_tc(p, s); });
-  else if (!use_simt_only(c) && solve_tc_supported(p)) {
-    // The sweep solve publishes per-slot ready words, so the frame scan may
-    // start on the slots finished while its last CTAs still run.
+  else if (sweep_tc) {
     p.ready = p.status + 64;
     st = run_kernel(ctx, K_SOLVE_TC, s, [&] { return launch_solve_tc(p, s); });
   }
