@@ -136,15 +136,21 @@ def kernel_flops(name: str, cfg) -> float:
 # rather than by HBM streaming: their roofline is the bf16 tensor peak.
 TENSOR_BOUND = ("solve_chol_tc", "solve_simt")
 
-# Kernels whose time is set by fp32 FMAs on the CUDA cores. The symmetric sweep
-# applies every pivot's rank-1 update to the whole d x d matrix: d^3 FMAs per
-# slot. Peak: 148 SMs x 128 fp32 lanes x 2 flop per FMA x the SM clock.
-ALU_BOUND = ("solve_tc",)
+# Kernels whose time is set by fp32 FMAs on the CUDA cores. The sweep of a
+# d x d matrix applies every pivot's rank-1 update to the whole matrix: d^3 FMAs
+# per slot (the kernel exploits symmetry and executes about half of them). The
+# separable conv prep takes a 5x5 spatial sum of every input frame and a 5-tap
+# temporal sum per output: (25 T / (T-2) + 5) FMAs per prepared K or V value.
+# Peak: 148 SMs x 128 fp32 lanes x 2 flop per FMA x the SM clock.
+ALU_BOUND = ("solve_tc", "prep_video")
 
 
 def kernel_alu_flops(name: str, cfg) -> float:
     if name == "solve_tc":
         return cfg.B * cfg.H * (cfg.T - 1) * 2 * cfg.d ** 3
+    if name == "prep_video":
+        F = cfg.T - 2
+        return cfg.B * cfg.H * 2 * F * cfg.U * cfg.d * 2 * (25 * cfg.T / F + 5)
     return 0.0
 
 
