@@ -59,6 +59,15 @@ def load_peaks():
 # Whether the tensor-core scan runs over composed chunk maps (VDA_SCAN_CHUNKED)
 # or frame by frame (the default); set from --scan.
 SCAN_CHUNKED = False
+# Whether the Cholesky solve is selected (VDA_SOLVE_CHOLESKY); set from --solve.
+SOLVE_CHOLESKY = False
+
+
+def inject_in_scan(cfg) -> bool:
+    """Whether the frame scan forms the injections itself, (S Diag(alpha_t) + B_t) P_t,
+    so that the sweep solve writes P_t's images and no C_t for frames."""
+    from frame_level_delta_b200 import vda as V
+    return "inject=scan" in V.describe(V.make_config(cfg, cholesky=SOLVE_CHOLESKY, chunked=SCAN_CHUNKED))
 
 
 def composed_chunks(cfg):
@@ -83,6 +92,8 @@ def kernel_bytes(name: str, cfg) -> float:
         return BH * ((F * U + L) * (2 * d * esz + 4) + 2 * NS * dd4)
     if name == "solve_simt":
         return BH * (4 * NS * dd4 + F * d * 4)
+    if name == "solve_tc" and inject_in_scan(cfg):  # A read, P's hi/lo images written; B, C of the text slot
+        return BH * (NS * dd4 + F * dd4 + 2 * dd4)
     if name in ("solve_tc", "solve_chol_tc"):  # A, B, alpha read; C (fp32) and M's hi/lo operand images written
         return BH * (3 * NS * dd4 + F * dd4 + F * d * 4)
     if name == "scan_tc":  # per step: a (chunk) map's hi/lo images + its C; S_T; readout states
@@ -90,7 +101,8 @@ def kernel_bytes(name: str, cfg) -> float:
             steps = 2 * (J - 2)
         else:
             steps = max(0, c * (J - 2) - 1) + max(0, (T - 2) - 2 * c + 1)
-        return BH * (steps * 2 * dd4 + 2 * dd4 + 2 * J * dd4)
+        alpha = steps * d * 4 if inject_in_scan(cfg) else 0  # per step: P images + B rows + alpha
+        return BH * (steps * 2 * dd4 + alpha + 2 * dd4 + 2 * J * dd4)
     if name == "compose_tc":  # per frame of a composed chunk: M images + C; per chunk: map + C out
         ch = composed_chunks(cfg)
         return BH * (sum(ch) * 2 * dd4 + len(ch) * 2 * dd4)
@@ -117,6 +129,8 @@ def kernel_flops(name: str, cfg) -> float:
     F, NS, J = T - 2, T - 1, cfg.J
     if name.startswith("gram"):
         return B * H * (F * U + L) * 4 * d * d
+    if name == "solve_tc" and inject_in_scan(cfg):  # the inverse d^3 per slot; C = B P for S_T only
+        return B * H * (NS * d ** 3 + 2 * d ** 3)
     if name.startswith("solve"):  # Cholesky d^3/3, L^-1 d^3/3, P d^3/3, C = B P 2 d^3
         return B * H * NS * 3 * d ** 3
     if name == "compose_tc":  # two d x d x d products per absorbed frame
@@ -395,8 +409,9 @@ def main():
     inp_cpu = make_inputs(cfg, seed=cfg.seed + rank)
     inp_host = {k: v.pin_memory() for k, v in inp_cpu.items()}
     inp_dev = {k: v.to(dev, non_blocking=True) for k, v in inp_host.items()}
-    global SCAN_CHUNKED
+    global SCAN_CHUNKED, SOLVE_CHOLESKY
     SCAN_CHUNKED = args.scan == "chunked"
+    SOLVE_CHOLESKY = args.solve == "cholesky"
     lib = V.VDA(cfg, device=dev, cholesky=args.solve == "cholesky", chunked=SCAN_CHUNKED)
     O = lib.new_output()
     stream = torch.cuda.current_stream(dev)

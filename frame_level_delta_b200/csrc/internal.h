@@ -55,6 +55,9 @@ struct Problem {
   // for the sweep solve, launched to overlap that kernel's last units. nullptr
   // when the statistics kernel that ran does not raise them.
   uint32_t* gready;
+  // 1 when the sweep solve writes P_t's images (not M_t's, and no C_t for
+  // frames) because the frame scan forms S Diag(alpha_t) + B_t itself.
+  int pform;
   unsigned long long spin_limit;  // wall-time bound (ns) of every device-side wait
 };
 

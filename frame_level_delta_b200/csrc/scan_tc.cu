@@ -33,7 +33,9 @@ constexpr int D = 128;
 constexpr int kThreads = 320;  // copy warp, MMA warp, eight epilogue warps
 constexpr int kImg = D * D * 2;           // one bf16 operand image
 constexpr int kMBuf = 2 * kImg;           // hi + lo images of one M_t
-constexpr int kBarOff = 2 * kMBuf;        // barriers after the two M buffers
+constexpr int kARing = 4;                 // pform: alpha of the frames two steps ahead
+constexpr int kAOff = 2 * kMBuf;          // pform: alpha ring (kARing x D floats)
+constexpr int kBarOff = kAOff + kARing * D * 4;  // barriers after the two M buffers and the alpha ring
 constexpr int kSmemUsed = kBarOff + 128 + 1024;
 // Launched while the solve's last CTAs run, a scan CTA must not share an SM
 // with one (67 KB of shared memory each): it would wait in tcgen05.alloc for
@@ -53,6 +55,13 @@ struct ScanArgs {
   const uint8_t* CMi; // [B,H,2,J] x (hi, lo) composed chunk transitions
   const float* CC;    // [B,H,2,J,D,D] composed chunk injections
   const uint32_t* ready;  // [B,H,T-1] slot-ready words to acquire first, or nullptr
+  // Injection form. 0: the step operands are M_t = Diag(alpha_t) P_t and the
+  // injections C_t = B_t P_t. 1: the operands are P_t and the epilogue forms the
+  // next product's left factor S Diag(alpha_t) + B_t itself, since
+  // S M_t + C_t = (S Diag(alpha_t) + B_t) P_t; C_t is never materialised.
+  int pform;
+  const float* Bm;     // [B,H,T-1,D,D] B_t (pform)
+  const float* alpha;  // [B,H,T,D] (pform)
   float* Sf;
   float* Sr;
   uint32_t* status;
@@ -94,12 +103,14 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = sm100::align_smem_1024(smem_raw);
   uint8_t* sM = smem;           // [2][hi, lo]
+  const float* sA = reinterpret_cast<const float*>(smem + kAOff);  // [kARing][D]
   uint64_t* mfull = reinterpret_cast<uint64_t*>(smem + kBarOff);
   uint64_t* mempty = mfull + 2;
   uint64_t* tfull = mempty + 2;
   uint64_t* sready = tfull + 1;  // [4]: K-chunk q (state columns 32q..32q+31) of the next image written
   uint64_t* drain = sready + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* afull = drain + 1;  // [kARing] pform: alpha of step st in buffer st % kARing
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(afull + kARing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // Slots whose ready word the copy thread has acquired: 1 = slot 0 (S_T), then
   // st + 2 once step st's slot is.
@@ -122,6 +133,13 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
     if (a.chunked) return a.CC + (((long long)bh * 2 + dir) * J + (dir == 0 ? st : J - 1 - st)) * (long long)D * D;
     return a.C + (slots + (dir == 0 ? f_first + st : f_first - st)) * (long long)D * D;
   };
+  // Frame mode with pform: B_t and alpha_t of step st's frame.
+  auto step_b = [&](int st) -> const float* {
+    return a.Bm + (slots + (dir == 0 ? f_first + st : f_first - st)) * (long long)D * D;
+  };
+  auto step_alpha = [&](int st) -> const float* {
+    return a.alpha + ((long long)bh * T + (dir == 0 ? f_first + st : f_first - st)) * D;
+  };
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -131,6 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
     mbar_init(tfull, 1);
     for (int q = 0; q < 4; ++q) mbar_init(&sready[q], 8);
     mbar_init(drain, 1);
+    for (int r = 0; r < kARing; ++r) mbar_init(&afull[r], 1);
     *abort_flag = 0;
     *cgot = 0;
     fence_mbar_init();
@@ -144,11 +163,17 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   int issued = 0;
+  int aissued = 0;  // alpha copies issued (steps 0 .. aissued - 1)
 
   if (warp == 0) {
     if (lane == 0) {
       bool go = a.ready == nullptr || flag_wait_gpu(a.ready + slots, 1u, abort_flag, a.status, a.wait_ns);
       if (go) smem_release_u32(cgot, 1u);
+      for (int st = 0; go && a.pform && st < 2 && st < nsteps; ++st) {  // alpha is an input: no slot to wait for
+        mbar_arrive_expect_tx(&afull[st], D * 4);
+        bulk_load(smem + kAOff + st * D * 4, step_alpha(st), D * 4, &afull[st]);
+        aissued = st + 1;
+      }
       for (int st = 0; go && st < nsteps; ++st) {
         const int s = st & 1;
         // Acquire the slot before anything reads it: ahead of the wait for the
@@ -162,10 +187,26 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
         if (!mbar_wait(&mempty[s], ((st >> 1) & 1) ^ 1, abort_flag, a.status, a.wait_ns)) break;
         mbar_arrive_expect_tx(&mfull[s], kMBuf);
         const uint8_t* src = step_img(st);
-        // The step's injection rows are read by the epilogue threads with plain
-        // loads: bring them into L2 now, about two steps ahead.
-        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(step_c(st)), "r"((uint32_t)(D * D * 4))
-                     : "memory");
+        // alpha two steps ahead: its buffer's previous frame (st - 2) was read by
+        // the epilogue before it released the operand of step st - 2, whose MMA
+        // freed the image buffer waited for above.
+        if (a.pform && st + 2 < nsteps) {
+          const int r = (st + 2) % kARing;
+          mbar_arrive_expect_tx(&afull[r], D * 4);
+          bulk_load(smem + kAOff + r * D * 4, step_alpha(st + 2), D * 4, &afull[r]);
+          aissued = st + 3;
+        }
+        // The injection rows the epilogue reads with plain loads (C_t of this
+        // step, or B_t of this and the next step under pform): into L2 now.
+        if (!a.pform) {
+          asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(step_c(st)), "r"((uint32_t)(D * D * 4))
+                       : "memory");
+        } else {
+          // The epilogue of step st reads B of step st + 1: fetch two steps ahead.
+          for (int u = st == 0 ? 0 : st + 2; u <= st + 2 && u < nsteps; ++u)
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(step_b(u)), "r"((uint32_t)(D * D * 4))
+                         : "memory");
+        }
         bulk_load(sM + s * kMBuf, src, kImg, &mfull[s]);
         bulk_load(sM + s * kMBuf + kImg, src + kImg, kImg, &mfull[s]);
         issued = st + 1;
@@ -219,9 +260,27 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
       for (int t = 0; t < n / 4; ++t)
         d4[(col0 / 4 + t) * D + i] = make_float4(x[4 * t], x[4 * t + 1], x[4 * t + 2], x[4 * t + 3]);
     };
+    // x (16 state columns col..) <- x Diag(alpha) + B, row i: a pform operand
+    // (alpha from shared memory).
+    auto next_operand = [&](float* x, const float* bsrc, const float* al, int col0) {
+      const float4* b4 = reinterpret_cast<const float4*>(bsrc);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float4 w = b4[(col0 / 4 + t) * D + i];
+        const float4 g = reinterpret_cast<const float4*>(al + col0)[t];
+        x[4 * t] = fmaf(x[4 * t], g.x, w.x);
+        x[4 * t + 1] = fmaf(x[4 * t + 1], g.y, w.y);
+        x[4 * t + 2] = fmaf(x[4 * t + 2], g.z, w.z);
+        x[4 * t + 3] = fmaf(x[4 * t + 3], g.w, w.w);
+      }
+    };
     // Initial state S_T / 2: readout states of the chunks that see no frame of
     // this direction, and the first operand image.
-    const bool live = smem_wait_geq(cgot, 1u, abort_flag, a.status, a.wait_ns);
+    // Under pform the first operand is S_T/2 Diag(alpha) + B of the first frame:
+    // its slot must be acquired too.
+    bool live = smem_wait_geq(cgot, (a.pform && nsteps > 0) ? 2u : 1u, abort_flag, a.status, a.wait_ns);
+    // ... and its alpha, copied with the first frame's images.
+    if (live && a.pform && nsteps > 0) live = mbar_wait(&afull[0], 0, abort_flag, a.status, a.wait_ns);
     if (live) {
       const float4* st0 = reinterpret_cast<const float4*>(a.C + slots * (long long)D * D);
       float4 row[kCols / 4];  // all of this warp's columns first: one load latency
@@ -240,6 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
         }
         for (int j = 0; j < J; ++j)
           if (dir == 0 ? (c * (j - 1) - 1 <= 0) : (c * (j + 2) >= T - 1)) store_row(j, x, col, 16);
+        if (a.pform && nsteps > 0) next_operand(x, step_b(0), sA, col);
         uint32_t hi[8], lo[8];
         split16(x, hi, lo);
         tmem_st8(tl + kShi + col / 2, hi);
@@ -253,18 +313,27 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
     }
     for (int st = 0; live && st < nsteps; ++st) {
       const int f = dir == 0 ? f_first + st : f_first - st;
-      if (!smem_wait_geq(cgot, (uint32_t)st + 2u, abort_flag, a.status, a.wait_ns)) break;
-      // Prefetch this warp's columns of the injection's row i while the MMAs run.
+      // Under pform the epilogue of step st forms the operand of step st + 1.
+      const bool nxt = a.pform && st + 1 < nsteps;
+      if (!smem_wait_geq(cgot, (uint32_t)st + (nxt ? 3u : 2u), abort_flag, a.status, a.wait_ns)) break;
+      // Prefetch this warp's columns of the injection's row i while the MMAs run:
+      // C_t of this step, or B_t of the next step under pform.
       float crow[kCols];
-      const float4* csrc = reinterpret_cast<const float4*>(step_c(st));
+      if (!a.pform || nxt) {
+        const float4* csrc = reinterpret_cast<const float4*>(a.pform ? step_b(st + 1) : step_c(st));
 #pragma unroll
-      for (int cc = 0; cc < kCols / 16; ++cc)
+        for (int cc = 0; cc < kCols / 16; ++cc)
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const float4 v = csrc[(col_of(cc) / 4 + t) * D + i];
-          crow[16 * cc + 4 * t] = v.x; crow[16 * cc + 4 * t + 1] = v.y;
-          crow[16 * cc + 4 * t + 2] = v.z; crow[16 * cc + 4 * t + 3] = v.w;
-        }
+          for (int t = 0; t < 4; ++t) {
+            const float4 v = csrc[(col_of(cc) / 4 + t) * D + i];
+            crow[16 * cc + 4 * t] = v.x; crow[16 * cc + 4 * t + 1] = v.y;
+            crow[16 * cc + 4 * t + 2] = v.z; crow[16 * cc + 4 * t + 3] = v.w;
+          }
+      }
+      // alpha of the next step's frame, copied two steps ahead.
+      if (nxt && !mbar_wait(&afull[(st + 1) % kARing], ((st + 1) / kARing) & 1, abort_flag, a.status, a.wait_ns))
+        break;
+      const float* anext = nxt ? sA + ((st + 1) % kARing) * D : nullptr;
       if (!mbar_wait(tfull, st & 1, abort_flag, a.status, a.wait_ns)) break;
       tc_fence_after();
       int jout = -1;
@@ -275,18 +344,37 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
       } else {
         if (f % c == 0 && f / c - 2 >= 0) jout = f / c - 2;
       }
-      float xs[kCols];  // the new state's half row, stored once the MMAs have it
 #pragma unroll
       for (int c16 = 0; c16 < kCols / 16; ++c16) {
         const int col = col_of(c16);
+        // pform: this group's alpha, read while the accumulator columns load.
+        float4 g[4];
+        if (nxt) {
+#pragma unroll
+          for (int t = 0; t < 4; ++t) g[t] = reinterpret_cast<const float4*>(anext + col)[t];
+        }
         uint32_t v[16];
         tmem_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(st & 1) * 128 + col, v);
         tmem_ld_wait();
+        // The new state's 16 columns: the product plus C_t, or under pform the
+        // product itself. A readout state is stored as it is formed (the stores
+        // do not hold up the operand).
         float x[16];
 #pragma unroll
-        for (int t = 0; t < 16; ++t) x[t] = __uint_as_float(v[t]) + crow[c16 * 16 + t];
+        for (int t = 0; t < 16; ++t) x[t] = __uint_as_float(v[t]) + (a.pform ? 0.f : crow[c16 * 16 + t]);
+        if (jout >= 0) store_row(jout, x, col, 16);
+        if (a.pform) {
+          // The next operand is S Diag(alpha) + B.
+          if (nxt) {
 #pragma unroll
-        for (int t = 0; t < 16; ++t) xs[c16 * 16 + t] = x[t];
+            for (int t = 0; t < 4; ++t) {
+              x[4 * t] = fmaf(x[4 * t], g[t].x, crow[c16 * 16 + 4 * t]);
+              x[4 * t + 1] = fmaf(x[4 * t + 1], g[t].y, crow[c16 * 16 + 4 * t + 1]);
+              x[4 * t + 2] = fmaf(x[4 * t + 2], g[t].z, crow[c16 * 16 + 4 * t + 2]);
+              x[4 * t + 3] = fmaf(x[4 * t + 3], g[t].w, crow[c16 * 16 + 4 * t + 3]);
+            }
+          }
+        }
         uint32_t hi[8], lo[8];
         split16(x, hi, lo);
         tmem_st8(tl + kShi + col / 2, hi);
@@ -297,9 +385,6 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
         __syncwarp();
         if (lane == 0) mbar_arrive(&sready[col >> 5]);
       }
-      // The readout state leaves while the next step's MMAs run.
-      if (jout >= 0)
-        for (int cc = 0; cc < kCols / 16; ++cc) store_row(jout, xs + 16 * cc, col_of(cc), 16);
     }
   }
 
@@ -310,6 +395,11 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
       int last = -1;
       for (int st = s; st < issued; st += 2) last = st;
       if (last >= 0) mbar_wait(&mfull[s], (last >> 1) & 1, nullptr, a.status, a.wait_ns);
+    }
+    for (int r = 0; r < kARing; ++r) {
+      int last = -1;
+      for (int st = r; st < aissued; st += kARing) last = st;
+      if (last >= 0) mbar_wait(&afull[r], (last / kARing) & 1, nullptr, a.status, a.wait_ns);
     }
   }
   if (warp == 1) {
@@ -335,8 +425,8 @@ cudaError_t launch_scan_tc(const Problem& p, cudaStream_t s, bool chunked) {
   // frame scan waits on the slot-ready words, and only it overlaps the solve.
   const bool overlap = !chunked && p.ready != nullptr;
   ScanArgs a{p.B, p.H, p.T, p.c, p.J, chunked ? 1 : 0, p.C, static_cast<const uint8_t*>(p.Msplit),
-             static_cast<const uint8_t*>(p.CMi), p.CC, overlap ? p.ready : nullptr, p.Sf, p.Sr, p.status,
-             p.spin_limit};
+             static_cast<const uint8_t*>(p.CMi), p.CC, overlap ? p.ready : nullptr,
+             (!chunked && p.pform) ? 1 : 0, p.Bm, p.alpha, p.Sf, p.Sr, p.status, p.spin_limit};
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(p.B * p.H, 2);
   cfg.blockDim = dim3(kThreads);

@@ -58,6 +58,7 @@ struct SolveArgs {
   uint8_t* Msplit;
   uint32_t* status;
   unsigned long long wait_ns;
+  int pform;  // frames write P_t's images and no C_t (the scan forms the injection)
 };
 
 // Byte offset of element (row, col) in a bf16 image with 128-byte rows of 64
@@ -191,6 +192,9 @@ __global__ void __launch_bounds__(kThreads, 3) solve_tc_kernel(const SolveArgs a
   key_slot(blockIdx.x, a.B * a.H, a.T - 1, bh, slot);
   const long long off = ((long long)bh * (a.T - 1) + slot) * (long long)D * D;
   const bool active = tid < kTiles;
+  // C = B P on tcgen05: for every slot, or only for the text slot (S_T) when
+  // the frame scan forms the frames' injections itself.
+  const bool mma = !a.pform || slot == 0;
   int ti = -1, tj = -1;
   if (active) tile_of(tid, ti, tj);
 
@@ -206,13 +210,15 @@ __global__ void __launch_bounds__(kThreads, 3) solve_tc_kernel(const SolveArgs a
       flag_wait_gpu(a.gready + (long long)bh * (a.T - 1) + slot, kGramReadyCount, abort_flag, a.status, a.wait_ns);
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, kTmemCols);
+    if (mma) tmem_alloc(tmem_slot, kTmemCols);
+    // Also when not allocating: until a CTA gives up its permit, no other CTA
+    // of the grid is placed on the SM.
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = mma ? *tmem_slot : 0u;
   // Let the scan kernel launch once every solve CTA holds its TMEM (the scan
   // then waits on the slot-ready words, not on the end of this grid, and never
   // competes with a solve CTA for TMEM columns).
@@ -265,7 +271,10 @@ __global__ void __launch_bounds__(kThreads, 3) solve_tc_kernel(const SolveArgs a
     if (slot > 0) {
       const float* al = a.alpha + ((long long)bh * a.T + slot) * D;
       float ar[8], ac[8];
-      {
+      if (a.pform) {  // the images of P itself
+#pragma unroll
+        for (int r = 0; r < 8; ++r) ar[r] = ac[r] = 1.f;
+      } else {
         const float4 p0 = reinterpret_cast<const float4*>(al + 8 * ti)[0];
         const float4 p1 = reinterpret_cast<const float4*>(al + 8 * ti)[1];
         const float4 q0 = reinterpret_cast<const float4*>(al + 8 * tj)[0];
@@ -304,6 +313,7 @@ __global__ void __launch_bounds__(kThreads, 3) solve_tc_kernel(const SolveArgs a
 
   // ---------------- C = B P in two halves of the contraction index k
   bool ok = true;
+  if (mma) {
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     if (h == 1) {
@@ -377,11 +387,12 @@ __global__ void __launch_bounds__(kThreads, 3) solve_tc_kernel(const SolveArgs a
       mma_commit(&bar[h]);
     }
   }
-  ok = mbar_wait(&bar[1], 0, abort_flag, a.status, a.wait_ns) && ok;
+  }
+  if (mma) ok = mbar_wait(&bar[1], 0, abort_flag, a.status, a.wait_ns) && ok;
   tc_fence_after();
 
   // ---------------- C out: warp q < 4 reads TMEM lanes (rows of C) 32 q..
-  if (ok && warp < 4) {
+  if (mma && ok && warp < 4) {
     const int i = warp * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
     float4* cd = reinterpret_cast<float4*>(a.C + off);
@@ -400,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 3) solve_tc_kernel(const SolveArgs a
   // ---------------- teardown: the MMAs must be complete before TMEM is freed
   tc_fence_before();
   __syncthreads();
-  if (tid == 0 && *abort_flag) {
+  if (mma && tid == 0 && *abort_flag) {
     mbar_wait(&bar[0], 0, nullptr, a.status, a.wait_ns);
     mbar_wait(&bar[1], 0, nullptr, a.status, a.wait_ns);
   }
@@ -410,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 3) solve_tc_kernel(const SolveArgs a
     flag_release_gpu(a.ready + (long long)bh * (a.T - 1) + slot, 1u);
   }
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 0 && mma) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -428,7 +439,7 @@ cudaError_t launch_solve_tc(const Problem& p, cudaStream_t s) {
     attr_set = true;
   }
   SolveArgs a{p.B, p.H, p.T, p.ready, p.gready, p.A, p.Bm, p.alpha, p.M, p.C, static_cast<uint8_t*>(p.Msplit),
-              p.status, p.spin_limit};
+              p.status, p.spin_limit, p.pform};
   const long long n = (long long)p.B * p.H * (p.T - 1);
   // After the tensor-core statistics kernel, launch as its programmatic
   // dependent: CTAs start on the SMs its finished CTAs leave.

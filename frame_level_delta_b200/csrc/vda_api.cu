@@ -242,6 +242,16 @@ vda_status vda_workspace_region(const vda_config* cfg, int region, size_t* offse
 
 const char* vda_last_error(const vda_ctx* ctx) { return ctx ? ctx->err.c_str() : ""; }
 
+// Whether the sweep solve leaves the frames' injections to the tensor-core
+// frame scan (S M_t + C_t = (S Diag(alpha_t) + B_t) P_t): writes P_t's images
+// and no C_t. Not with the chunked scan, which composes M_t and C_t.
+static bool pform_of(const vda_config& c, const Problem& p) {
+  if (use_simt_only(c) || !solve_tc_supported(p) || !scan_tc_supported(p)) return false;
+  if (c.flags & VDA_SOLVE_CHOLESKY) return false;
+  const bool chunked = (c.flags & VDA_SCAN_CHUNKED) && c.chunk > 1 && J_of(c) >= 3;
+  return !chunked;
+}
+
 vda_status vda_describe(const vda_config* cfg, const char** text) {
   if (!text) return VDA_ERR_INVALID_ARG;
   vda_status st = check_config(cfg, nullptr);
@@ -254,10 +264,12 @@ vda_status vda_describe(const vda_config* cfg, const char** text) {
   const bool g = !simt && gram_tc_supported(p), r = !simt && readout_tc_supported(p);
   const bool v = !simt && solve_tc_supported(p), n = !simt && scan_tc_supported(p);
   const bool chol = v && (cfg->flags & VDA_SOLVE_CHOLESKY);
-  static char table[2][2][2][2][2][96];
-  char* t = table[g][v][chol][n][r];
-  std::snprintf(t, 96, "gram=%s solve=%s scan=%s readout=%s", g ? "tcgen05" : "simt",
-                v ? (chol ? "tcgen05-cholesky" : "tcgen05") : "simt", n ? "tcgen05" : "simt", r ? "tcgen05" : "simt");
+  const bool pf = pform_of(*cfg, p);
+  static char table[2][2][2][2][2][2][112];
+  char* t = table[g][v][chol][n][r][pf];
+  std::snprintf(t, 112, "gram=%s solve=%s scan=%s readout=%s%s", g ? "tcgen05" : "simt",
+                v ? (chol ? "tcgen05-cholesky" : "tcgen05") : "simt", n ? "tcgen05" : "simt", r ? "tcgen05" : "simt",
+                pf ? " inject=scan" : "");
   *text = t;
   return VDA_OK;
 }
@@ -343,6 +355,7 @@ vda_status vda_prepare(vda_ctx* ctx, const void* Q, const void* K, const void* V
     st = run_kernel(ctx, K_SOLVE_CHOL_TC, s, [&] { return launch_solve_chol_tc(p, s); });
   else if (sweep_tc) {
     p.ready = p.status + 64;
+    p.pform = pform_of(c, p) ? 1 : 0;
     st = run_kernel(ctx, K_SOLVE_TC, s, [&] { return launch_solve_tc(p, s); });
   }
   else

@@ -177,7 +177,9 @@ typedef enum vda_region {
   VDA_REGION_M = 3,      /* float32 [B, H, T-1, d_k, d_k]; slot t = M_t (slot 0 unused); written by the
                             CUDA-core solve only: the tensor-core solves write M_t as the hi/lo images of
                             VDA_REGION_M_SPLIT, the form their scan reads */
-  VDA_REGION_C = 4,      /* float32 [B, H, T-1, d_v, d_k]; slot 0 = S_T, slot t = C_t */
+  VDA_REGION_C = 4,      /* float32 [B, H, T-1, d_v, d_k]; slot 0 = S_T, slot t = C_t. When vda_describe
+                            reports "inject=scan", only slot 0 is written: the tensor-core frame scan
+                            forms each step as (S Diag(alpha_t) + B_t) P_t and C_t never exists */
   VDA_REGION_S_FWD = 5,  /* float32 [B, H, J, d_v, d_k]; forward readout state of chunk j */
   VDA_REGION_S_REV = 6,  /* float32 [B, H, J, d_v, d_k]; reverse readout state of chunk j */
   VDA_REGION_K_PREP = 7, /* storage dtype [B, H, T, U, d]; prepared K (VDA_PREP_CONV only) */
@@ -188,7 +190,9 @@ typedef enum vda_region {
                               each in the swizzled shared-memory operand layout of the tensor-core
                               scan: element (i, j) at byte (j / 64) * d * 128 + i * 128 +
                               (((j % 64) / 8) XOR (i % 8)) * 16 + (j % 8) * 2 of its image
-                              (written by the tensor-core solves, unused otherwise) */
+                              (written by the tensor-core solves, unused otherwise). Under
+                              "inject=scan" the images hold P_t = (I + A_t)^-1 itself, and
+                              M_t = Diag(alpha_t) P_t */
   VDA_REGION_CHUNK_M = 12, /* bf16 [B, H, 2, J, 2, d*d]: per direction and chunk, the composed transition
                               of the chunk's frames (hi, lo operand images; identity for empty chunks) */
   VDA_REGION_CHUNK_C = 13, /* float32 [B, H, 2, J, d_v, d_k]: the composed injection of those frames */

@@ -39,10 +39,17 @@ def run_gpu(cfg, inp_cpu, force_simt=False, cholesky=False, chunked=False):
     torch.cuda.synchronize()
     assert lib.poll_device_status() == 0
     regions = {k: lib.region(k).detach().cpu().clone() for k in ("A", "B", "M", "C", "S_fwd", "S_rev")}
-    if "solve=tcgen05" in V.describe(lib.c):
-        # The tensor-core solves write M_t only as hi/lo operand images.
+    desc = V.describe(lib.c)
+    if "solve=tcgen05" in desc:
+        # The tensor-core solves write M_t only as hi/lo operand images; when the
+        # frame scan forms the injections itself they are P_t's images, and
+        # M_t = Diag(alpha_t) P_t.
         mi = lib.region("M_split").detach().cpu()
         regions["M"] = mi[:, :, :, 0] + mi[:, :, :, 1]
+        if "inject=scan" in desc:
+            al = inp_cpu["alpha"].float()[:, :, : cfg.T - 1]  # slot t <-> frame t
+            regions["M"] = regions["M"] * al[..., :, None]
+    regions["inject_scan"] = "inject=scan" in desc
     if cfg.prep_conv:
         regions["K_prep"] = lib.region("K_prep").float().cpu()
         regions["V_prep"] = lib.region("V_prep").float().cpu()
@@ -62,7 +69,8 @@ def staged_errors(cfg, regions, ref):
             upd("B", rel_fro(regions["B"][b, h, s], it["B"][s]))
         for t in range(1, cfg.T - 1):
             upd("M", rel_fro(regions["M"][b, h, t], it["M"][t]))
-            upd("C", rel_fro(regions["C"][b, h, t], it["C"][t]))
+            if not regions["inject_scan"]:  # otherwise C_t is never materialised
+                upd("C", rel_fro(regions["C"][b, h, t], it["C"][t]))
         upd("S_T", rel_fro(regions["C"][b, h, 0], it["S_T"]))
         for j in range(cfg.J):
             upd("S_fwd", rel_fro(regions["S_fwd"][b, h, j], it["S_fwd"][j]))

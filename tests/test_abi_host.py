@@ -130,6 +130,12 @@ def test_status_strings_and_describe():
     assert "gram=" in text and "readout=" in text
     assert "tcgen05" not in text  # fp32 storage always takes the CUDA-core path
     assert "tcgen05" not in V.describe(V.make_config(CONFIGS["h3"], force_simt=True))
+    # The frame scan forms the injections (S Diag(alpha) + B) P itself after the
+    # sweep solve; the chunked scan and the Cholesky solve keep M_t and C_t.
+    assert "inject=scan" in V.describe(V.make_config(CONFIGS["h3"]))
+    assert "inject=scan" not in V.describe(V.make_config(CONFIGS["h3"], chunked=True))
+    assert "inject=scan" not in V.describe(V.make_config(CONFIGS["h3"], cholesky=True))
+    assert "inject=scan" not in V.describe(V.make_config(CONFIGS["small"]))  # d = 64: CUDA-core solve
 
 
 def test_region_view_undoes_column_quad_layout():
