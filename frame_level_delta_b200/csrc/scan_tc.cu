@@ -76,7 +76,9 @@ __device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
     const __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * q], x[2 * q + 1]);
     const float2 hf = __bfloat1622float2(hh);
     h[q] = hh;
-    l[q] = __floats2bfloat162_rn(x[2 * q] - hf.x, x[2 * q + 1] - hf.y);
+    // x - hi is exact in fp32; one packed add for the pair.
+    const float2 d = __fadd2_rn(make_float2(x[2 * q], x[2 * q + 1]), make_float2(-hf.x, -hf.y));
+    l[q] = __floats2bfloat162_rn(d.x, d.y);
   }
 }
 
@@ -268,10 +270,10 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
       for (int t = 0; t < 4; ++t) {
         const float4 w = b4[(col0 / 4 + t) * D + i];
         const float4 g = reinterpret_cast<const float4*>(al + col0)[t];
-        x[4 * t] = fmaf(x[4 * t], g.x, w.x);
-        x[4 * t + 1] = fmaf(x[4 * t + 1], g.y, w.y);
-        x[4 * t + 2] = fmaf(x[4 * t + 2], g.z, w.z);
-        x[4 * t + 3] = fmaf(x[4 * t + 3], g.w, w.w);
+        const float2 p0 = __ffma2_rn(make_float2(x[4 * t], x[4 * t + 1]), make_float2(g.x, g.y), make_float2(w.x, w.y));
+        const float2 p1 =
+            __ffma2_rn(make_float2(x[4 * t + 2], x[4 * t + 3]), make_float2(g.z, g.w), make_float2(w.z, w.w));
+        x[4 * t] = p0.x; x[4 * t + 1] = p0.y; x[4 * t + 2] = p1.x; x[4 * t + 3] = p1.y;
       }
     };
     // Initial state S_T / 2: readout states of the chunks that see no frame of
@@ -359,20 +361,30 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
         // The new state's 16 columns: the product plus C_t, or under pform the
         // product itself. A readout state is stored as it is formed (the stores
         // do not hold up the operand).
+        // (Packed fp32x2 arithmetic: the epilogue's instruction issue paces the scan.)
         float x[16];
+        if (!a.pform) {
 #pragma unroll
-        for (int t = 0; t < 16; ++t) x[t] = __uint_as_float(v[t]) + (a.pform ? 0.f : crow[c16 * 16 + t]);
+          for (int t = 0; t < 8; ++t) {
+            const float2 r = __fadd2_rn(make_float2(__uint_as_float(v[2 * t]), __uint_as_float(v[2 * t + 1])),
+                                        make_float2(crow[c16 * 16 + 2 * t], crow[c16 * 16 + 2 * t + 1]));
+            x[2 * t] = r.x;
+            x[2 * t + 1] = r.y;
+          }
+        } else {
+#pragma unroll
+          for (int t = 0; t < 16; ++t) x[t] = __uint_as_float(v[t]);
+        }
         if (jout >= 0) store_row(jout, x, col, 16);
-        if (a.pform) {
-          // The next operand is S Diag(alpha) + B.
-          if (nxt) {
+        if (nxt) {  // pform: the next operand is S Diag(alpha) + B
 #pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              x[4 * t] = fmaf(x[4 * t], g[t].x, crow[c16 * 16 + 4 * t]);
-              x[4 * t + 1] = fmaf(x[4 * t + 1], g[t].y, crow[c16 * 16 + 4 * t + 1]);
-              x[4 * t + 2] = fmaf(x[4 * t + 2], g[t].z, crow[c16 * 16 + 4 * t + 2]);
-              x[4 * t + 3] = fmaf(x[4 * t + 3], g[t].w, crow[c16 * 16 + 4 * t + 3]);
-            }
+          for (int t = 0; t < 4; ++t) {
+            const float* cr = crow + c16 * 16 + 4 * t;
+            const float2 p0 = __ffma2_rn(make_float2(x[4 * t], x[4 * t + 1]), make_float2(g[t].x, g[t].y),
+                                         make_float2(cr[0], cr[1]));
+            const float2 p1 = __ffma2_rn(make_float2(x[4 * t + 2], x[4 * t + 3]), make_float2(g[t].z, g[t].w),
+                                         make_float2(cr[2], cr[3]));
+            x[4 * t] = p0.x; x[4 * t + 1] = p0.y; x[4 * t + 2] = p1.x; x[4 * t + 3] = p1.y;
           }
         }
         uint32_t hi[8], lo[8];
