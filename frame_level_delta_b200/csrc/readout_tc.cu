@@ -133,8 +133,14 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// Fast division intrinsic: a few ulp, far below the bf16 rounding of the output.
-__device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
+// The hardware's approximate tanh (about 2^-11 relative error, below the bf16
+// rounding of the output): sigmoid(x) = (1 + tanh(x / 2)) / 2, one special-
+// function operation instead of an exponential and a reciprocal.
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 template <int D, bool GATE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -410,6 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (qnorm) scale = rsqrtf(qq + __uint_as_float(pq) + a.l2_eps);
         if constexpr (GATE) rn = rsqrtf(scale * scale * (ss + __uint_as_float(ps)) / D + a.rms_eps);
       }
+      const float hr = 0.5f * rn;
       // Output half row into registers: 16-byte chunk pair (2cc, 2cc+1) holds columns col0+16cc..+15.
       uint4 outs[kHalf / 8];
 #pragma unroll
@@ -432,10 +439,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint4 gv = gr[2 * cc + half];
             const __nv_bfloat162* ge = reinterpret_cast<const __nv_bfloat162*>(&gv);
 #pragma unroll
-            for (int k2 = 0; k2 < 4; ++k2) {
+            for (int k2 = 0; k2 < 4; ++k2) {  // rn * sigmoid(g) = hr + hr * tanh(g / 2), hr = rn / 2
               const float2 f = __bfloat1622float2(ge[k2]);
-              g8[2 * k2] = sigmoid_f(f.x) * rn;
-              g8[2 * k2 + 1] = sigmoid_f(f.y) * rn;
+              g8[2 * k2] = fmaf(hr, tanh_approx(0.5f * f.x), hr);
+              g8[2 * k2 + 1] = fmaf(hr, tanh_approx(0.5f * f.y), hr);
             }
           } else {
 #pragma unroll

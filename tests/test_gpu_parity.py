@@ -169,6 +169,36 @@ def test_repeated_runs_are_bitwise_identical():
     assert torch.equal(O1, O2)
 
 
+@pytest.mark.parametrize("chunked", [False, True])
+def test_interleaved_calls_on_overlapped_path(chunked):
+    """The d = 128 path runs the solve and the frame scan as overlapping kernels
+    that hand slots over through per-slot ready words (cleared by vda_prepare).
+    Repeated and interleaved calls - a second scan and readout after one
+    prepare, two prepares in a row, a readout on another stream after a
+    synchronise - must give the same output bit for bit and report no timeout."""
+    cfg = CONFIGS["h3"].with_(H=3, T=12, grid_h=6, grid_w=9, L=20)
+    inp = {k: v.cuda() for k, v in make_inputs(cfg).items()}
+    lib = V.VDA(cfg, chunked=chunked)
+    ref = lib.run(inp).clone()
+    O = lib.new_output()
+    lib.scan_bidir()
+    lib.readout(O)
+    torch.cuda.synchronize()
+    assert torch.equal(O, ref)
+    lib.prepare(inp)
+    lib.prepare(inp)
+    lib.scan_bidir()
+    lib.scan_bidir()
+    O.zero_()
+    side = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(side):
+        lib.readout(O, stream=side)
+    side.synchronize()
+    assert torch.equal(O, ref)
+    assert lib.poll_device_status() == 0
+
+
 def test_bounded_wait_reports_timeout_without_faulting():
     status = torch.zeros(4, dtype=torch.int32, device="cuda")
     assert V.selftest_bounded_wait(status, 2000) == 0
