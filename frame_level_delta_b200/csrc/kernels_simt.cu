@@ -102,70 +102,152 @@ __global__ void __launch_bounds__(256) gram_simt_kernel(Problem p) {
 }
 
 // ---------------------------------------------------------------------------
-// Frame solve: Cholesky I + A = L L^T, Y = L^-1, P = Y^T Y = (I + A)^-1,
-// M = Diag(alpha) P, C = B P. Slot 0 (text) writes only C = S_T.
-// Grid (T-1, H, B), 256 threads, 2 * D * (D+1) floats of shared memory.
+// Frame solve on the CUDA cores: P = (I + A)^-1 by the symmetric sweep
+// (Gauss-Jordan elimination without pivoting; I + A is symmetric positive
+// definite with every eigenvalue >= 1). Sweeping pivot k of a symmetric X:
+//   x_ij -= x_ik x_kj / x_kk  (i, j != k),  x_ik /= x_kk,  x_kj /= x_kk,  x_kk = -1 / x_kk,
+// and after all D pivots X = -P. Then M = Diag(alpha) P and C = B P in fp32.
+// Slot 0 (text) writes only C = S_T.
+// Grid (T-1, H, B); (D/8)^2 threads, each holding an 8 x 8 tile of X in
+// registers; the pivot row is published through a double-buffered shared
+// vector, one block barrier per pivot. Shared memory: the pivot vectors and P.
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(256) solve_simt_kernel(Problem p) {
-  constexpr int LD = D + 1;
+struct SweepCfg {
+  static constexpr int NT = D / 8;             // tile rows (and columns)
+  static constexpr int kThreads = NT * NT;
+  static constexpr int kPv = D + 4;            // floats per pivot buffer
+  static constexpr int kSmemFloats = 2 * kPv + D * D;
+};
+
+// The pivot vector in two halves (entries 8t..8t+3 of tile t at float4 t,
+// 8t+4..8t+7 at float4 D/8 + t): a warp's float4 reads of different tiles' entries
+// fall on consecutive words.
+template <int D, int row>
+__device__ __forceinline__ void sweep_publish(float* pv, const float (&x)[8][8], int ti, int tj) {
+  reinterpret_cast<float4*>(pv)[tj] = make_float4(x[row][0], x[row][1], x[row][2], x[row][3]);
+  reinterpret_cast<float4*>(pv + D / 2)[tj] = make_float4(x[row][4], x[row][5], x[row][6], x[row][7]);
+  if (ti == tj) pv[D] = 1.f / x[row][row];
+}
+
+// Pivot k = 8 K + s on the tile (ti, tj).
+template <int D, int s>
+__device__ __forceinline__ void sweep_simt_step(float (&x)[8][8], float* pv_all, int K, int ti, int tj) {
+  const float* v = pv_all + (s & 1) * SweepCfg<D>::kPv;
+  float* vn = pv_all + ((s + 1) & 1) * SweepCfg<D>::kPv;
+  const float4 r0 = reinterpret_cast<const float4*>(v)[ti], r1 = reinterpret_cast<const float4*>(v + D / 2)[ti];
+  const float4 c0 = reinterpret_cast<const float4*>(v)[tj], c1 = reinterpret_cast<const float4*>(v + D / 2)[tj];
+  const float inv = v[D];
+  const float vr[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+  const float vc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  float ur[8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) ur[r] = vr[r] * inv;  // x_ik / x_kk
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) x[r][c] = fmaf(-ur[r], vc[c], x[r][c]);
+  if (tj == K) {  // column k
+#pragma unroll
+    for (int r = 0; r < 8; ++r) x[r][s] = ur[r];
+  }
+  if (ti == K) {  // row k
+#pragma unroll
+    for (int c = 0; c < 8; ++c) x[s][c] = vc[c] * inv;
+    if (tj == K) x[s][s] = -inv;
+  }
+  // The next pivot is row s + 1 of tile row K, or row 0 of tile row K + 1.
+  if (s < 7) {
+    if (ti == K) sweep_publish<D, (s + 1) & 7>(vn, x, ti, tj);
+  } else {
+    if (ti == K + 1) sweep_publish<D, 0>(vn, x, ti, tj);
+  }
+  __syncthreads();
+}
+
+template <int D>
+__global__ void __launch_bounds__(SweepCfg<D>::kThreads) solve_simt_kernel(Problem p) {
+  using C = SweepCfg<D>;
   extern __shared__ float smem[];
-  float* X = smem;           // I + A, then L (lower), then P
-  float* Y = smem + D * LD;  // L^-1 (lower)
+  float* pv = smem;                // [2][kPv]
+  float* sP = smem + 2 * C::kPv;   // P, row-major [D][D]
   const int s = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, nt = blockDim.x;
+  const int tid = threadIdx.x, ti = tid / C::NT, tj = tid % C::NT;
   const long long off = slot_off(p, b, h, s);
-  const float* A = p.A + off;
-  for (int e = tid; e < D * D; e += nt) {
-    const int i = quad_row(D, e), j = quad_col(D, e);
-    X[i * LD + j] = A[e] + (i == j ? 1.f : 0.f);
+  // X = I + A: tile rows 8 ti.., columns 8 tj.. (column quads 2 tj, 2 tj + 1).
+  float x[8][8];
+  const float4* A4 = reinterpret_cast<const float4*>(p.A + off);
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int i = 8 * ti + r;
+    const float4 w0 = A4[(2 * tj) * D + i], w1 = A4[(2 * tj + 1) * D + i];
+    x[r][0] = w0.x; x[r][1] = w0.y; x[r][2] = w0.z; x[r][3] = w0.w;
+    x[r][4] = w1.x; x[r][5] = w1.y; x[r][6] = w1.z; x[r][7] = w1.w;
+  }
+  if (ti == tj) {
+#pragma unroll
+    for (int r = 0; r < 8; ++r) x[r][r] += 1.f;
+  }
+  if (ti == 0) sweep_publish<D, 0>(pv, x, ti, tj);
+  __syncthreads();
+#pragma unroll 1
+  for (int K = 0; K < C::NT; ++K) {
+    sweep_simt_step<D, 0>(x, pv, K, ti, tj);
+    sweep_simt_step<D, 1>(x, pv, K, ti, tj);
+    sweep_simt_step<D, 2>(x, pv, K, ti, tj);
+    sweep_simt_step<D, 3>(x, pv, K, ti, tj);
+    sweep_simt_step<D, 4>(x, pv, K, ti, tj);
+    sweep_simt_step<D, 5>(x, pv, K, ti, tj);
+    sweep_simt_step<D, 6>(x, pv, K, ti, tj);
+    sweep_simt_step<D, 7>(x, pv, K, ti, tj);
+  }
+  // P = -X into shared memory; M = Diag(alpha) P in column quads.
+  const float* alpha = p.alpha + (((long long)b * p.H + h) * p.T + s) * D;
+  float4* M4 = reinterpret_cast<float4*>(p.M + off);
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int i = 8 * ti + r;
+    const float4 q0 = make_float4(-x[r][0], -x[r][1], -x[r][2], -x[r][3]);
+    const float4 q1 = make_float4(-x[r][4], -x[r][5], -x[r][6], -x[r][7]);
+    reinterpret_cast<float4*>(sP + i * D + 8 * tj)[0] = q0;
+    reinterpret_cast<float4*>(sP + i * D + 8 * tj)[1] = q1;
+    if (s > 0) {
+      const float al = alpha[i];
+      M4[(2 * tj) * D + i] = make_float4(al * q0.x, al * q0.y, al * q0.z, al * q0.w);
+      M4[(2 * tj + 1) * D + i] = make_float4(al * q1.x, al * q1.y, al * q1.z, al * q1.w);
+    }
   }
   __syncthreads();
-  // Right-looking Cholesky, column by column.
-  for (int k = 0; k < D; ++k) {
-    if (tid == 0) X[k * LD + k] = sqrtf(X[k * LD + k]);
-    __syncthreads();
-    const float dkk = X[k * LD + k];
-    for (int i = k + 1 + tid; i < D; i += nt) X[i * LD + k] /= dkk;
-    __syncthreads();
-    const int n = D - k - 1;
-    for (int e = tid; e < n * n; e += nt) {
-      const int i = k + 1 + e / n, j = k + 1 + e % n;
-      if (j <= i) X[i * LD + j] -= X[i * LD + k] * X[j * LD + k];
-    }
-    __syncthreads();
-  }
-  // Y = L^-1 by forward substitution, one row at a time, all columns in parallel.
-  for (int i = 0; i < D; ++i) {
-    const float lii = X[i * LD + i];
-    for (int j = tid; j <= i; j += nt) {
-      float acc = (i == j) ? 1.f : 0.f;
-      for (int k = j; k < i; ++k) acc -= X[i * LD + k] * Y[k * LD + j];
-      Y[i * LD + j] = acc / lii;
-    }
-    __syncthreads();
-  }
-  // P = Y^T Y (symmetric); P[i][j] = sum_{k >= max(i,j)} Y[k][i] Y[k][j].
-  for (int e = tid; e < D * D; e += nt) {
-    const int i = e / D, j = e % D, m = i > j ? i : j;
-    float acc = 0.f;
-    for (int k = m; k < D; ++k) acc = fmaf(Y[k * LD + i], Y[k * LD + j], acc);
-    X[i * LD + j] = acc;
-  }
-  __syncthreads();
-  if (s > 0) {
-    const float* alpha = p.alpha + (((long long)b * p.H + h) * p.T + s) * D;
-    for (int e = tid; e < D * D; e += nt) {
-      const int i = quad_row(D, e), j = quad_col(D, e);
-      p.M[off + e] = alpha[i] * X[i * LD + j];
+  // C = B P: this thread's 8 x 8 tile, k in column quads of B.
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) x[r][c] = 0.f;
+  const float4* B4 = reinterpret_cast<const float4*>(p.Bm + off);
+#pragma unroll 1
+  for (int kq = 0; kq < D / 4; ++kq) {
+    float4 bq[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) bq[r] = B4[kq * D + 8 * ti + r];  // B[8 ti + r][4 kq .. 4 kq + 3]
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float* prow = sP + (4 * kq + u) * D + 8 * tj;
+      const float4 p0 = reinterpret_cast<const float4*>(prow)[0], p1 = reinterpret_cast<const float4*>(prow)[1];
+      const float pc[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const float bv = u == 0 ? bq[r].x : u == 1 ? bq[r].y : u == 2 ? bq[r].z : bq[r].w;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) x[r][c] = fmaf(bv, pc[c], x[r][c]);
+      }
     }
   }
-  const float* Bm = p.Bm + off;
-  for (int e = tid; e < D * D; e += nt) {
-    const int i = quad_row(D, e), j = quad_col(D, e);
-    float acc = 0.f;
-    for (int k = 0; k < D; ++k) acc = fmaf(Bm[quad_off(D, i, k)], X[k * LD + j], acc);
-    p.C[off + e] = acc;
+  float4* C4 = reinterpret_cast<float4*>(p.C + off);
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int i = 8 * ti + r;
+    C4[(2 * tj) * D + i] = make_float4(x[r][0], x[r][1], x[r][2], x[r][3]);
+    C4[(2 * tj + 1) * D + i] = make_float4(x[r][4], x[r][5], x[r][6], x[r][7]);
   }
 }
 
@@ -371,10 +453,10 @@ cudaError_t launch_solve_simt(const Problem& p, cudaStream_t s) {
   dim3 grid(p.T - 1, p.H, p.B);
   return dispatch_d(p.D, [&](auto dc) {
     constexpr int D = decltype(dc)::value;
-    const size_t smem = 2ull * D * (D + 1) * sizeof(float);
+    const size_t smem = (size_t)SweepCfg<D>::kSmemFloats * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(solve_simt_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    solve_simt_kernel<D><<<grid, 256, smem, s>>>(p);
+    solve_simt_kernel<D><<<grid, SweepCfg<D>::kThreads, smem, s>>>(p);
     return cudaGetLastError();
   });
 }
