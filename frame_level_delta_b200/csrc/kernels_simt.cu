@@ -252,57 +252,144 @@ __global__ void __launch_bounds__(SweepCfg<D>::kThreads) solve_simt_kernel(Probl
 }
 
 // ---------------------------------------------------------------------------
-// Bidirectional scan. Grid (B*H, 2 directions, D/16 row slabs). The rows of the
-// state evolve independently under S <- S M + C, so each CTA carries 16 rows.
+// Bidirectional scan on the CUDA cores. Grid (B*H, 2 directions), 256 threads.
 // Forward: F(0) = S_T/2, F(f) = F(f-1) M_f + C_f for f = 1 .. c(J-2)-1.
 // Reverse: R(T-1) = S_T/2, R(f) = R(f+1) M_f + C_f for f = T-2 .. 2c.
 // Chunk j's forward readout state is F(max(0, c(j-1)-1)); its reverse one is
 // R(min(T-1, c(j+2))).
+// The state lives in shared memory transposed (ST[k][i] = S[i][k]) and each
+// frame's M_f row-major, both with rows padded to D + 4 floats; M_{f+1} is
+// copied in (cp.async) while step f computes. Each thread owns 4 x 4 tiles of
+// the new state: per k one float4 of S's column and one of M's row, 16 FMAs.
 // ---------------------------------------------------------------------------
 template <int D>
+struct ScanSimtCfg {
+  static constexpr int LD = D + 4;              // padded row (floats)
+  static constexpr int NQ = D / 4;              // 4-wide quads per row
+  static constexpr int kTiles = NQ * NQ;        // 4 x 4 tiles of the state
+  static constexpr int kTPT = (kTiles + 255) / 256;  // tiles per thread
+  static constexpr int kSmemFloats = 3 * D * LD;     // ST, then M for two steps
+};
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <int D>
 __global__ void __launch_bounds__(256) scan_simt_kernel(Problem p) {
-  constexpr int R = 16, NC = D / 16;
-  __shared__ float sS[R][D + 1];
-  const int bh = blockIdx.x, dir = blockIdx.y, r0 = blockIdx.z * R;
+  using C = ScanSimtCfg<D>;
+  constexpr int LD = C::LD, NQ = C::NQ;
+  extern __shared__ float smem[];
+  float* ST = smem;  // [D][LD]
+  float* sM = smem + D * LD;  // [2][D][LD]
+  const int bh = blockIdx.x, dir = blockIdx.y;
   const int b = bh / p.H, h = bh % p.H;
-  const int r = threadIdx.x / 16, l = threadIdx.x % 16;
-  const float* S_T = p.C + slot_off(p, b, h, 0);
+  const int tid = threadIdx.x;
   float* out = dir == 0 ? p.Sf : p.Sr;
   const int c = p.c, T = p.T, J = p.J;
-#pragma unroll
-  for (int m = 0; m < NC; ++m) sS[r][l + 16 * m] = 0.5f * S_T[quad_off(D, r0 + r, l + 16 * m)];
-  __syncthreads();
-  auto store = [&](int j) {
-    const long long o = chunk_off(p, b, h, j);
-#pragma unroll
-    for (int m = 0; m < NC; ++m) out[o + quad_off(D, r0 + r, l + 16 * m)] = sS[r][l + 16 * m];
-  };
-  for (int j = 0; j < J; ++j)
-    if (dir == 0 ? (c * (j - 1) - 1 <= 0) : (c * (j + 2) >= T - 1)) store(j);
   const int f_first = dir == 0 ? 1 : T - 2;
   const int f_last = dir == 0 ? c * (J - 2) - 1 : 2 * c;
-  const int nsteps = dir == 0 ? f_last - f_first + 1 : f_first - f_last + 1;
+  const int nsteps = max(0, dir == 0 ? f_last - f_first + 1 : f_first - f_last + 1);
+  auto frame = [&](int st) { return dir == 0 ? f_first + st : f_first - st; };
+  // M_f (column quads in global memory: float4 q * D + k holds M[k][4q..4q+3]) into buffer u.
+  auto load_m = [&](int st, int u) {
+    const float4* src = reinterpret_cast<const float4*>(p.M + slot_off(p, b, h, frame(st)));
+    float* dst = sM + u * D * LD;
+    for (int e = tid; e < D * NQ; e += 256) {
+      const int q = e / D, k = e % D;
+      cp_async16(dst + k * LD + 4 * q, src + e);
+    }
+    cp_async_commit();
+  };
+  // Readout state j from this thread's tiles (quad layout).
+  auto store_tiles = [&](int j, const float (&v)[C::kTPT][4][4]) {
+    float4* o4 = reinterpret_cast<float4*>(out + chunk_off(p, b, h, j));
+#pragma unroll
+    for (int tt = 0; tt < C::kTPT; ++tt) {
+      const int t = tid + 256 * tt;
+      if (t >= C::kTiles) break;
+      const int i0 = 4 * (t / NQ), q = t % NQ;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) o4[q * D + i0 + r] = make_float4(v[tt][r][0], v[tt][r][1], v[tt][r][2], v[tt][r][3]);
+    }
+  };
+  if (nsteps > 0) load_m(0, 0);
+  // S = S_T / 2, transposed into ST; the readout states of chunks that see no frame.
+  float v[C::kTPT][4][4];
+  {
+    const float4* s4 = reinterpret_cast<const float4*>(p.C + slot_off(p, b, h, 0));
+#pragma unroll
+    for (int tt = 0; tt < C::kTPT; ++tt) {
+      const int t = tid + 256 * tt;
+      if (t >= C::kTiles) break;
+      const int i0 = 4 * (t / NQ), q = t % NQ;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float4 w = s4[q * D + i0 + r];
+        v[tt][r][0] = 0.5f * w.x; v[tt][r][1] = 0.5f * w.y; v[tt][r][2] = 0.5f * w.z; v[tt][r][3] = 0.5f * w.w;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) ST[(4 * q + cc) * LD + i0 + r] = v[tt][r][cc];
+      }
+    }
+  }
+  for (int j = 0; j < J; ++j)
+    if (dir == 0 ? (c * (j - 1) - 1 <= 0) : (c * (j + 2) >= T - 1)) store_tiles(j, v);
   for (int st = 0; st < nsteps; ++st) {
-    const int f = dir == 0 ? f_first + st : f_first - st;
-    const float* Mf = p.M + slot_off(p, b, h, f);
-    const float* Cf = p.C + slot_off(p, b, h, f);
-    float acc[NC];
-#pragma unroll
-    for (int m = 0; m < NC; ++m) acc[m] = Cf[quad_off(D, r0 + r, l + 16 * m)];
-#pragma unroll 4
-    for (int k = 0; k < D; ++k) {
-      const float sv = sS[r][k];
-#pragma unroll
-      for (int m = 0; m < NC; ++m) acc[m] = fmaf(sv, Mf[quad_off(D, k, l + 16 * m)], acc[m]);
+    const int f = frame(st);
+    if (st + 1 < nsteps) {
+      load_m(st + 1, (st + 1) & 1);
+      cp_async_wait<1>();  // this step's M is in
+    } else {
+      cp_async_wait<0>();
     }
     __syncthreads();
+    const float* m = sM + (st & 1) * D * LD;
+    const float4* c4 = reinterpret_cast<const float4*>(p.C + slot_off(p, b, h, f));
 #pragma unroll
-    for (int m = 0; m < NC; ++m) sS[r][l + 16 * m] = acc[m];
-    __syncthreads();
+    for (int tt = 0; tt < C::kTPT; ++tt) {
+      const int t = tid + 256 * tt;
+      if (t >= C::kTiles) break;
+      const int i0 = 4 * (t / NQ), q = t % NQ;
+      float acc[4][4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float4 w = c4[q * D + i0 + r];
+        acc[r][0] = w.x; acc[r][1] = w.y; acc[r][2] = w.z; acc[r][3] = w.w;
+      }
+#pragma unroll 8
+      for (int k = 0; k < D; ++k) {
+        const float4 sc = *reinterpret_cast<const float4*>(ST + k * LD + i0);     // S[i0..i0+3][k]
+        const float4 mr = *reinterpret_cast<const float4*>(m + k * LD + 4 * q);   // M[k][4q..4q+3]
+        const float sv[4] = {sc.x, sc.y, sc.z, sc.w}, mv[4] = {mr.x, mr.y, mr.z, mr.w};
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) acc[r][cc] = fmaf(sv[r], mv[cc], acc[r][cc]);
+      }
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) v[tt][r][cc] = acc[r][cc];
+    }
+    __syncthreads();  // every read of the old state and of this M buffer is done
+#pragma unroll
+    for (int tt = 0; tt < C::kTPT; ++tt) {
+      const int t = tid + 256 * tt;
+      if (t >= C::kTiles) break;
+      const int i0 = 4 * (t / NQ), q = t % NQ;
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) ST[(4 * q + cc) * LD + i0 + r] = v[tt][r][cc];
+    }
     if (dir == 0) {
-      if ((f + 1) % c == 0 && (f + 1) / c + 1 < J) store((f + 1) / c + 1);
+      if ((f + 1) % c == 0 && (f + 1) / c + 1 < J) store_tiles((f + 1) / c + 1, v);
     } else {
-      if (f % c == 0 && f / c - 2 >= 0) store(f / c - 2);
+      if (f % c == 0 && f / c - 2 >= 0) store_tiles(f / c - 2, v);
     }
   }
 }
@@ -462,10 +549,13 @@ cudaError_t launch_solve_simt(const Problem& p, cudaStream_t s) {
 }
 
 cudaError_t launch_scan_simt(const Problem& p, cudaStream_t s) {
-  dim3 grid(p.B * p.H, 2, p.D / 16);
+  dim3 grid(p.B * p.H, 2);
   return dispatch_d(p.D, [&](auto dc) {
     constexpr int D = decltype(dc)::value;
-    scan_simt_kernel<D><<<grid, 256, 0, s>>>(p);
+    const size_t smem = (size_t)ScanSimtCfg<D>::kSmemFloats * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(scan_simt_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    scan_simt_kernel<D><<<grid, 256, smem, s>>>(p);
     return cudaGetLastError();
   });
 }
