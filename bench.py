@@ -53,6 +53,54 @@ def load_peaks():
 
 
 # ----------------------------------------------------------------------------
+# Ranks: one process per GPU, each rank its own batch (weak scaling). The only
+# collectives are the barriers around the timed regions and the max-over-ranks
+# reduction of the measured times; the data path has none.
+# ----------------------------------------------------------------------------
+def rank_env():
+    """(rank, world size, local rank) as torch.distributed.run exports them."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def rank_seed(cfg, rank: int) -> int:
+    """Seed of the batch a rank draws: independent problems per rank."""
+    return cfg.seed + rank
+
+
+def init_ranks(world: int, device, timeout_s: float = 120.0):
+    """Process group for the barriers and the time reduction (NCCL between CUDA
+    ranks, gloo between CPU ranks); None for a single rank."""
+    if world <= 1:
+        return None
+    import torch.distributed as dist
+    timeout = datetime.timedelta(seconds=timeout_s)
+    if device.type == "cuda":
+        dist.init_process_group("nccl", timeout=timeout, device_id=device)
+    else:
+        dist.init_process_group("gloo", timeout=timeout)
+    return dist
+
+
+def barrier(dist) -> None:
+    if dist is not None:
+        dist.barrier()
+
+
+def max_over_ranks(dist, ms: float, device) -> float:
+    """The slowest rank's time: every rank takes part, every rank gets the max."""
+    t = torch.tensor([float(ms)], device=device, dtype=torch.float64)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, cfg, steps: int, ms_max: float) -> float:
+    """Head-tokens all ranks processed divided by the slowest rank's time."""
+    return world * cfg.head_tokens * steps / (ms_max / 1e3)
+
+
+# ----------------------------------------------------------------------------
 # Algorithmic bytes / flops per launch of each kernel (each input byte read
 # once, each output byte written once).
 # ----------------------------------------------------------------------------
@@ -387,26 +435,17 @@ def main():
     cfg = CONFIGS[args.config]
     if args.heads > 0:
         cfg = cfg.with_(H=args.heads)
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = rank_env()
     if args.impl == "reference":
         return run_reference(args, cfg, rank)
 
     from frame_level_delta_b200 import vda as V
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    dist = None
-    if world > 1:
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
+    dist = init_ranks(world, dev)
 
     # Each rank draws its own batch (independent problems).
-    inp_cpu = make_inputs(cfg, seed=cfg.seed + rank)
+    inp_cpu = make_inputs(cfg, seed=rank_seed(cfg, rank))
     inp_host = {k: v.pin_memory() for k, v in inp_cpu.items()}
     inp_dev = {k: v.to(dev, non_blocking=True) for k, v in inp_host.items()}
     global SCAN_CHUNKED, SOLVE_CHOLESKY
@@ -429,7 +468,7 @@ def main():
     # and the roofline.
     n0 = lib.launch_count()
     clocks = ClockSampler(local)
-    barrier()
+    barrier(dist)
     torch.cuda.synchronize(dev)
     clocks.start()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -439,14 +478,14 @@ def main():
     ev1.record(stream)
     torch.cuda.synchronize(dev)
     clocks.stop()
-    barrier()
+    barrier(dist)
     ms = ev0.elapsed_time(ev1)
     launches = lib.launch_count() - n0
     if lib.poll_device_status() != 0:
         raise RuntimeError("device status reported a timeout in the timed region")
     # ---- per-kernel pass: the same K steps with CUDA events around every launch
     lib.profile_enable(True)
-    barrier()
+    barrier(dist)
     torch.cuda.synchronize(dev)
     ep0, ep1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ep0.record(stream)
@@ -454,18 +493,14 @@ def main():
         lib.run(inp_dev, O)
     ep1.record(stream)
     torch.cuda.synchronize(dev)
-    barrier()
+    barrier(dist)
     ms_profiled = ep0.elapsed_time(ep1)
     prof = lib.profile_read()
     lib.profile_enable(False)
     if lib.poll_device_status() != 0:
         raise RuntimeError("device status reported a timeout in the per-kernel pass")
-    t = torch.tensor([ms], device=dev, dtype=torch.float64)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
-    units = world * cfg.head_tokens * args.steps
-    value = units / (ms_max / 1e3)
+    ms_max = max_over_ranks(dist, ms, dev)
+    value = whole_job_rate(world, cfg, args.steps, ms_max)
 
     # ---- end to end through the public API: pinned host inputs -> device ->
     # prepare/scan/readout -> O back to pinned host memory, every step. The
@@ -486,7 +521,7 @@ def main():
     up_done = [ev() for _ in range(ke)]
     run_done = [ev() for _ in range(ke)]
     down_done = [ev() for _ in range(ke)]
-    barrier()
+    barrier(dist)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -512,11 +547,8 @@ def main():
     stream.wait_stream(down)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    barrier()
-    t = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_value = world * cfg.head_tokens * ke / (float(t.item()) / 1e3)
+    barrier(dist)
+    e2e_value = whole_job_rate(world, cfg, ke, max_over_ranks(dist, e0.elapsed_time(e1), dev))
 
     # ---- roofline of the dominant kernel (live per-kernel CUDA events) -------
     peaks, peak_src = load_peaks()

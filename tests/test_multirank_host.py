@@ -1,0 +1,125 @@
+"""Host side of the N>1 path on CPU: two gloo ranks run bench.py's rank helpers.
+
+The path shards by batch: every rank draws and processes its own batch and no
+collective touches the data. What the ranks share is the timing protocol (a
+barrier on both sides of each timed region, the max over ranks of the measured
+time, the whole-job rate over all ranks' units, rank 0 printing alone); these
+tests run exactly those functions over a gloo process group on 127.0.0.1.
+"""
+import hashlib
+import json
+import os
+import socket
+import subprocess
+import sys
+import time
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _set_env(rank, world, port):
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port), "RANK": str(rank),
+                       "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank)})
+
+
+def _rank_timing(rank, world, port, out_dir):
+    sys.path.insert(0, ROOT)
+    _set_env(rank, world, port)
+    import bench
+    from frame_level_delta_b200.inputs import CONFIGS, make_inputs
+
+    r, w, local = bench.rank_env()
+    cpu = torch.device("cpu")
+    dist = bench.init_ranks(w, cpu, timeout_s=60)
+    cfg = CONFIGS["tiny"]
+    inp = make_inputs(cfg, seed=bench.rank_seed(cfg, r))
+    h = hashlib.sha256()
+    for k in sorted(inp):
+        h.update(inp[k].contiguous().numpy().tobytes())
+    digests = [None] * w
+    dist.all_gather_object(digests, h.hexdigest())
+    bench.barrier(dist)
+    ms = 1.0 + 2.5 * r  # rank r "took" this long
+    ms_max = bench.max_over_ranks(dist, ms, cpu)
+    rate = bench.whole_job_rate(w, cfg, 7, ms_max)
+    bench.barrier(dist)
+    dist.destroy_process_group()
+    with open(os.path.join(out_dir, f"rank{r}.json"), "w") as f:
+        json.dump({"rank": r, "world": w, "local": local, "digests": digests, "ms_max": ms_max,
+                   "rate": rate, "head_tokens": cfg.head_tokens}, f)
+
+
+def _rank_leaves(rank, world, port, out_dir):
+    """Rank 1 leaves between steps (before the barrier); rank 0 must end with an
+    error from its barrier within the process group's timeout, not wait for good."""
+    sys.path.insert(0, ROOT)
+    _set_env(rank, world, port)
+    import bench
+
+    dist = bench.init_ranks(world, torch.device("cpu"), timeout_s=5)
+    if rank == 1:
+        os._exit(0)
+    t0 = time.monotonic()
+    err = None
+    try:
+        bench.barrier(dist)
+        bench.barrier(dist)
+    except Exception as e:  # noqa: BLE001 - any error is the expected outcome
+        err = type(e).__name__
+    with open(os.path.join(out_dir, "rank0.json"), "w") as f:
+        json.dump({"error": err, "seconds": time.monotonic() - t0}, f)
+    os._exit(0)
+
+
+def test_two_gloo_ranks_barrier_max_and_shards(tmp_path):
+    world = 2
+    mp.start_processes(_rank_timing, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    res = [json.loads((tmp_path / f"rank{r}.json").read_text()) for r in range(world)]
+    for r, d in enumerate(res):
+        assert (d["rank"], d["world"], d["local"]) == (r, world, r)
+        # every rank sees the slowest rank's time
+        assert d["ms_max"] == pytest.approx(1.0 + 2.5 * (world - 1))
+        # whole-job rate: all ranks' head-tokens over that time
+        assert d["rate"] == pytest.approx(world * d["head_tokens"] * 7 / (d["ms_max"] / 1e3))
+    # each rank drew its own batch (independent problems), and both agree on the set
+    assert res[0]["digests"] == res[1]["digests"]
+    assert len(set(res[0]["digests"])) == world
+
+
+def test_rank_that_leaves_ends_peer_barrier_with_error(tmp_path):
+    world = 2
+    ctx = mp.start_processes(_rank_leaves, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                             join=False, start_method="spawn")
+    deadline = time.monotonic() + 120
+    while not ctx.join(timeout=5):
+        assert time.monotonic() < deadline, "rank 0 kept waiting on a rank that left"
+    d = json.loads((tmp_path / "rank0.json").read_text())
+    assert d["error"] is not None
+    assert d["seconds"] < 60
+
+
+def test_reference_arm_prints_once_under_torchrun():
+    """`bench.py --impl reference` under torchrun with two ranks: rank 0 alone
+    times the oracle and prints one JSON line; rank 1 exits 0 without work."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py", "--impl",
+           "reference", "--gpus", "2", "--config", "tiny", "--steps", "2", "--warmup", "3"]
+    p = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [json.loads(x) for x in p.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    line = lines[0]
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["steps"] == 2
+    assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
+    assert line["cpu_baseline"]["kind"] == "oracle"
