@@ -11,12 +11,16 @@
 // walks the frames t = 0..T. A producer warp brings each frame's 5-row x
 // (kCW + 4)-column neighbourhood of the block (all d channels of head h) into
 // shared memory with one 4-D TMA load (zero fill outside the grid), two frames
-// in flight, two CTAs per SM. Each compute thread owns two consecutive tokens and
-// four channels: it forms the two 5x5 spatial sums of the frame (every staged
-// value it loads serves both tokens' taps) and keeps the last five frames'
-// sums in registers; the centred temporal sum of frame t - 2 follows, then
-// SiLU, the key norm (a shuffle reduction over the token's d / 4 lanes) and the
-// store of frames 1..T-2 in the prepared layout [B, H, T, U, d].
+// in flight, three CTAs per SM at d = 128. Each compute thread owns four
+// consecutive tokens and four channels: it forms the four 5x5 spatial sums of
+// the frame (each staged value it loads serves up to four taps, each weight
+// load four tokens) and keeps the last five frames' sums in registers; the
+// centred temporal sum of frame t - 2 follows, then SiLU, the key norm (a
+// shuffle reduction over the token's d / 4 lanes) and the store of frames
+// 1..T-2 in the prepared layout [B, H, T, U, d]. The kernel is bound by
+// instruction issue and shared-memory bandwidth: four tokens per thread halve
+// the shared-memory wavefronts per output and cut the instructions per output
+// by about a third against two tokens per thread.
 #include <cuda_bf16.h>
 
 #include "internal.h"
@@ -28,20 +32,25 @@ namespace vda {
 namespace {
 
 constexpr int kCW = 16;      // grid columns (tokens) per CTA
-constexpr int kTPT = 2;      // tokens per compute thread
 constexpr int kTileCols = kCW + 4;
 
 template <typename TIn, int D>
 struct PrepCfg {
+  // Tokens per compute thread: four; two at d = 16, so that the compute
+  // threads still fill a whole warp (the shuffles and __syncwarp take all lanes).
+  static constexpr int kTPT = D >= 32 ? 4 : 2;
   static constexpr int kCompute = (kCW / kTPT) * (D / 4);  // compute threads
   static constexpr int kThreads = kCompute + 32;           // + producer warp
   static constexpr int kLanesPerGroup = D / 4;              // threads sharing a token group
-  static constexpr int kStages = 2;                          // frames in flight per CTA (two CTAs per SM)
+  static constexpr int kStages = 2;                          // frames in flight per CTA
   static constexpr int kStageBytes = (5 * kTileCols * D * (int)sizeof(TIn) + 1023) / 1024 * 1024;
   static constexpr int kWOff = kStages * kStageBytes;       // spatial weights [25][D] fp32
-  static constexpr int kBarOff = kWOff + 25 * D * 4;
+  static constexpr int kWtOff = kWOff + 25 * D * 4;         // temporal weights [5][D] fp32
+  static constexpr int kBarOff = kWtOff + 5 * D * 4;
   static constexpr int kSmemBytes = kBarOff + 128 + 1024;
+  static constexpr int kMinBlocks = 3;                       // CTAs per SM (d = 128, bf16: 3 x 66 KB)
   static_assert(kSmemBytes <= 232448, "shared memory");
+  static_assert(kCompute % 32 == 0, "compute threads fill whole warps");
 };
 
 template <typename TIn>
@@ -71,15 +80,17 @@ struct PrepIO<float> {
 __device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.f + __expf(-x)); }
 
 template <typename TIn, int D>
-__global__ void __launch_bounds__(PrepCfg<TIn, D>::kThreads, 2)
+__global__ void __launch_bounds__(PrepCfg<TIn, D>::kThreads, PrepCfg<TIn, D>::kMinBlocks)
     prep_video_kernel(const __grid_constant__ CUtensorMap mK, const __grid_constant__ CUtensorMap mV,
                       const Problem p, const float* __restrict__ w) {
   using C = PrepCfg<TIn, D>;
   constexpr int kStages = C::kStages;
+  constexpr int kTPT = C::kTPT;
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   float* sw = reinterpret_cast<float*>(smem + C::kWOff);
+  float* swt = reinterpret_cast<float*>(smem + C::kWtOff);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* empty = full + kStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
@@ -99,13 +110,17 @@ __global__ void __launch_bounds__(PrepCfg<TIn, D>::kThreads, 2)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  // Spatial weights of this (head, K|V) into shared memory as [tap][channel].
+  // Spatial and temporal weights of this (head, K|V) into shared memory as [tap][channel].
   const long long hd = (long long)H * D;
   const float* wsp = w + (which == 0 ? 0 : hd * 30) + (long long)h * D * 25;
   const float* wtp = w + (which == 0 ? hd * 25 : hd * 55) + (long long)h * D * 5;
   for (int e = tid; e < 25 * D; e += C::kThreads) {
     const int c = e / 25, tap = e % 25;
     sw[tap * D + c] = wsp[e];
+  }
+  for (int e = tid; e < 5 * D; e += C::kThreads) {
+    const int c = e / 5, tap = e % 5;
+    swt[tap * D + c] = wtp[e];
   }
   __syncthreads();
 
@@ -129,14 +144,9 @@ __global__ void __launch_bounds__(PrepCfg<TIn, D>::kThreads, 2)
     return;
   }
 
-  // ---------------- compute threads: tokens x0 + 4 xg .. +3, channels 4 g .. 4 g + 3
+  // ---------------- compute threads: tokens x0 + kTPT xg .. + kTPT - 1, channels 4 g .. 4 g + 3
   const int xg = tid / C::kLanesPerGroup, g = tid % C::kLanesPerGroup;
   const int ch = 4 * g;
-  float ft[5][4];
-#pragma unroll
-  for (int s = 0; s < 5; ++s)
-#pragma unroll
-    for (int k = 0; k < 4; ++k) ft[s][k] = wtp[(ch + k) * 5 + s];
   float ring[5][kTPT][4];  // spatial sums of frames t-4 .. t (zero outside the clip)
 #pragma unroll
   for (int s = 0; s < 5; ++s)
@@ -194,15 +204,24 @@ __global__ void __launch_bounds__(PrepCfg<TIn, D>::kThreads, 2)
     // Frame t - 2 now has all five temporal taps (frames t-4 .. t).
     const int to = t - 2;
     if (to >= 1 && to <= T - 2) {
+      float ft[5][4];
+#pragma unroll
+      for (int s = 0; s < 5; ++s) {
+        const float4 f = *reinterpret_cast<const float4*>(swt + s * D + ch);
+        ft[s][0] = f.x; ft[s][1] = f.y; ft[s][2] = f.z; ft[s][3] = f.w;
+      }
 #pragma unroll
       for (int k = 0; k < kTPT; ++k) {
         float o[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          float v = 0.f;
+        for (int cp = 0; cp < 2; ++cp) {  // channel pairs: packed fp32x2 FMAs, each lane as fmaf
+          float2 v = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int s = 0; s < 5; ++s) v = fmaf(ft[s][c], ring[s][k][c], v);
-          o[c] = silu(v);
+          for (int s = 0; s < 5; ++s)
+            v = __ffma2_rn(make_float2(ft[s][2 * cp], ft[s][2 * cp + 1]),
+                           make_float2(ring[s][k][2 * cp], ring[s][k][2 * cp + 1]), v);
+          o[2 * cp] = silu(v.x);
+          o[2 * cp + 1] = silu(v.y);
         }
         float sc = 1.f;
         if (which == 0) {

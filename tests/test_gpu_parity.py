@@ -151,6 +151,40 @@ def test_edge_conv_gate_small():
     check_config(cfg.with_(dtype="f32"))
 
 
+# Conv prep at every head dimension and storage type, on grids whose width is
+# not a multiple of the 16-column block (a ragged last block) and with a single
+# grid row; the prepared keys and values are compared with the oracle's prep.
+CONV_EDGE = [
+    ("conv_d16", dict(d=16, grid_h=5, grid_w=9)),
+    ("conv_d32", dict(d=32, grid_h=3, grid_w=17)),
+    ("conv_d64", dict(d=64, grid_h=4, grid_w=35)),
+    ("conv_d128", dict(d=128, grid_h=7, grid_w=21)),
+    ("conv_d128_single_row", dict(d=128, grid_h=1, grid_w=33)),
+]
+
+
+@pytest.mark.parametrize("name,kw", CONV_EDGE, ids=[e[0] for e in CONV_EDGE])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_edge_conv_dims(name, kw, dtype):
+    cfg = CONFIGS["hires"].with_(name=name, H=2, T=9, L=5, chunk=2, dtype=dtype, **kw)
+    inp = make_inputs(cfg)
+    check_config(cfg, inp=inp)
+    _, regions, _ = run_gpu(cfg, inp)
+    w = inp["conv_w"].double().numpy()
+    hd = cfg.H * cfg.d
+    tol = 5e-3 if dtype == "bf16" else 1e-5
+    for h in range(cfg.H):
+        for which, off in (("K", 0), ("V", hd * 30)):
+            X = inp[which][0, :, h].double().numpy().reshape(cfg.T, cfg.U, cfg.d)
+            ws = w[off:off + hd * 25].reshape(cfg.H, cfg.d, 5, 5)[h]
+            wt = w[off + hd * 25:off + hd * 30].reshape(cfg.H, cfg.d, 5)[h]
+            want = vo.prep_video_kv(X, ws, wt, cfg.grid_h, cfg.grid_w)
+            if which == "K":
+                want = vo.l2_normalize(want, 1e-6)
+            got = regions[which + "_prep"][0, h, 1:cfg.T - 1].numpy()
+            assert rel_fro(got, want[1:cfg.T - 1]) <= tol, (which, h)
+
+
 def test_degenerate_gates():
     cfg = CONFIGS["small"].with_(H=2, T=10, grid_h=4, grid_w=4)
     inp = make_inputs(cfg)
