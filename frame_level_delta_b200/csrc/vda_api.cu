@@ -75,8 +75,15 @@ vda_status check_config(const vda_config* c, std::string* why) {
     if (why) *why = "d must be one of 16, 32, 64, 128";
     return VDA_ERR_UNSUPPORTED;
   }
-  if ((c->flags & VDA_PREP_CONV) && (size_t)c->grid_w * d * sizeof(float) > 200 * 1024) {
-    if (why) *why = "grid_w * d too large for the prep kernel's row buffer";
+  // Launch-grid limits, checked here so that no call fails after it has begun
+  // to enqueue work: the conv prep runs grid rows on grid.y and (b, h, K|V) on
+  // grid.z; the chunk composition runs (b, h) on grid.z.
+  if ((c->flags & VDA_PREP_CONV) && (c->grid_h > 65535 || (long long)c->B * c->H * 2 > 65535)) {
+    if (why) *why = "conv prep needs grid_h <= 65535 and 2 * B * H <= 65535";
+    return VDA_ERR_UNSUPPORTED;
+  }
+  if ((c->flags & VDA_SCAN_CHUNKED) && (long long)c->B * c->H > 65535) {
+    if (why) *why = "the chunked scan needs B * H <= 65535";
     return VDA_ERR_UNSUPPORTED;
   }
   const long long tokens = (long long)c->B * c->T * c->U * c->H * d;
@@ -204,7 +211,7 @@ vda_status vda_create(const vda_config* cfg, vda_ctx** out) {
   vda_status st = check_config(cfg, nullptr);
   if (st != VDA_OK) return st;
   vda_ctx* ctx = new (std::nothrow) vda_ctx();
-  if (!ctx) return VDA_ERR_INVALID_ARG;
+  if (!ctx) return VDA_ERR_UNSUPPORTED;  // host allocation failed
   ctx->cfg = *cfg;
   *out = ctx;
   return VDA_OK;

@@ -70,14 +70,17 @@ typedef enum vda_dtype {
 /* vda_config.flags */
 #define VDA_PREP_CONV 0x1u         /* video K, V: depthwise 5x5 spatial + centred 5-tap temporal
                                       cross-correlation (zero padding, no bias) then SiLU; text K, V:
-                                      SiLU; then K, K_txt and Q divided by sqrt(|x|^2 + l2_eps) */
+                                      SiLU; then K, K_txt and Q divided by sqrt(|x|^2 + l2_eps).
+                                      Needs grid_h <= 65535 and 2 * B * H <= 65535, else
+                                      VDA_ERR_UNSUPPORTED from vda_create */
 #define VDA_READOUT_NORM_GATE 0x2u /* o <- o / sqrt(mean(o^2) + rms_eps) * sigmoid(gate) */
 #define VDA_SOLVE_CHOLESKY 0x4u    /* tensor-core frame solve by blocked Cholesky of I + A_t and
                                       the triangular inverse, instead of the default symmetric
                                       sweep (Gauss-Jordan) in registers; the same M_t and C_t */
 #define VDA_SCAN_CHUNKED 0x8u      /* tensor-core scan over composed chunk maps (each chunk's frame
                                       maps composed in parallel first) instead of the default scan
-                                      frame by frame; the same readout states */
+                                      frame by frame; the same readout states. Needs
+                                      B * H <= 65535, else VDA_ERR_UNSUPPORTED from vda_create */
 #define VDA_FORCE_SIMT 0x100u      /* run the generic CUDA-core kernels even where a tensor-core
                                       kernel exists (diagnostics and cross-checks) */
 

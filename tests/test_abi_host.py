@@ -56,6 +56,26 @@ def test_create_rejects_bad_configs(field, value, want):
     assert V.lib().vda_workspace_size(ctypes.byref(c), ctypes.byref(n)) == want
 
 
+@pytest.mark.parametrize("kw,want", [
+    (dict(grid_h=65536, grid_w=1, U=65536), 2),   # conv prep: grid rows on grid.y
+    (dict(B=1, H=32768), 2),                       # conv prep: 2 B H on grid.z
+    (dict(B=1, H=32767), 0),
+    (dict(grid_h=2, grid_w=4096, U=8192, d_k=128, d_v=128), 0),  # wide grids tile in 16-column blocks
+])
+def test_conv_prep_launch_limits_are_checked_at_create(kw, want):
+    c = _cfg(flags=V.VDA_PREP_CONV, **kw)
+    st, ctx = _create(c)
+    assert st == want
+    if ctx.value:
+        assert V.lib().vda_destroy(ctx) == 0
+
+
+def test_chunked_scan_launch_limit_is_checked_at_create():
+    c = _cfg(flags=V.VDA_SCAN_CHUNKED, B=2, H=32768)
+    st, ctx = _create(c)
+    assert st == 2 and not ctx.value
+
+
 def test_workspace_regions_are_disjoint_and_aligned():
     for name in ("tiny", "small", "h3", "long", "hires"):
         c = V.make_config(CONFIGS[name])
