@@ -247,7 +247,8 @@ def path_flops(cfg) -> float:
 
 def source_digest(kernel: str):
     files = {"gram_tc": "gram_tc.cu", "readout_tc": "readout_tc.cu", "solve_tc": "solve_tc.cu",
-             "scan_tc": "scan_tc.cu", "compose_tc": "compose_tc.cu", "solve_chol_tc": "solve_chol_tc.cu"}
+             "scan_tc": "scan_tc.cu", "compose_tc": "compose_tc.cu", "solve_chol_tc": "solve_chol_tc.cu",
+             "prep_video": "prep_video.cu"}
     fn = files.get(kernel, "kernels_simt.cu")
     p = os.path.join(ROOT, "frame_level_delta_b200", "csrc", fn)
     with open(p, "rb") as f:
