@@ -339,12 +339,8 @@ __global__ void __launch_bounds__(kThreads, 1) compose_tc_kernel(const ComposeAr
 }  // namespace
 
 cudaError_t launch_compose_tc(const Problem& p, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(compose_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(compose_tc_kernel), kSmemBytes);
+  if (e != cudaSuccess) return e;
   if (p.J < 3) return cudaSuccess;  // no readout state sees a composed chunk
   if ((long long)p.B * p.H > 65535) return cudaErrorInvalidConfiguration;
   ComposeArgs a{p.H, p.T, p.c, p.J, static_cast<const uint8_t*>(p.Msplit), p.C, static_cast<uint8_t*>(p.CMi),

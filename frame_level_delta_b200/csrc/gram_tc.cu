@@ -398,12 +398,8 @@ cudaError_t launch_d(const Problem& p, cudaStream_t s) {
   GramArgs a{p.B, p.H, p.T, p.U, p.L, 0, p.beta, p.beta_txt, p.A, p.Bm, p.status, p.gready, p.spin_limit};
   cudaError_t e = encode_maps(p, &mK, &mV, &mKt, &mVt, &a.layout);
   if (e != cudaSuccess) return e;
-  static bool attr_set = false;
-  if (!attr_set) {
-    e = cudaFuncSetAttribute(gram_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  e = set_max_dynamic_smem(reinterpret_cast<const void*>(gram_tc_kernel<D>), C::kSmemBytes);
+  if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -141,6 +141,9 @@ bool gram_tc_supported(const Problem& p);
 cudaError_t launch_gram_tc(const Problem& p, cudaStream_t s);
 bool readout_tc_supported(const Problem& p);
 bool solve_tc_supported(const Problem& p);
+// Raise `func`'s dynamic shared-memory limit to `bytes` on the current device,
+// once per (function, device): the attribute belongs to the device's context.
+cudaError_t set_max_dynamic_smem(const void* func, int bytes);
 cudaError_t launch_solve_tc(const Problem& p, cudaStream_t s);
 cudaError_t launch_solve_chol_tc(const Problem& p, cudaStream_t s);
 bool scan_tc_supported(const Problem& p);

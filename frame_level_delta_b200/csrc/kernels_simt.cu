@@ -541,7 +541,7 @@ cudaError_t launch_solve_simt(const Problem& p, cudaStream_t s) {
   return dispatch_d(p.D, [&](auto dc) {
     constexpr int D = decltype(dc)::value;
     const size_t smem = (size_t)SweepCfg<D>::kSmemFloats * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(solve_simt_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(solve_simt_kernel<D>), (int)smem);
     if (e != cudaSuccess) return e;
     solve_simt_kernel<D><<<grid, SweepCfg<D>::kThreads, smem, s>>>(p);
     return cudaGetLastError();
@@ -553,7 +553,7 @@ cudaError_t launch_scan_simt(const Problem& p, cudaStream_t s) {
   return dispatch_d(p.D, [&](auto dc) {
     constexpr int D = decltype(dc)::value;
     const size_t smem = (size_t)ScanSimtCfg<D>::kSmemFloats * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(scan_simt_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(scan_simt_kernel<D>), (int)smem);
     if (e != cudaSuccess) return e;
     scan_simt_kernel<D><<<grid, 256, smem, s>>>(p);
     return cudaGetLastError();
@@ -566,7 +566,7 @@ cudaError_t launch_readout_simt(const Problem& p, const void* gate, void* O, cud
   return dispatch_d(p.D, [&](auto dc) {
     constexpr int D = decltype(dc)::value;
     const size_t smem = (size_t)(D + 64) * (D + 1) * sizeof(float);
-    cudaError_t e = cudaFuncSetAttribute(readout_simt_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(readout_simt_kernel<D>), (int)smem);
     if (e != cudaSuccess) return e;
     readout_simt_kernel<D><<<grid, 256, smem, s>>>(p, gate, O, tiles);
     return cudaGetLastError();

@@ -243,13 +243,8 @@ __global__ void __launch_bounds__(PrepCfg<TIn, D>::kThreads, PrepCfg<TIn, D>::kM
 template <typename TIn, int D>
 cudaError_t launch_typed(const Problem& p, const void* K, const void* V, const float* w, cudaStream_t s) {
   using C = PrepCfg<TIn, D>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(prep_video_kernel<TIn, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(prep_video_kernel<TIn, D>), C::kSmemBytes);
+  if (e != cudaSuccess) return e;
   // [B * T frames][gh rows][gw columns][H * D channels], channels innermost.
   const uint64_t esz = sizeof(TIn);
   const uint64_t dims[4] = {(uint64_t)p.H * D, (uint64_t)p.gw, (uint64_t)p.gh, (uint64_t)p.B * p.T};
@@ -257,7 +252,7 @@ cudaError_t launch_typed(const Problem& p, const void* K, const void* V, const f
   const uint32_t box[4] = {(uint32_t)D, (uint32_t)kTileCols, 5u, 1u};
   const CUtensorMapDataType dt = sizeof(TIn) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   CUtensorMap mK, mV;
-  cudaError_t e = make_tmap_typed(&mK, dt, K, 4, dims, strides, box);
+  e = make_tmap_typed(&mK, dt, K, 4, dims, strides, box);
   if (e != cudaSuccess) return e;
   e = make_tmap_typed(&mV, dt, V, 4, dims, strides, box);
   if (e != cudaSuccess) return e;

@@ -526,13 +526,9 @@ cudaError_t launch_dg(const Problem& p, const void* gate, void* O, cudaStream_t 
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  static bool attr_set = false;
   cudaError_t e;
-  if (!attr_set) {
-    e = cudaFuncSetAttribute(readout_tc_kernel<D, GATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  e = set_max_dynamic_smem(reinterpret_cast<const void*>(readout_tc_kernel<D, GATE>), C::kSmemBytes);
+  if (e != cudaSuccess) return e;
   int per_sm = 1;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, readout_tc_kernel<D, GATE>, kThreads, C::kSmemBytes);
   if (per_sm < 1) per_sm = 1;

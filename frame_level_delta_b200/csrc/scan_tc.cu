@@ -427,12 +427,8 @@ __global__ void __launch_bounds__(kThreads, 1) scan_tc_kernel(const ScanArgs a) 
 bool scan_tc_supported(const Problem& p) { return solve_tc_supported(p); }
 
 cudaError_t launch_scan_tc(const Problem& p, cudaStream_t s, bool chunked) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(scan_tc_kernel), kSmemBytes);
+  if (e != cudaSuccess) return e;
   // Composed chunks come from a kernel that ran after the whole solve: only the
   // frame scan waits on the slot-ready words, and only it overlaps the solve.
   const bool overlap = !chunked && p.ready != nullptr;

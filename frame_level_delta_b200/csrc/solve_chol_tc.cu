@@ -423,12 +423,8 @@ __global__ void __launch_bounds__(kThreads, 2) solve_chol_tc_kernel(const SolveA
 }  // namespace
 
 cudaError_t launch_solve_chol_tc(const Problem& p, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(solve_chol_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(solve_chol_tc_kernel), kSmemBytes);
+  if (e != cudaSuccess) return e;
   SolveArgs a{p.B, p.H, p.T, p.A, p.Bm, p.alpha, p.M, p.C, static_cast<uint8_t*>(p.Msplit), p.status,
               p.spin_limit};
   dim3 grid(p.T - 1, p.H, p.B);

@@ -432,12 +432,8 @@ __global__ void __launch_bounds__(kThreads, 3) solve_tc_kernel(const SolveArgs a
 bool solve_tc_supported(const Problem& p) { return p.bf16 && p.D == 128; }
 
 cudaError_t launch_solve_tc(const Problem& p, cudaStream_t s) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(solve_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(solve_tc_kernel), kSmemBytes);
+  if (e != cudaSuccess) return e;
   SolveArgs a{p.B, p.H, p.T, p.ready, p.gready, p.A, p.Bm, p.alpha, p.M, p.C, static_cast<uint8_t*>(p.Msplit),
               p.status, p.spin_limit, p.pform};
   const long long n = (long long)p.B * p.H * (p.T - 1);
