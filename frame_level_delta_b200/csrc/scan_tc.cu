@@ -15,6 +15,14 @@
 // layout the solve wrote) arrive by bulk copies, double-buffered; C_t rows are
 // prefetched into registers (and into L2 two steps ahead) during the MMAs.
 //
+// In frame mode after the sweep solve (the default path) the step is written
+// as S <- (S Diag(alpha_t) + B_t) P_t, which equals S M_t + C_t: the solve then
+// writes only P_t's images, and the epilogue of step t forms the next step's
+// operand S Diag(alpha_{t+1}) + B_{t+1} (one FMA per element; alpha from a
+// four-deep ring of bulk copies, B rows prefetched) before it splits it into
+// the hi/lo A operand. The first operand is S_T/2 Diag(alpha) + B of the
+// direction's first frame.
+//
 // In frame mode the kernel may be launched while the solve's last CTAs still
 // run (programmatic dependent launch): the copy thread then acquires each
 // slot's ready word before it copies that slot's M_t or lets the epilogue read
