@@ -171,7 +171,58 @@ class VDA:
             self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=self.device)
         return self.workspace
 
+    # -- argument checks (before any call into the library) -----------------------
+    def _expect(self, name: str, t, shape, dtype):
+        if not isinstance(t, torch.Tensor):
+            raise ValueError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+        if t.device.type != self.device.type or (self.device.index is not None and t.device.index != self.device.index):
+            raise ValueError(f"{name} is on {t.device}; this context runs on {self.device}")
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}; expected {tuple(shape)}")
+        if t.dtype != dtype:
+            raise ValueError(f"{name} has dtype {t.dtype}; expected {dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+
+    def check_inputs(self, inp: Dict[str, torch.Tensor]):
+        """Raise ValueError unless every input of vda_prepare has the device,
+        shape, dtype and contiguous layout the C ABI takes."""
+        cfg = self.cfg
+        B, H, d, T, U, L = cfg.B, cfg.H, cfg.d, cfg.T, cfg.U, cfg.L
+        sd = torch.float32 if cfg.dtype == "f32" else torch.bfloat16
+        f32 = torch.float32
+        spec = {"Q": ((B, T * U, H, d), sd), "K": ((B, T * U, H, d), sd), "V": ((B, T * U, H, d), sd),
+                "K_txt": ((B, L, H, d), sd), "V_txt": ((B, L, H, d), sd), "alpha": ((B, H, T, d), f32),
+                "beta": ((B, H, T, U), f32), "beta_txt": ((B, H, L), f32)}
+        if cfg.prep_conv:
+            spec["conv_w"] = ((H * d * 60,), f32)
+        for name, (shape, dt) in spec.items():
+            if name not in inp:
+                raise ValueError(f"missing input {name}")
+            self._expect(name, inp[name], shape, dt)
+
+    def check_output(self, O: torch.Tensor, gate: Optional[torch.Tensor] = None):
+        """Raise ValueError unless O (and the gate, when given) match the C ABI."""
+        cfg = self.cfg
+        sd = torch.float32 if cfg.dtype == "f32" else torch.bfloat16
+        shape = (cfg.B, cfg.T * cfg.U, cfg.H, cfg.d)
+        self._expect("O", O, shape, sd)
+        if gate is not None:
+            self._expect("gate", gate, shape, sd)
+        elif cfg.norm_gate:
+            raise ValueError("gate is required by the normalised, gated readout")
+
+    def _on_device(self):
+        if self.device.type != "cuda":
+            raise ValueError(f"the library runs on CUDA devices; this context is on {self.device}")
+        return torch.cuda.device(self.device)
+
     def prepare(self, inp: Dict[str, torch.Tensor], stream=None):
+        self.check_inputs(inp)
+        with self._on_device():
+            self._prepare(inp, stream)
+
+    def _prepare(self, inp: Dict[str, torch.Tensor], stream=None):
         ws = self.ensure_workspace()
         self._keep = inp  # inputs must outlive the readout
         st = lib().vda_prepare(self._ctx, _ptr(inp["Q"]), _ptr(inp["K"]), _ptr(inp["V"]), _ptr(inp["K_txt"]),
@@ -180,10 +231,13 @@ class VDA:
         self._check(st, "vda_prepare")
 
     def scan_bidir(self, stream=None):
-        self._check(lib().vda_scan_bidir(self._ctx, _stream_handle(stream)), "vda_scan_bidir")
+        with self._on_device():
+            self._check(lib().vda_scan_bidir(self._ctx, _stream_handle(stream)), "vda_scan_bidir")
 
     def readout(self, O: torch.Tensor, gate: Optional[torch.Tensor] = None, stream=None):
-        self._check(lib().vda_readout(self._ctx, _ptr(gate), _ptr(O), _stream_handle(stream)), "vda_readout")
+        self.check_output(O, gate)
+        with self._on_device():
+            self._check(lib().vda_readout(self._ctx, _ptr(gate), _ptr(O), _stream_handle(stream)), "vda_readout")
 
     def new_output(self) -> torch.Tensor:
         cfg = self.cfg
@@ -194,13 +248,18 @@ class VDA:
         """One pass of the whole path: prepare, bidirectional scan, readout."""
         if O is None:
             O = self.new_output()
-        self.prepare(inp, stream)
-        self.scan_bidir(stream)
-        self.readout(O, inp.get("gate"), stream)
+        gate = inp.get("gate")
+        self.check_inputs(inp)
+        self.check_output(O, gate)
+        with self._on_device():
+            self._prepare(inp, stream)
+            self._check(lib().vda_scan_bidir(self._ctx, _stream_handle(stream)), "vda_scan_bidir")
+            self._check(lib().vda_readout(self._ctx, _ptr(gate), _ptr(O), _stream_handle(stream)), "vda_readout")
         return O
 
     def poll_device_status(self, stream=None) -> int:
-        return lib().vda_poll_device_status(self._ctx, _stream_handle(stream))
+        with self._on_device():
+            return lib().vda_poll_device_status(self._ctx, _stream_handle(stream))
 
     def region(self, name: str) -> torch.Tensor:
         """A view of one workspace region (float32 unless it is a prepared token copy)."""

@@ -186,3 +186,41 @@ def test_region_view_decodes_operand_images():
             img[byte // 2] = vals[i, j]
     out = _from_images(img.view(torch.uint8), (1,), D)[0]
     assert torch.equal(out, vals.bfloat16().float())
+
+
+def test_binding_checks_tensors_before_calling_the_library():
+    """The Python binding rejects inputs the C ABI would misread (wrong device,
+    shape, dtype or layout) before any call that could reach a kernel."""
+    import torch
+    from frame_level_delta_b200.inputs import make_inputs
+
+    cfg = CONFIGS["hires"].with_(H=2, T=5, grid_h=3, grid_w=4, L=3)
+    inp = make_inputs(cfg)
+    O = torch.empty(cfg.B, cfg.T * cfg.U, cfg.H, cfg.d, dtype=inp["Q"].dtype)
+    host = V.VDA(cfg, device="cpu")  # checks only: a CPU context never calls the library
+    host.check_inputs(inp)
+    host.check_output(O, inp["gate"])
+    with pytest.raises(ValueError, match="CUDA devices"):
+        host.run(inp, O)
+
+    def bad(mutate, match):
+        x = dict(inp)
+        mutate(x)
+        with pytest.raises(ValueError, match=match):
+            host.check_inputs(x)
+
+    bad(lambda x: x.pop("beta"), "missing input beta")
+    bad(lambda x: x.update(Q=inp["Q"][:, :-1]), "shape")
+    bad(lambda x: x.update(alpha=inp["alpha"].double()), "dtype")
+    bad(lambda x: x.update(K=inp["K"].transpose(2, 3).contiguous().transpose(2, 3)), "contiguous")
+    bad(lambda x: x.update(conv_w=inp["conv_w"][:-1]), "shape")
+    with pytest.raises(ValueError, match="gate is required"):
+        host.check_output(O, None)
+    with pytest.raises(ValueError, match="shape"):
+        host.check_output(O[:, :-1], inp["gate"])
+    # a CUDA context handed host tensors refuses them before any library call
+    dev = V.VDA(cfg, device="cuda")
+    with pytest.raises(ValueError, match="is on cpu"):
+        dev.prepare(inp)
+    with pytest.raises(ValueError, match="is on cpu"):
+        dev.run(inp, O)
