@@ -29,7 +29,10 @@
  * is > T-2); anchor frames read out exactly zero.
  *
  * Conventions shared by every call:
- *  - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *  - All tensor pointers are DEVICE pointers owned by the caller, in memory of
+ *    the device that is current when the call is made. The library does not
+ *    check what kind of memory a pointer addresses (a host pointer reaches the
+ *    kernels as it is); the Python binding checks its tensors first. The library
  *    never allocates or frees device memory; its only device memory is the
  *    caller's workspace.
  *  - Every call only enqueues work on the caller's CUDA stream (passed as
@@ -112,8 +115,10 @@ vda_status vda_workspace_size(const vda_config* cfg, size_t* bytes);
 
 /*
  * Stage 1: feature prep (VDA_PREP_CONV only), frame statistics A_t, B_t for the
- * text slot and frames 1..T-2, and the frame solve (Cholesky of I + A_t) giving
- * M_t, C_t and S_T. Layouts (row-major, innermost last):
+ * text slot and frames 1..T-2, and the frame solve giving S_T and each frame's
+ * transition and injection (the inverse of I + A_t by the symmetric sweep, or by
+ * Cholesky under VDA_SOLVE_CHOLESKY; see VDA_REGION_C and VDA_REGION_M_SPLIT for
+ * what is stored). Layouts (row-major, innermost last):
  *   Q, K, V       [B, T*U, H, d]   token-major with heads interleaved; token
  *                                  index t*U + u for frame t, grid position u
  *   K_txt, V_txt  [B, L, H, d]
