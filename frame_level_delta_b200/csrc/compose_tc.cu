@@ -1,7 +1,7 @@
 // Chunk composition for the bidirectional scan (Video DeltaNet summary,
-// onedev.kr/papers/80, section "how to use", kernel notes: the frame maps of a
-// VAE chunk compose into S_out = S_in M_chunk + J_chunk, and the shorter chunk
-// sequence is scanned in both directions).
+// onedev.kr/papers/80, section "assumptions and limits", notes on the inference
+// kernels: the frame maps of a VAE chunk compose into S_out = S_in M_chunk +
+// J_chunk, and the shorter chunk sequence is scanned in both directions).
 //
 // One CTA per (chunk m, direction, b*h). The forward direction composes the
 // chunk's non-anchor frames in increasing order, the reverse direction in

@@ -159,7 +159,8 @@ def text_state(A_txt: np.ndarray, B_txt: np.ndarray) -> np.ndarray:
     """S_T: the frame solve from S = 0 over the text tokens, B_txt (I + A_txt)^-1.
 
     [P1 "how it works": all text tokens are summarised into S_T before the video
-    scan; P1 "how to use" (kernel notes): the prompt enters as a leading virtual frame.]
+    scan; P1 "assumptions and limits" (notes on the inference kernels): the
+    prompt enters as a leading virtual frame.]
     (I + A) is symmetric, so S (I + A) = B is the transpose of (I + A) S^T = B^T.
     """
     d_k = A_txt.shape[0]
