@@ -368,6 +368,24 @@ def blas_threads() -> int:
     return len(os.sched_getaffinity(0))
 
 
+def blas_library() -> str:
+    """The BLAS numpy calls into, as threadpoolctl reports it (library and version)."""
+    try:
+        import threadpoolctl
+        for d in threadpoolctl.threadpool_info():
+            if d.get("user_api") == "blas":
+                return f"{d.get('internal_api')} {d.get('version')} ({os.path.basename(str(d.get('filepath')))})"
+    except Exception:
+        pass
+    return "unknown"
+
+
+def one_blas_thread():
+    """Context manager limiting numpy's BLAS to one thread."""
+    import threadpoolctl
+    return threadpoolctl.threadpool_limits(limits=1, user_api="blas")
+
+
 def time_oracle(cfg, inp, heads, budget_s=None):
     from oracle.vda_oracle import vda_reference
     done = 0
@@ -382,12 +400,22 @@ def time_oracle(cfg, inp, heads, budget_s=None):
 
 
 def cpu_baseline(cfg, inp, budget_s=10.0):
+    """The float64 oracle on the host cores: all the BLAS threads the process may
+    use for ~budget_s, then one BLAS thread for ~budget_s / 2."""
     heads = [(b, h) for b in range(cfg.B) for h in range(cfg.H)]
+    threads = blas_threads()
     done, dt = time_oracle(cfg, inp, heads, budget_s=budget_s)
     value = done * cfg.T * cfg.U / dt
-    return {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+    with one_blas_thread():
+        done1, dt1 = time_oracle(cfg, inp, heads, budget_s=budget_s / 2)
+    value1 = done1 * cfg.T * cfg.U / dt1
+    return {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "blas": blas_library(), "host_cpus": len(os.sched_getaffinity(0)),
+            "one_thread": {"value": value1, "unit": UNIT, "cores": 1,
+                           "sample": f"{done1} (batch, head) pairs, {dt1:.2f} s"},
             "sample": f"float64 numpy oracle over {done} of {len(heads)} (batch, head) pairs of the "
-                      f"workload ({cfg.T * cfg.U} tokens each), {dt:.2f} s, BLAS threads={blas_threads()}"}
+                      f"workload ({cfg.T * cfg.U} tokens each), {dt:.2f} s, BLAS threads={threads} "
+                      f"({blas_library()})"}
 
 
 def run_reference(args, cfg, rank):
@@ -408,6 +436,7 @@ def run_reference(args, cfg, rank):
             "impl": "reference",
             "config": {"workload": workload_desc(cfg), "step": "one (batch, head) pair of the workload"},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "blas": blas_library(),
                              "sample": f"one (batch, head) pair per step, {cfg.T * cfg.U} tokens"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

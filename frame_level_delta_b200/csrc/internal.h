@@ -135,6 +135,8 @@ cudaError_t launch_scan_simt(const Problem& p, cudaStream_t s);
 cudaError_t launch_readout_simt(const Problem& p, const void* gate, void* O, cudaStream_t s);
 cudaError_t launch_zero_anchors(const Problem& p, void* O, cudaStream_t s);
 cudaError_t launch_selftest_wait(uint32_t* status, unsigned long long spins, cudaStream_t s);
+// The sweep solve's pivot reciprocal applied to x[0..n) (for an error bound test).
+cudaError_t launch_recip_selftest(const float* x, float* y, int n, cudaStream_t s);
 
 // Tensor-core (tcgen05) kernels, bf16 with D in {64, 128}.
 bool gram_tc_supported(const Problem& p);

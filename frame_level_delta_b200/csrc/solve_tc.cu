@@ -86,9 +86,12 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// 1 / d by the hardware's approximate reciprocal plus one Newton-Raphson step
-// (r <- r + r (1 - d r)), which leaves about one ulp of error. Pivots of I + A
-// are >= 1, so no special cases arise.
+// 1 / d by the hardware's approximate reciprocal refined with one step of
+// Newton's iteration for the reciprocal (the Newton-Raphson method applied to
+// f(r) = 1/r - d: r <- r + r (1 - d r), which roughly squares the relative
+// error of the starting value); about one ulp of error remains. Pivots of
+// I + A are >= 1, so no special cases arise. vda_selftest_recip runs this same
+// function so a test can bound its error against the correctly rounded 1/d.
 __device__ __forceinline__ float recip(float d) {
   float r;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(d));
@@ -427,9 +430,20 @@ __global__ void __launch_bounds__(kThreads, 3) solve_tc_kernel(const SolveArgs a
   }
 }
 
+__global__ void recip_selftest_kernel(const float* x, float* y, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = recip(x[i]);
+}
+
 }  // namespace
 
 bool solve_tc_supported(const Problem& p) { return p.bf16 && p.D == 128; }
+
+cudaError_t launch_recip_selftest(const float* x, float* y, int n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  recip_selftest_kernel<<<(n + 255) / 256, 256, 0, s>>>(x, y, n);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_solve_tc(const Problem& p, cudaStream_t s) {
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(solve_tc_kernel), kSmemBytes);

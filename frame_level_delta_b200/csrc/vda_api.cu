@@ -477,4 +477,10 @@ vda_status vda_selftest_bounded_wait(uint32_t* status_dev, uint64_t spins, void*
   return e == cudaSuccess ? VDA_OK : VDA_ERR_CUDA;
 }
 
+vda_status vda_selftest_recip(const float* x, float* y, int n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return VDA_ERR_INVALID_ARG;
+  cudaError_t e = launch_recip_selftest(x, y, n, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VDA_OK : VDA_ERR_CUDA;
+}
+
 }  // extern "C"

@@ -34,7 +34,8 @@ EXPORTS = ["vda_create", "vda_destroy", "vda_workspace_size", "vda_prepare", "vd
            "vda_readout", "vda_poll_device_status", "vda_workspace_region", "vda_status_string",
            "vda_last_error", "vda_profile_enable", "vda_num_kernels", "vda_profile_read",
            "vda_launch_count", "vda_describe", "vda_selftest_bounded_wait",
-           "vda_static_workspace_capacity", "vda_run_static_workspace"]
+           "vda_selftest_recip", "vda_static_workspace_capacity", "vda_run_static_workspace",
+           "vda_static_workspace_poll"]
 
 
 class VDAError(RuntimeError):
@@ -83,6 +84,8 @@ def lib() -> ctypes.CDLL:
         L.vda_launch_count.argtypes = [vp, ctypes.POINTER(ctypes.c_uint64)]
         L.vda_describe.argtypes = [cfgp, ctypes.POINTER(ctypes.c_char_p)]
         L.vda_selftest_bounded_wait.argtypes = [vp, ctypes.c_uint64, vp]
+        L.vda_selftest_recip.argtypes = [vp, vp, i, vp]
+        L.vda_static_workspace_poll.argtypes = [vp]
         L.vda_static_workspace_capacity.argtypes = []
         L.vda_static_workspace_capacity.restype = ctypes.c_size_t
         L.vda_run_static_workspace.argtypes = [cfgp] + [vp] * 11 + [vp]
@@ -334,6 +337,23 @@ def run_static_workspace(cfg: VDAConfig, inp: Dict[str, torch.Tensor], O: torch.
         ctypes.byref(c), _ptr(inp["Q"]), _ptr(inp["K"]), _ptr(inp["V"]), _ptr(inp["K_txt"]), _ptr(inp["V_txt"]),
         _ptr(inp["alpha"]), _ptr(inp["beta"]), _ptr(inp["beta_txt"]), _ptr(inp.get("conv_w")),
         _ptr(inp.get("gate")), _ptr(O), _stream_handle(stream))
+
+
+def static_workspace_poll(stream=None) -> int:
+    """Status of the last vda_run_static_workspace call on the current device
+    (synchronises the stream; VDA_ERR_TIMEOUT if a device-side wait gave up)."""
+    return lib().vda_static_workspace_poll(_stream_handle(stream))
+
+
+def selftest_recip(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """The sweep solve's pivot reciprocal applied to a float32 CUDA tensor."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 CUDA tensor")
+    y = torch.empty_like(x)
+    st = lib().vda_selftest_recip(_ptr(x), _ptr(y), x.numel(), _stream_handle(stream))
+    if st != VDA_OK:
+        raise VDAError(st, "vda_selftest_recip")
+    return y
 
 
 def selftest_bounded_wait(status: torch.Tensor, spins: int, stream=None) -> int:

@@ -176,10 +176,13 @@ vda_status vda_poll_device_status(vda_ctx* ctx, void* stream);
  */
 typedef enum vda_region {
   VDA_REGION_STATUS = 0, /* uint32 device status word (+ padding to byte 256), then uint32 [B, H, T-1]
-                            slot-ready words: vda_prepare clears the region, the tensor-core sweep
-                            solve sets word (b, h, s) to 1 once slot s's C_t and M_t are written, and
-                            the tensor-core frame scan (which may start while the solve's last CTAs
-                            run) reads a slot only after its word is 1 */
+                            slot-ready words of the solve, then uint32 [B, H, T-1] slot counts of the
+                            statistics kernel: vda_prepare clears the region; the tensor-core sweep
+                            solve sets word (b, h, s) to 1 once everything the scan reads from slot s
+                            is written (the hi/lo images of M_t, or of P_t under "inject=scan", and
+                            C_t where it is formed; S_T for the text slot), and the tensor-core frame
+                            scan (which may start while the solve's last CTAs run) reads a slot only
+                            after its word is 1 */
   VDA_REGION_A = 1,      /* float32 [B, H, T-1, d_k, d_k]; slot 0 = text, slot t = frame t */
   VDA_REGION_B = 2,      /* float32 [B, H, T-1, d_v, d_k]; same slots */
   VDA_REGION_M = 3,      /* float32 [B, H, T-1, d_k, d_k]; slot t = M_t (slot 0 unused); written by the
@@ -244,6 +247,15 @@ vda_status vda_describe(const vda_config* cfg, const char** text);
 vda_status vda_selftest_bounded_wait(uint32_t* status_dev, uint64_t spins, void* stream);
 
 /*
+ * Numerical self test of the sweep solve's pivot reciprocal: y[i] = r(x[i]) for
+ * i < n, where r is the device function every pivot step of the tensor-core
+ * sweep uses (the hardware's approximate reciprocal refined by one Newton-Raphson
+ * step). x and y are device float32 arrays of n values. Lets a test bound r's
+ * error against the correctly rounded 1/x over the pivot range (x >= 1).
+ */
+vda_status vda_selftest_recip(const float* x, float* y, int n, void* stream);
+
+/*
  * The whole path (vda_prepare, vda_scan_bidir, vda_readout) in one call whose
  * scratch lives in a static device array owned by the library, for callers that
  * cannot allocate device memory: code that has no allocator at hand (a plugin
@@ -262,6 +274,8 @@ vda_status vda_selftest_bounded_wait(uint32_t* status_dev, uint64_t spins, void*
  *    overlap on the GPU (other streams, other host threads) race and corrupt each
  *    other's results, so serialise them.
  *  - No cudaMalloc, cudaFree or allocating library routine is called.
+ *  - A bounded device-side wait that gives up does not change the return code
+ *    (the call only enqueues work): read it with vda_static_workspace_poll.
  * Arguments are those of vda_prepare and vda_readout; the call only enqueues
  * work on `stream`.
  */
@@ -270,6 +284,17 @@ vda_status vda_run_static_workspace(const vda_config* cfg, const void* Q, const 
                                     const void* K_txt, const void* V_txt, const float* alpha,
                                     const float* beta, const float* beta_txt, const float* conv_w,
                                     const void* gate, void* O, void* stream);
+
+/*
+ * The device status word of the static array, for vda_run_static_workspace
+ * what vda_poll_device_status is for the caller-workspace calls: synchronise
+ * `stream`, read the word, clear it, and return VDA_ERR_TIMEOUT if a bounded
+ * device-side wait of the last call on this device gave up, VDA_OK otherwise.
+ * Each vda_run_static_workspace call clears the word when it starts, so poll
+ * after a call and before the next one. Allocates nothing; the first use on a
+ * device looks up the array's address as vda_run_static_workspace does.
+ */
+vda_status vda_static_workspace_poll(void* stream);
 
 #ifdef __cplusplus
 }

@@ -35,8 +35,11 @@ def test_small_bf16(force_simt):
     check_config(CONFIGS["small"], force_simt=force_simt)
 
 
-def test_h3_full_size_sampled_heads():
-    check_config(CONFIGS["h3"], heads=[(0, 0), (0, 11), (0, 23)])
+def test_h3_full_size_all_heads():
+    """The H3-like clip at full size, every one of its 24 heads against the
+    oracle: whole-output, per-(head, frame) and per-token bounds, and the staged
+    intermediates of every slot and chunk of every head."""
+    check_config(CONFIGS["h3"])
 
 
 def test_h3_full_size_cholesky_solve():
@@ -47,32 +50,33 @@ def test_h3_full_size_chunked_scan():
     check_config(CONFIGS["h3"], heads=[(0, 7), (0, 16)], chunked=True)
 
 
-def test_long_full_size_sampled_heads():
-    check_config(CONFIGS["long"], heads=[(0, 5), (0, 23)])
+# Six heads spread over the head range (first, last and four between).
+SPREAD_HEADS = [(0, 0), (0, 5), (0, 10), (0, 14), (0, 19), (0, 23)]
 
 
-def test_hires_full_size_sampled_heads():
+def test_long_full_size_spread_heads():
+    check_config(CONFIGS["long"], heads=SPREAD_HEADS)
+
+
+def test_hires_full_size_spread_heads():
+    """The high-res clip with conv prep and the gated readout at full size, on six
+    heads: output bounds (whole, per frame, per token), every staged
+    intermediate, and the prepared keys and values against the oracle's prep."""
     cfg = CONFIGS["hires"]
     inp = make_inputs(cfg)
-    O_gpu, regions, lib = run_gpu(cfg, inp)
-    heads = [(0, 0), (0, 13)]
-    ref = vo.vda_reference(inp, cfg, heads=heads)
-    O_ref = ref["O"]
-    for (_, h) in heads:
-        assert rel_fro(O_gpu[0, :, h].numpy(), O_ref[0, :, h]) <= TOL_O["bf16"]
-    # Prepared keys/values against the oracle's prep (bf16 storage of the copy).
+    _, _, regions = check_config(cfg, heads=SPREAD_HEADS, inp=inp, return_regions=True)
     w = inp["conv_w"].double().numpy()
     hd = cfg.H * cfg.d
-    for (_, h) in heads:
-        K = inp["K"][0, :, h].double().numpy().reshape(cfg.T, cfg.U, cfg.d)
-        Kp = vo.l2_normalize(vo.prep_video_kv(K, w[:hd * 25].reshape(cfg.H, cfg.d, 5, 5)[h],
-                                              w[hd * 25:hd * 30].reshape(cfg.H, cfg.d, 5)[h],
-                                              cfg.grid_h, cfg.grid_w), 1e-6)
-        got = regions["K_prep"][0, h, 1:cfg.T - 1].numpy()
-        assert rel_fro(got, Kp[1:cfg.T - 1]) <= 5e-3
-    assert torch.isfinite(O_gpu).all()
-    U, T = cfg.U, cfg.T
-    assert (O_gpu[:, :U] == 0).all() and (O_gpu[:, (T - 1) * U:] == 0).all()
+    for (_, h) in SPREAD_HEADS:
+        for which, off in (("K", 0), ("V", hd * 30)):
+            X = inp[which][0, :, h].double().numpy().reshape(cfg.T, cfg.U, cfg.d)
+            want = vo.prep_video_kv(X, w[off:off + hd * 25].reshape(cfg.H, cfg.d, 5, 5)[h],
+                                    w[off + hd * 25:off + hd * 30].reshape(cfg.H, cfg.d, 5)[h],
+                                    cfg.grid_h, cfg.grid_w)
+            if which == "K":
+                want = vo.l2_normalize(want, 1e-6)
+            got = regions[which + "_prep"][0, h, 1:cfg.T - 1].numpy()
+            assert rel_fro(got, want[1:cfg.T - 1]) <= 5e-3, (which, h)
 
 
 def test_low_write_long_memory_diagnostic():
@@ -255,3 +259,25 @@ def test_launch_accounting_and_profiling():
     prof = lib.profile_read()
     assert sum(v[0] for v in prof.values()) == n
     assert all(v[1] > 0 for v in prof.values())
+
+
+def test_pivot_reciprocal_error_bound():
+    """The sweep solve's pivot reciprocal (hardware approximation plus one
+    Newton-Raphson step) against the correctly rounded 1/x, over the pivot range
+    x in [1, 1e4]: log-spaced values, powers of two and random draws. Every
+    result must lie within two ulps (2^-22 relative) of the exact reciprocal,
+    and its rounding error against CUDA's correctly rounded 1.0f/x is at most
+    one ulp."""
+    g = torch.Generator().manual_seed(0)
+    xs = torch.cat([torch.logspace(0, 4, 200001, dtype=torch.float64).float(),
+                    torch.tensor([2.0 ** k for k in range(14)]),
+                    1 + torch.rand(100000, generator=g) * 9999]).contiguous()
+    y = V.selftest_recip(xs.cuda()).cpu()
+    exact = 1.0 / xs.double()
+    rel = ((y.double() - exact).abs() / exact).max().item()
+    assert rel <= 2.0 ** -22, rel
+    cr = exact.float()  # the correctly rounded reciprocal (what IEEE 1.0f / x returns)
+    ulp = torch.nextafter(cr, torch.full_like(cr, float("inf"))) - cr
+    assert ((y - cr).abs() <= ulp).all()
+    dev_div = (1.0 / xs.cuda()).cpu()  # CUDA's own division, for the record
+    assert ((dev_div - cr).abs() <= ulp).all()
