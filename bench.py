@@ -7,9 +7,13 @@ storage, fp32 state), with inputs resident in HBM. Prints one JSON line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config h3] [--impl reference]
 
-N > 1 is launched with torch.distributed.run: every rank processes its own
-batch (independent problems, no data-path collective: weak scaling); the timed
-region is bracketed by barriers and the time is the max over ranks.
+N > 1 runs one process per GPU under torch.distributed.run (bench.py starts
+it itself when launched without RANK in the environment). `--shard batch`
+(default): every rank processes its own batch (independent problems, weak
+scaling). `--shard heads`: the ranks share one batch and each serves a slice of
+its heads in place (vda_config.H_total, h0; strong scaling). Neither form has a
+data-path collective; the timed region is bracketed by barriers and the time is
+the max over ranks.
 `--impl reference` times the float64 CPU oracle on the host cores instead (rank
 0 only), one (batch, head) pair of the workload per step.
 """
@@ -63,9 +67,24 @@ def rank_env():
             int(os.environ.get("LOCAL_RANK", "0")))
 
 
-def rank_seed(cfg, rank: int) -> int:
-    """Seed of the batch a rank draws: independent problems per rank."""
-    return cfg.seed + rank
+def rank_seed(cfg, rank: int, shard: str = "batch") -> int:
+    """Seed of the batch a rank draws: independent problems per rank, or the one
+    shared batch when the ranks split its heads."""
+    return cfg.seed + (rank if shard == "batch" else 0)
+
+
+def relaunch_under_torchrun(argv, gpus: int) -> int:
+    """Run this script again as `gpus` ranks under torch.distributed.run (one
+    process per GPU of this node, rendezvous on 127.0.0.1) and return its exit
+    code."""
+    import socket
+    import subprocess
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + list(argv)
+    return subprocess.call(cmd)
 
 
 def init_ranks(world: int, device, timeout_s: float = 120.0):
@@ -95,9 +114,11 @@ def max_over_ranks(dist, ms: float, device) -> float:
     return float(t.item())
 
 
-def whole_job_rate(world: int, cfg, steps: int, ms_max: float) -> float:
-    """Head-tokens all ranks processed divided by the slowest rank's time."""
-    return world * cfg.head_tokens * steps / (ms_max / 1e3)
+def whole_job_rate(world: int, cfg, steps: int, ms_max: float, shard: str = "batch") -> float:
+    """Head-tokens all ranks processed divided by the slowest rank's time (each
+    rank a batch; or, with the heads split, one batch among them all)."""
+    batches = world if shard == "batch" else 1
+    return batches * cfg.head_tokens * steps / (ms_max / 1e3)
 
 
 # ----------------------------------------------------------------------------
@@ -418,7 +439,7 @@ def cpu_baseline(cfg, inp, budget_s=10.0):
                       f"({blas_library()})"}
 
 
-def run_reference(args, cfg, rank):
+def run_reference(args, cfg, rank, world):
     if rank != 0:
         return 0
     inp = make_inputs(cfg)
@@ -430,7 +451,7 @@ def run_reference(args, cfg, rank):
         time_oracle(cfg, inp, [heads[i % len(heads)]])
     dt = time.perf_counter() - t0
     value = args.steps * cfg.T * cfg.U / dt
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
@@ -459,29 +480,44 @@ def main():
                     help="tensor-core scan frame by frame (default) or over composed chunk maps")
     ap.add_argument("--heads", type=int, default=0,
                     help="override H (a smaller case of the same workload, e.g. for profiler captures)")
+    ap.add_argument("--shard", default="batch", choices=["batch", "heads"],
+                    help="N > 1: a batch per rank (weak scaling) or one batch's heads split over the ranks")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if args.gpus > 1 and "RANK" not in os.environ:
+        return relaunch_under_torchrun(sys.argv[1:], args.gpus)
     cfg = CONFIGS[args.config]
     if args.heads > 0:
         cfg = cfg.with_(H=args.heads)
     rank, world, local = rank_env()
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch one rank per GPU")
     if args.impl == "reference":
-        return run_reference(args, cfg, rank)
+        return run_reference(args, cfg, rank, world)
 
     from frame_level_delta_b200 import vda as V
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     dist = init_ranks(world, dev)
 
-    # Each rank draws its own batch (independent problems).
-    inp_cpu = make_inputs(cfg, seed=rank_seed(cfg, rank))
+    # Each rank draws its own batch (independent problems), or all draw the one
+    # batch whose heads they split.
+    inp_cpu = make_inputs(cfg, seed=rank_seed(cfg, rank, args.shard))
+    heads = None
+    if args.shard == "heads" and world > 1:
+        from frame_level_delta_b200.shard import head_partition
+        heads = head_partition(cfg.H, world)[rank]
     inp_host = {k: v.pin_memory() for k, v in inp_cpu.items()}
     inp_dev = {k: v.to(dev, non_blocking=True) for k, v in inp_host.items()}
     global SCAN_CHUNKED, SOLVE_CHOLESKY
     SCAN_CHUNKED = args.scan == "chunked"
     SOLVE_CHOLESKY = args.solve == "cholesky"
-    lib = V.VDA(cfg, device=dev, cholesky=args.solve == "cholesky", chunked=SCAN_CHUNKED)
+    lib = V.VDA(cfg, device=dev, cholesky=args.solve == "cholesky", chunked=SCAN_CHUNKED, heads=heads)
+    # Per-kernel accounting below is for the heads this rank serves.
+    kcfg = cfg if heads is None else cfg.with_(H=heads[1])
     O = lib.new_output()
     stream = torch.cuda.current_stream(dev)
     for _ in range(args.warmup):
@@ -530,7 +566,7 @@ def main():
     if lib.poll_device_status() != 0:
         raise RuntimeError("device status reported a timeout in the per-kernel pass")
     ms_max = max_over_ranks(dist, ms, dev)
-    value = whole_job_rate(world, cfg, args.steps, ms_max)
+    value = whole_job_rate(world, cfg, args.steps, ms_max, args.shard)
 
     # ---- end to end through the public API: pinned host inputs -> device ->
     # prepare/scan/readout -> O back to pinned host memory, every step. The
@@ -578,26 +614,26 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(dist)
-    e2e_value = whole_job_rate(world, cfg, ke, max_over_ranks(dist, e0.elapsed_time(e1), dev))
+    e2e_value = whole_job_rate(world, cfg, ke, max_over_ranks(dist, e0.elapsed_time(e1), dev), args.shard)
 
     # ---- roofline of the dominant kernel (live per-kernel CUDA events) -------
     peaks, peak_src = load_peaks()
     dom = max(prof.items(), key=lambda kv: kv[1][1])
     dom_name, (dom_n, dom_ms) = dom
     dom_avg_s = dom_ms / dom_n / 1e3
-    dom_bytes = kernel_bytes(dom_name, cfg)
-    traffic = traffic_for(dom_name, cfg.name)
+    dom_bytes = kernel_bytes(dom_name, kcfg)
+    traffic = traffic_for(dom_name, cfg.name) if heads is None else None
     if dom_name in ALU_BOUND:
         bound, unit = "alu", "TFLOP/s"
         sm_mhz = float(clocks.summary().get("sm_mhz") or 1965.0)
-        achieved = kernel_alu_flops(dom_name, cfg) / dom_avg_s / 1e12
+        achieved = kernel_alu_flops(dom_name, kcfg) / dom_avg_s / 1e12
         peak = alu_peak_tflops(sm_mhz)
         peak_note = (f"fp32 FMA peak derived: 148 SMs x 128 lanes x 2 flop x {sm_mhz:.0f} MHz "
                      f"(median SM clock in the timed region)")
     elif dom_name in TENSOR_BOUND:
         # timed inside a long step: the sustained bf16 figure is the denominator
         bound, unit = "tensor", "TFLOP/s"
-        achieved = kernel_flops(dom_name, cfg) / dom_avg_s / 1e12
+        achieved = kernel_flops(dom_name, kcfg) / dom_avg_s / 1e12
         peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
         peak_note = f"bf16_tflops_sustained of {peak_src}"
     else:
@@ -607,9 +643,9 @@ def main():
         peak_note = f"hbm_gbs of {peak_src}"
     hbm_peak = float(peaks["hbm_gbs"])
     kernels = {k: {"launches": n, "avg_us": tot / n * 1e3, "share": tot / sum(x[1] for x in prof.values()),
-                   "algorithmic_GBps": kernel_bytes(k, cfg) / (tot / n / 1e3) / 1e9,
-                   "hbm_frac": kernel_bytes(k, cfg) / (tot / n / 1e3) / 1e9 / hbm_peak,
-                   "algorithmic_TFLOPs": kernel_flops(k, cfg) / (tot / n / 1e3) / 1e12}
+                   "algorithmic_GBps": kernel_bytes(k, kcfg) / (tot / n / 1e3) / 1e9,
+                   "hbm_frac": kernel_bytes(k, kcfg) / (tot / n / 1e3) / 1e9 / hbm_peak,
+                   "algorithmic_TFLOPs": kernel_flops(k, kcfg) / (tot / n / 1e3) / 1e12}
                for k, (n, tot) in prof.items()}
 
     if rank == 0:
@@ -617,10 +653,11 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32",
+            "scaling": "weak" if args.shard == "batch" else "strong", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32",
             "data": "synthetic",
-            "config": {"workload": workload_desc(cfg), "global_batch": cfg.B * world,
-                       "parallelism": f"dp{world} (independent batches, no collective)",
+            "config": {"workload": workload_desc(cfg), "global_batch": cfg.B * (world if args.shard == "batch" else 1),
+                       "parallelism": (f"dp{world} (independent batches, no collective)" if args.shard == "batch"
+                                       else f"heads{world} (one batch, heads {heads} on rank 0, no collective)"),
                        "l2": "no flush: each step reads and writes > 1 GB, far above the 126 MB L2",
                        "path": V.describe(lib.c),
                        "stream": "one CUDA stream, kernels back to back"},
@@ -628,13 +665,13 @@ def main():
                          "unit": unit, "frac": achieved / peak, "traffic": traffic,
                          "peak_source": peak_note,
                          "algorithmic_bytes_per_launch": dom_bytes,
-                         "algorithmic_flops_per_launch": kernel_flops(dom_name, cfg),
-                         "alu_flops_per_launch": kernel_alu_flops(dom_name, cfg) or None},
-            "path_roofline": {"algorithmic_bytes_per_step": path_bytes(cfg),
-                              "hbm_GBps": path_bytes(cfg) / step_s / 1e9,
-                              "hbm_frac": path_bytes(cfg) / step_s / 1e9 / hbm_peak,
-                              "tflops": path_flops(cfg) / step_s / 1e12,
-                              "tensor_frac_of_bf16_burst": path_flops(cfg) / step_s / 1e12 / float(peaks["bf16_tflops"])},
+                         "algorithmic_flops_per_launch": kernel_flops(dom_name, kcfg),
+                         "alu_flops_per_launch": kernel_alu_flops(dom_name, kcfg) or None},
+            "path_roofline": {"algorithmic_bytes_per_step": path_bytes(kcfg),
+                              "hbm_GBps": path_bytes(kcfg) / step_s / 1e9,
+                              "hbm_frac": path_bytes(kcfg) / step_s / 1e9 / hbm_peak,
+                              "tflops": path_flops(kcfg) / step_s / 1e12,
+                              "tensor_frac_of_bf16_burst": path_flops(kcfg) / step_s / 1e12 / float(peaks["bf16_tflops"])},
             "kernels": kernels,
             "kernel_pass": {"steps": args.steps, "ms_per_step": ms_profiled / args.steps,
                             "note": "per-kernel times, shares and the roofline come from this second pass of "

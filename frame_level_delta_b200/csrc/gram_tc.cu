@@ -359,20 +359,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 cudaError_t encode_maps(const Problem& p, CUtensorMap* mK, CUtensorMap* mV, CUtensorMap* mKt, CUtensorMap* mVt,
                         int* layout) {
-  const uint64_t D = p.D, H = p.H, T = p.T, U = p.U, L = p.L, B = p.B;
+  const uint64_t D = p.D, H = p.H, T = p.T, U = p.U, L = p.L, B = p.B, Ht = p.Ht;
   const bool prep = (p.flags & VDA_PREP_CONV) != 0;
   *layout = prep ? 1 : 0;
   cudaError_t e;
   if (!prep) {
-    // [B, T*U, H, D]: dims (d, h, u, t, b)
+    // [B, T*U, Ht, D] from this problem's first head on: dims (d, h, u, t, b)
     uint64_t dv[5] = {D, H, U, T, B};
-    uint64_t sv[4] = {D * 2, H * D * 2, U * H * D * 2, T * U * H * D * 2};
+    uint64_t sv[4] = {D * 2, Ht * D * 2, U * Ht * D * 2, T * U * Ht * D * 2};
     uint32_t box[5] = {64, 1, (uint32_t)kTileU, 1, 1};
     if ((e = make_tmap_bf16(mK, p.Kv.p, 5, dv, sv, box)) != cudaSuccess) return e;
     if ((e = make_tmap_bf16(mV, p.Vv.p, 5, dv, sv, box)) != cudaSuccess) return e;
-    // [B, L, H, D]: dims (d, h, u, 1, b)
+    // [B, L, Ht, D]: dims (d, h, u, 1, b)
     uint64_t dt[5] = {D, H, L, 1, B};
-    uint64_t st[4] = {D * 2, H * D * 2, L * H * D * 2, L * H * D * 2};
+    uint64_t st[4] = {D * 2, Ht * D * 2, L * Ht * D * 2, L * Ht * D * 2};
     if ((e = make_tmap_bf16(mKt, p.Kt.p, 5, dt, st, box)) != cudaSuccess) return e;
     if ((e = make_tmap_bf16(mVt, p.Vt.p, 5, dt, st, box)) != cudaSuccess) return e;
   } else {

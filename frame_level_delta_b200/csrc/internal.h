@@ -19,6 +19,11 @@ struct TokView {
 // Everything a kernel needs, passed by value.
 struct Problem {
   int B, H, T, U, L, D, c, J, gh, gw;
+  // Heads per token row of the token tensors (Q, K, V, K_txt, V_txt, gate, O):
+  // H_total of the config. Their pointers here are already advanced to the
+  // context's first head, so head h of this problem sits at channel offset h*D
+  // of a row of Ht*D values.
+  int Ht;
   int bf16;            // 1: token tensors are bf16, 0: fp32
   unsigned flags;
   float l2_eps, rms_eps;

@@ -417,7 +417,7 @@ __global__ void __launch_bounds__(256) readout_simt_kernel(Problem p, const void
   const long long co = chunk_off(p, b, h, j);
   for (int e = threadIdx.x; e < D * D; e += blockDim.x)
     sS[quad_row(D, e) * LD + quad_col(D, e)] = p.Sf[co + e] + p.Sr[co + e];
-  const long long rowstride = (long long)p.H * D;
+  const long long rowstride = (long long)p.Ht * D;
   const long long qbase = ((long long)b * p.T * p.U) * rowstride + (long long)h * D;
   for (int e = threadIdx.x; e < TT * D; e += blockDim.x) {
     const int uu = e / D, k = e % D;
@@ -462,19 +462,21 @@ __global__ void __launch_bounds__(256) readout_simt_kernel(Problem p, const void
   }
 }
 
-// Anchor frames 0 and T-1 read out exactly zero: for each batch element both
-// frames are contiguous ranges of U*H*D elements of O.
-// Grid (x, 2 * B): blockIdx.y names one contiguous slab (batch b, anchor frame
-// 0 or T-1) of U * H * D values; the x blocks stride over its 16-byte words.
+// Anchor frames 0 and T-1 read out exactly zero. For each batch element each
+// anchor frame is U token rows; this problem owns H * D values of each row
+// (row stride Ht * D, O already advanced to its first head).
+// Grid (x, 2 * B): blockIdx.y names one (batch b, anchor frame 0 or T-1); the x
+// blocks stride over the 16-byte words of its U rows.
 __global__ void zero_anchors_kernel(Problem p, void* O) {
-  const long long per = (long long)p.U * p.H * p.D;
   const int esz = p.bf16 ? 2 : 4;
-  const long long words = per * esz / 16;  // per is a multiple of 16 (D >= 16)
+  const long long rw = (long long)p.H * p.D * esz / 16;    // words of a row (H * D * esz is a multiple of 16)
+  const long long row16 = (long long)p.Ht * p.D * esz / 16;  // row stride in words
+  const long long words = (long long)p.U * rw;
   const long long b = blockIdx.y >> 1, frame = (blockIdx.y & 1) ? p.T - 1 : 0;
-  uint4* base = reinterpret_cast<uint4*>(static_cast<char*>(O) + (b * p.T + frame) * per * esz);
+  uint4* base = reinterpret_cast<uint4*>(static_cast<char*>(O) + (b * p.T + frame) * p.U * row16 * 16);
   for (long long w = blockIdx.x * (long long)blockDim.x + threadIdx.x; w < words;
        w += (long long)gridDim.x * blockDim.x)
-    base[w] = make_uint4(0, 0, 0, 0);
+    base[(w / rw) * row16 + w % rw] = make_uint4(0, 0, 0, 0);
 }
 
 // Text prep: SiLU on K_txt and V_txt, then L2 on K_txt; one warp per token.
@@ -484,7 +486,7 @@ __global__ void prep_text_kernel(Problem p, const void* Kt, const void* Vt) {
   const int D = p.D, H = p.H, L = p.L;
   if (warp >= p.B * L * H) return;
   const int h = warp % H, l = (warp / H) % L, b = warp / (H * L);
-  const long long ib = (((long long)b * L + l) * H + h) * D;
+  const long long ib = (((long long)b * L + l) * p.Ht + h) * D;
   const long long ob = (((long long)b * H + h) * L + l) * D;
   float ss = 0.f;
   for (int k = lane; k < D; k += 32) {

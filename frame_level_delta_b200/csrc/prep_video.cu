@@ -245,10 +245,13 @@ cudaError_t launch_typed(const Problem& p, const void* K, const void* V, const f
   using C = PrepCfg<TIn, D>;
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(prep_video_kernel<TIn, D>), C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  // [B * T frames][gh rows][gw columns][H * D channels], channels innermost.
+  // [B * T frames][gh rows][gw columns][H * D channels], channels innermost; a
+  // grid column's row holds Ht * D channels, of which this problem's H * D
+  // start at K and V.
   const uint64_t esz = sizeof(TIn);
   const uint64_t dims[4] = {(uint64_t)p.H * D, (uint64_t)p.gw, (uint64_t)p.gh, (uint64_t)p.B * p.T};
-  const uint64_t strides[3] = {dims[0] * esz, dims[0] * dims[1] * esz, dims[0] * dims[1] * dims[2] * esz};
+  const uint64_t row = (uint64_t)p.Ht * D * esz;
+  const uint64_t strides[3] = {row, row * dims[1], row * dims[1] * dims[2]};
   const uint32_t box[4] = {(uint32_t)D, (uint32_t)kTileCols, 5u, 1u};
   const CUtensorMapDataType dt = sizeof(TIn) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   CUtensorMap mK, mV;

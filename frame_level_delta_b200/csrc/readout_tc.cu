@@ -57,6 +57,7 @@ struct RoCfg {
 
 struct RoArgs {
   int B, H, T, U, c, J;
+  int Ht;  // heads per token row of Q, gate and O (O points at this problem's first head)
   unsigned flags;
   float l2_eps, rms_eps;
   const float* Sf;
@@ -280,16 +281,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int hf = (warp - 2) / 4;
     const int r = q * 32 + lane;      // tile row == TMEM lane this warp may read
     // Anchor frames 0 and T-1 read no linear memory: while the first tile's
-    // MMAs are in flight these threads zero this CTA's share of their rows
-    // (one contiguous slab of U * H * D values per batch and anchor).
+    // MMAs are in flight these threads zero this CTA's share of their rows (per
+    // batch and anchor, U token rows of this problem's H * D values, at a row
+    // stride of Ht * D; one contiguous slab when Ht == H).
     {
-      const long long per16 = (long long)a.U * a.H * D * 2 / 16;  // uint4 words per slab
+      const long long rw = (long long)a.H * D * 2 / 16;  // uint4 words per token row
+      const long long per16 = (long long)a.U * rw;       // uint4 words per slab
       const long long G = gridDim.x;
       const long long lo = per16 * blockIdx.x / G, hi = per16 * (blockIdx.x + 1) / G;
       for (int slab = 0; slab < 2 * a.B; ++slab) {
         const long long b = slab >> 1, f = (slab & 1) ? a.T - 1 : 0;
-        uint4* base = reinterpret_cast<uint4*>(a.O + (b * a.T + f) * (long long)a.U * a.H * D);
-        for (long long w = lo + et; w < hi; w += kEpiThreads) base[w] = make_uint4(0, 0, 0, 0);
+        uint4* base = reinterpret_cast<uint4*>(a.O + (b * a.T + f) * (long long)a.U * a.Ht * D);
+        const long long row16 = (long long)a.Ht * D * 2 / 16;
+        for (long long w = lo + et; w < hi; w += kEpiThreads) base[(w / rw) * row16 + w % rw] = make_uint4(0, 0, 0, 0);
       }
     }
     int g_prev = -1;
@@ -474,7 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(orow + box * (kTileM * 128) + pc * 16) = outs[c];
         }
       } else if (r < ti.nvalid) {
-        uint4* dst = reinterpret_cast<uint4*>(a.O + ((ti.tok0 + r) * a.H + h) * (long long)D) + col0 / 8;
+        uint4* dst = reinterpret_cast<uint4*>(a.O + ((ti.tok0 + r) * a.Ht + h) * (long long)D) + col0 / 8;
 #pragma unroll
         for (int c = 0; c < kHalf / 8; ++c) dst[c] = outs[c];
       }
@@ -512,7 +516,7 @@ template <int D, bool GATE>
 cudaError_t launch_dg(const Problem& p, const void* gate, void* O, cudaStream_t s) {
   using C = RoCfg<D, GATE>;
   RoArgs a{};
-  a.B = p.B; a.H = p.H; a.T = p.T; a.U = p.U; a.c = p.c; a.J = p.J;
+  a.B = p.B; a.H = p.H; a.T = p.T; a.U = p.U; a.c = p.c; a.J = p.J; a.Ht = p.Ht;
   a.flags = p.flags; a.l2_eps = p.l2_eps; a.rms_eps = p.rms_eps;
   a.Sf = p.Sf; a.Sr = p.Sr; a.O = static_cast<__nv_bfloat16*>(O);
   a.status = p.status; a.wait_ns = p.spin_limit;
@@ -537,10 +541,11 @@ cudaError_t launch_dg(const Problem& p, const void* gate, void* O, cudaStream_t 
   a.tiles_per_seg = (int)((tiles_per_head + a.nseg - 1) / a.nseg);
   const long long ncta = (long long)a.BH * a.nseg;
 
-  // [B*T*U tokens, H, D] views of Q, gate and O: dims (d, h, token)
+  // [B*T*U tokens, H, D] views of Q, gate and O from this problem's first head
+  // (rows of Ht * D values): dims (d, h, token)
   const uint64_t D64 = D, H = p.H, NT = (uint64_t)p.B * p.T * p.U;
   uint64_t dims[3] = {D64, H, NT};
-  uint64_t strides[2] = {D64 * 2, H * D64 * 2};
+  uint64_t strides[2] = {D64 * 2, (uint64_t)p.Ht * D64 * 2};
   uint32_t box[3] = {64, 1, (uint32_t)kTileM};
   CUtensorMap mQ, mG, mO;
   if ((e = make_tmap_bf16(&mQ, p.Q, 3, dims, strides, box)) != cudaSuccess) return e;

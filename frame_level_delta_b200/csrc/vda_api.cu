@@ -8,6 +8,7 @@
 #include <mutex>
 #include <set>
 #include <string>
+#include <type_traits>
 #include <utility>
 #include <vector>
 
@@ -102,7 +103,10 @@ vda_status check_config(const vda_config* c, std::string* why) {
     if (why) *why = "the chunked scan needs B * H <= 65535";
     return VDA_ERR_UNSUPPORTED;
   }
-  const long long tokens = (long long)c->B * c->T * c->U * c->H * d;
+  if (c->H_total < 0 || c->h0 < 0) return bad("H_total and h0 must be >= 0");
+  if (c->H_total == 0 && c->h0 != 0) return bad("h0 must be 0 when H_total is 0 (all heads)");
+  if (c->H_total > 0 && (long long)c->h0 + c->H > c->H_total) return bad("h0 + H must be <= H_total");
+  const long long tokens = (long long)c->B * c->T * c->U * (c->H_total > 0 ? c->H_total : c->H) * d;
   if (tokens >= (1LL << 40)) return bad("tensor too large");
   return VDA_OK;
 }
@@ -202,6 +206,18 @@ vda_status run_kernel(vda_ctx* ctx, int id, cudaStream_t s, F&& launch) {
 }
 
 bool use_simt_only(const vda_config& c) { return (c.flags & VDA_FORCE_SIMT) != 0; }
+
+int heads_total(const vda_config& c) { return c.H_total > 0 ? c.H_total : c.H; }
+
+// A token-tensor pointer advanced to head h0 of its rows.
+template <typename P>
+P head_slice(const vda_config& c, P ptr) {
+  if (ptr == nullptr) return ptr;
+  const size_t esz = c.dtype == VDA_BF16 ? 2 : 4;
+  using Byte = typename std::conditional<std::is_const<typename std::remove_pointer<P>::type>::value, const char,
+                                         char>::type;
+  return reinterpret_cast<P>(reinterpret_cast<Byte*>(ptr) + (size_t)c.h0 * c.d_k * esz);
+}
 
 }  // namespace
 
@@ -319,6 +335,14 @@ vda_status vda_prepare(vda_ctx* ctx, const void* Q, const void* K, const void* V
   Problem& p = ctx->p;
   p = Problem{};
   p.B = c.B; p.H = c.H; p.T = c.T; p.U = c.U; p.L = c.L; p.D = c.d_k; p.c = c.chunk; p.J = J_of(c);
+  p.Ht = heads_total(c);
+  // Token tensors: advance to this context's first head (h0 * d elements; a
+  // multiple of 32 bytes, so 16-byte alignment is kept).
+  Q = head_slice(c, Q);
+  K = head_slice(c, K);
+  V = head_slice(c, V);
+  K_txt = head_slice(c, K_txt);
+  V_txt = head_slice(c, V_txt);
   p.gh = c.grid_h; p.gw = c.grid_w;
   p.bf16 = c.dtype == VDA_BF16;
   p.flags = c.flags;
@@ -336,7 +360,7 @@ vda_status vda_prepare(vda_ctx* ctx, const void* Q, const void* K, const void* V
   p.CMi = ws + L.off[VDA_REGION_CHUNK_M];
   p.CC = reinterpret_cast<float*>(ws + L.off[VDA_REGION_CHUNK_C]);
   p.spin_limit = 2000000000ull;  // 2 s of wall time per device-side wait
-  const long long D = p.D, H = p.H, T = p.T, U = p.U, Lt = p.L;
+  const long long D = p.D, H = p.H, T = p.T, U = p.U, Lt = p.L, Ht = p.Ht;
   if (prep) {
     p.Kp = ws + L.off[VDA_REGION_K_PREP];
     p.Vp = ws + L.off[VDA_REGION_V_PREP];
@@ -347,10 +371,10 @@ vda_status vda_prepare(vda_ctx* ctx, const void* Q, const void* K, const void* V
     p.Kt = TokView{p.Ktp, H * Lt * D, Lt * D, 0, D};
     p.Vt = TokView{p.Vtp, H * Lt * D, Lt * D, 0, D};
   } else {
-    p.Kv = TokView{K, T * U * H * D, D, U * H * D, H * D};
-    p.Vv = TokView{V, T * U * H * D, D, U * H * D, H * D};
-    p.Kt = TokView{K_txt, Lt * H * D, D, 0, H * D};
-    p.Vt = TokView{V_txt, Lt * H * D, D, 0, H * D};
+    p.Kv = TokView{K, T * U * Ht * D, D, U * Ht * D, Ht * D};
+    p.Vv = TokView{V, T * U * Ht * D, D, U * Ht * D, Ht * D};
+    p.Kt = TokView{K_txt, Lt * Ht * D, D, 0, Ht * D};
+    p.Vt = TokView{V_txt, Lt * Ht * D, D, 0, Ht * D};
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // Clears the status word and the slot-ready words the solve raises.
@@ -417,6 +441,8 @@ vda_status vda_readout(vda_ctx* ctx, const void* gate, void* O, void* stream) {
   if ((ctx->cfg.flags & VDA_READOUT_NORM_GATE) && !gate)
     return fail(ctx, VDA_ERR_INVALID_ARG, "gate is required with VDA_READOUT_NORM_GATE");
   if (!aligned16(O) || (gate && !aligned16(gate))) return fail(ctx, VDA_ERR_ALIGNMENT, "O and gate must be 16-byte aligned");
+  O = head_slice(ctx->cfg, O);
+  gate = head_slice(ctx->cfg, gate);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const Problem& p = ctx->p;
   // The tensor-core readout zeroes the anchor frames itself.

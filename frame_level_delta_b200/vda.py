@@ -8,7 +8,7 @@ from __future__ import annotations
 
 import ctypes
 import os
-from typing import Dict, Optional
+from typing import Dict, Optional, Tuple
 
 import torch
 
@@ -49,7 +49,7 @@ class vda_config(ctypes.Structure):
                 ("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int), ("L", ctypes.c_int),
                 ("d_k", ctypes.c_int), ("d_v", ctypes.c_int), ("chunk", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("flags", ctypes.c_uint), ("l2_eps", ctypes.c_float),
-                ("rms_eps", ctypes.c_float)]
+                ("rms_eps", ctypes.c_float), ("H_total", ctypes.c_int), ("h0", ctypes.c_int)]
 
 
 _lib = None
@@ -97,7 +97,10 @@ def lib() -> ctypes.CDLL:
 
 
 def make_config(cfg: VDAConfig, force_simt: bool = False, l2_eps: float = 1e-6,
-                rms_eps: float = 1e-6, cholesky: bool = False, chunked: bool = False) -> vda_config:
+                rms_eps: float = 1e-6, cholesky: bool = False, chunked: bool = False,
+                heads: Optional[Tuple[int, int]] = None) -> vda_config:
+    """The C config of a workload. ``heads = (h0, n)`` makes a context for heads
+    h0 .. h0+n-1 of the workload's cfg.H heads (token tensors keep all cfg.H)."""
     flags = (VDA_PREP_CONV if cfg.prep_conv else 0) | (VDA_READOUT_NORM_GATE if cfg.norm_gate else 0)
     if force_simt:
         flags |= VDA_FORCE_SIMT
@@ -105,10 +108,11 @@ def make_config(cfg: VDAConfig, force_simt: bool = False, l2_eps: float = 1e-6,
         flags |= VDA_SOLVE_CHOLESKY
     if chunked:
         flags |= VDA_SCAN_CHUNKED
-    return vda_config(B=cfg.B, H=cfg.H, T=cfg.T, U=cfg.U, grid_h=cfg.grid_h, grid_w=cfg.grid_w, L=cfg.L,
+    h0, n = heads if heads is not None else (0, cfg.H)
+    return vda_config(B=cfg.B, H=n, T=cfg.T, U=cfg.U, grid_h=cfg.grid_h, grid_w=cfg.grid_w, L=cfg.L,
                       d_k=cfg.d, d_v=cfg.d, chunk=cfg.chunk,
                       dtype=VDA_F32 if cfg.dtype == "f32" else VDA_BF16, flags=flags,
-                      l2_eps=l2_eps, rms_eps=rms_eps)
+                      l2_eps=l2_eps, rms_eps=rms_eps, H_total=cfg.H if heads is not None else 0, h0=h0)
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -145,12 +149,19 @@ def describe(c: vda_config) -> str:
 
 
 class VDA:
-    """One context of the library: prepare -> scan_bidir -> readout on a stream."""
+    """One context of the library: prepare -> scan_bidir -> readout on a stream.
+
+    With ``heads = (h0, n)`` the context serves heads h0 .. h0+n-1 of the
+    workload: the token tensors (Q, K, V, K_txt, V_txt, gate, O) keep all cfg.H
+    heads and are read and written in place, and the per-head parameters
+    (alpha, beta, beta_txt, conv_w) are passed for all cfg.H heads and sliced to
+    the context's heads here."""
 
     def __init__(self, cfg: VDAConfig, force_simt: bool = False, device="cuda", cholesky: bool = False,
-                 chunked: bool = False):
+                 chunked: bool = False, heads: Optional[Tuple[int, int]] = None):
         self.cfg = cfg
-        self.c = make_config(cfg, force_simt=force_simt, cholesky=cholesky, chunked=chunked)
+        self.heads = heads
+        self.c = make_config(cfg, force_simt=force_simt, cholesky=cholesky, chunked=chunked, heads=heads)
         self._ctx = ctypes.c_void_p()
         st = lib().vda_create(ctypes.byref(self.c), ctypes.byref(self._ctx))
         if st != VDA_OK:
@@ -225,8 +236,27 @@ class VDA:
         with self._on_device():
             self._prepare(inp, stream)
 
+    def _head_params(self, inp: Dict[str, torch.Tensor]) -> Dict[str, torch.Tensor]:
+        """The per-head parameters of this context's heads (views for B = 1)."""
+        if self.heads is None:
+            return inp
+        h0, n = self.heads
+        cfg = self.cfg
+        out = dict(inp)
+        for k in ("alpha", "beta", "beta_txt"):
+            out[k] = inp[k][:, h0:h0 + n].contiguous()
+        if cfg.prep_conv:
+            hd, d = cfg.H * cfg.d, cfg.d
+            w = inp["conv_w"]
+            parts = []
+            for off, taps in ((0, 25), (hd * 25, 5), (hd * 30, 25), (hd * 55, 5)):
+                parts.append(w[off + h0 * d * taps: off + (h0 + n) * d * taps])
+            out["conv_w"] = torch.cat(parts).contiguous()
+        return out
+
     def _prepare(self, inp: Dict[str, torch.Tensor], stream=None):
         ws = self.ensure_workspace()
+        inp = self._head_params(inp)
         self._keep = inp  # inputs must outlive the readout
         st = lib().vda_prepare(self._ctx, _ptr(inp["Q"]), _ptr(inp["K"]), _ptr(inp["V"]), _ptr(inp["K_txt"]),
                                _ptr(inp["V_txt"]), _ptr(inp["alpha"]), _ptr(inp["beta"]), _ptr(inp["beta_txt"]),
@@ -268,8 +298,8 @@ class VDA:
         """A view of one workspace region (float32 unless it is a prepared token copy)."""
         off, nb = workspace_region(self.c, name)
         raw = self.ensure_workspace()[off:off + nb]
-        cfg = self.cfg
-        D, BH = cfg.d, cfg.B * cfg.H
+        cfg = self.cfg.with_(H=self.c.H)  # the context's heads (all of them unless sliced)
+        D = cfg.d
         if name in ("A", "B", "M", "C"):
             return _from_quads(raw, (cfg.B, cfg.H, cfg.T - 1), D)
         if name in ("S_fwd", "S_rev"):

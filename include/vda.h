@@ -102,6 +102,15 @@ typedef struct vda_config {
   unsigned flags;
   float l2_eps;  /* default 1e-6 */
   float rms_eps; /* default 1e-6 */
+  /* Head slice, for running a subset of the heads of a larger token tensor (one
+   * rank's share when the heads are split across GPUs). The token tensors Q, K,
+   * V, K_txt, V_txt, gate and O hold H_total heads per token row ([B, tokens,
+   * H_total, d]); this context reads and writes heads h0 .. h0 + H - 1 of them
+   * and never touches the others. 0 for H_total means H_total = H (then h0 must
+   * be 0). The per-head parameters alpha, beta, beta_txt and conv_w are given
+   * for this context's H heads only. */
+  int H_total;
+  int h0;
 } vda_config;
 
 typedef struct vda_ctx vda_ctx; /* opaque host object; owns no device memory */

@@ -224,3 +224,25 @@ def test_binding_checks_tensors_before_calling_the_library():
         dev.prepare(inp)
     with pytest.raises(ValueError, match="is on cpu"):
         dev.run(inp, O)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(H_total=8, h0=0, H=8), 0),
+    (dict(H_total=8, h0=5, H=3), 0),
+    (dict(H_total=8, h0=6, H=3), 1),   # slice runs past the last head
+    (dict(H_total=0, h0=1, H=8), 1),   # h0 without H_total
+    (dict(H_total=-1, h0=0, H=8), 1),
+    (dict(H_total=8, h0=-1, H=2), 1),
+])
+def test_head_slice_fields_are_checked(kw, want):
+    c = _cfg(**kw)
+    st, ctx = _create(c)
+    assert st == want
+    if ctx.value:
+        assert V.lib().vda_destroy(ctx) == 0
+
+
+def test_head_slice_workspace_is_sized_by_the_slice():
+    whole = V.workspace_size(V.make_config(CONFIGS["small"].with_(H=3)))
+    part = V.workspace_size(V.make_config(CONFIGS["small"], heads=(5, 3)))
+    assert part == whole

@@ -81,6 +81,48 @@ def _rank_leaves(rank, world, port, out_dir):
     os._exit(0)
 
 
+def _rank_heads(rank, world, port, out_dir):
+    """Head-sharded ranks over one shared batch: each rank computes its heads'
+    output (the float64 oracle stands in for the library on CPU), the slices are
+    all-gathered, and rank 0 compares the assembly with the single-rank output."""
+    sys.path.insert(0, ROOT)
+    _set_env(rank, world, port)
+    import numpy as np
+
+    import bench
+    from frame_level_delta_b200.inputs import CONFIGS, make_inputs
+    from frame_level_delta_b200.shard import head_partition
+    from oracle.vda_oracle import vda_reference
+
+    r, w, _ = bench.rank_env()
+    dist = bench.init_ranks(w, torch.device("cpu"), timeout_s=60)
+    cfg = CONFIGS["small"].with_(H=5, T=8, grid_h=4, grid_w=4, L=6, d=16)
+    inp = make_inputs(cfg)  # the same batch on every rank
+    parts = head_partition(cfg.H, w, (5, 3))
+    h0, n = parts[r]
+    mine = vda_reference(inp, cfg, heads=[(0, h) for h in range(h0, h0 + n)], keep=False)["O"][:, :, h0:h0 + n]
+    slices = [None] * w
+    dist.all_gather_object(slices, (h0, n, mine))
+    bench.barrier(dist)
+    dist.destroy_process_group()
+    if r == 0:
+        whole = vda_reference(inp, cfg, keep=False)["O"]
+        got = np.zeros_like(whole)
+        for (a, k, o) in slices:
+            got[:, :, a:a + k] = o
+        with open(os.path.join(out_dir, "heads.json"), "w") as f:
+            json.dump({"parts": [list(p) for p in parts], "equal": bool(np.array_equal(got, whole))}, f)
+
+
+def test_two_gloo_ranks_head_slices_reassemble_the_output(tmp_path):
+    world = 2
+    mp.start_processes(_rank_heads, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    d = json.loads((tmp_path / "heads.json").read_text())
+    assert d["parts"] == [[0, 3], [3, 2]]
+    assert d["equal"]
+
+
 def test_two_gloo_ranks_barrier_max_and_shards(tmp_path):
     world = 2
     mp.start_processes(_rank_timing, args=(world, _free_port(), str(tmp_path)), nprocs=world,
@@ -123,3 +165,23 @@ def test_reference_arm_prints_once_under_torchrun():
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["steps"] == 2
     assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
     assert line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_bench_starts_its_own_ranks_without_torchrun():
+    """`bench.py --gpus 2` launched as one plain process re-launches itself as two
+    ranks under torch.distributed.run (the reference arm runs on CPU here)."""
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--gpus", "2", "--config", "tiny", "--steps", "2",
+           "--warmup", "3"]
+    p = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300, env=env)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [json.loads(x) for x in p.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1 and lines[0]["n_gpus"] == 2
+
+
+def test_bench_rejects_a_rank_count_that_differs_from_gpus():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="2", LOCAL_RANK="0")
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--gpus", "3", "--config", "tiny", "--steps", "1",
+           "--warmup", "3"]
+    p = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=120, env=env)
+    assert p.returncode != 0 and "WORLD_SIZE" in p.stderr
