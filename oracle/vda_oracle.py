@@ -231,7 +231,9 @@ def vda_reference(inp: Dict, cfg, heads: Optional[Iterable[Tuple[int, int]]] = N
 
     Returns ``O`` ([B, T*U, H, d] float64, zero for heads not computed) and, when
     ``keep``, per-(b, h) intermediates: A, B (slot 0 = text, slot t = frame t),
-    M, C, S_T, all forward and reverse states, and the per-chunk readout states.
+    M, C, S_T, all forward and reverse states, the per-chunk readout states, and
+    the Euclidean norm of every token's readout before RMSNorm and the gate
+    (o_pre_norm, [T*U], zero on anchor frames).
     """
     B_, H, d, T, c = cfg.B, cfg.H, cfg.d, cfg.T, cfg.chunk
     gh, gw = cfg.grid_h, cfg.grid_w
@@ -285,10 +287,12 @@ def vda_reference(inp: Dict, cfg, heads: Optional[Iterable[Tuple[int, int]]] = N
             S_fwd.append(F[max(0, c * (j - 1) - 1)])
             S_rev.append(R[min(T - 1, c * (j + 2))])
 
+        o_pre_norm = np.zeros(T * U)
         for t in range(1, T - 1):
             j = chunk_of(t, c)
             S = S_fwd[j] + S_rev[j]
             o = Qh[t] @ S.T  # row u is S q_u
+            o_pre_norm[t * U:(t + 1) * U] = np.linalg.norm(o, axis=1)
             if cfg.norm_gate:
                 g = _f64(inp["gate"][b, t * U:(t + 1) * U, h, :])
                 o = rms_norm_gate(o, g, eps)
@@ -296,5 +300,5 @@ def vda_reference(inp: Dict, cfg, heads: Optional[Iterable[Tuple[int, int]]] = N
 
         if keep:
             inter[(b, h)] = dict(A=A, B=Bm, M=M, C=C, S_T=S_T, F=F, R=R,
-                                 S_fwd=S_fwd, S_rev=S_rev)
+                                 S_fwd=S_fwd, S_rev=S_rev, o_pre_norm=o_pre_norm)
     return {"O": O, "inter": inter, "heads": heads}

@@ -83,8 +83,13 @@ def staged_errors(cfg, regions, ref):
 # Frobenius bound of the whole output. Per token: |o_gpu - o_ref| <= tol *
 # max(|o_ref|, floor) with floor = 5% of the RMS token norm of that (b, h), so
 # that the rare token whose reference output is near zero is judged against the
-# head's scale rather than its own.
+# head's scale rather than its own. With RMSNorm and the gate, each token is
+# divided by its own pre-norm magnitude, which scales that token's share of the
+# state's error by the same factor: a token whose pre-norm readout |o_pre| lies
+# below GATED_FLOOR times the head's RMS of |o_pre| gets its allowance raised by
+# that ratio.
 TOKEN_FLOOR = 0.05
+GATED_FLOOR = 0.5
 
 
 def readout_tiles(cfg, j: int):
@@ -98,10 +103,11 @@ def readout_tiles(cfg, j: int):
     return [(a, min(a + 128, end)) for a in range(first, end, 128)]
 
 
-def local_output_errors(cfg, O_g, O_ref, pairs):
+def local_output_errors(cfg, O_g, O_ref, pairs, pre_norms=None):
     """Worst per-(b, h, frame) relative error, worst per-token error ratio (error
     over the token's allowance), and the worst ratio among the tokens of each
-    chunk's last (ragged) readout tile. Returns a dict."""
+    chunk's last (ragged) readout tile. ``pre_norms`` maps (b, h) to the oracle's
+    per-token norms before RMSNorm (gated readouts). Returns a dict."""
     U, T = cfg.U, cfg.T
     tol = TOL_O[cfg.dtype]
     worst_frame, worst_tok, worst_tail = 0.0, 0.0, 0.0
@@ -115,6 +121,10 @@ def local_output_errors(cfg, O_g, O_ref, pairs):
         rn = np.linalg.norm(r[body], axis=1)
         floor = TOKEN_FLOOR * float(np.sqrt(np.mean(rn * rn))) if rn.size else 0.0
         allow = tol * np.maximum(rn, max(floor, 1e-30))
+        if pre_norms is not None:
+            pn = np.asarray(pre_norms[(b, h)], dtype=np.float64)[body]
+            pfloor = GATED_FLOOR * float(np.sqrt(np.mean(pn * pn)))
+            allow = allow * np.maximum(1.0, pfloor / np.maximum(pn, 1e-30))
         ratio = en / allow
         worst_tok = max(worst_tok, float(ratio.max()) if ratio.size else 0.0)
         for j in range(cfg.J):
@@ -147,7 +157,8 @@ def check_config(cfg, heads=None, force_simt=False, inp=None, stage_tol=None, ch
     tol_s = stage_tol if stage_tol is not None else (
         TOL_STAGE_PER_ROUNDING * roundings if roundings else TOL_STAGE_SIMT)
     assert err_o <= TOL_O[cfg.dtype], (err_o, stages)
-    local = local_output_errors(cfg, O_g, O_ref, ref["heads"])
+    pre = ({k: v["o_pre_norm"] for k, v in ref["inter"].items()} if cfg.norm_gate else None)
+    local = local_output_errors(cfg, O_g, O_ref, ref["heads"], pre)
     assert local["frame"] <= TOL_O[cfg.dtype], local
     assert local["token_ratio"] <= 1.0, local
     for k, e in stages.items():

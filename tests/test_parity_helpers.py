@@ -54,3 +54,16 @@ def test_local_bounds_catch_one_wrong_frame():
     got[0, t * cfg.U:(t + 1) * cfg.U] *= 1.05
     assert rel_fro(got, ref) < TOL_O["bf16"]
     assert local_output_errors(cfg, got, ref, [(0, 0)])["frame"] > TOL_O["bf16"]
+
+
+def test_gated_allowance_grows_for_tokens_with_a_small_pre_norm_readout():
+    cfg = CONFIGS["small"].with_(H=1, T=6, grid_h=4, grid_w=4, norm_gate=True)
+    rng = np.random.default_rng(2)
+    ref = rng.standard_normal((1, cfg.T * cfg.U, 1, cfg.d))
+    got = ref.copy()
+    u = 2 * cfg.U + 3
+    got[0, u, 0] *= 1.05  # 5% off on one token
+    pre = np.ones(cfg.T * cfg.U)
+    assert local_output_errors(cfg, got, ref, [(0, 0)], {(0, 0): pre})["token_ratio"] > 1.0
+    pre[u] = 0.1  # its pre-norm readout is a tenth of the head's: RMSNorm scaled its error up 10x
+    assert local_output_errors(cfg, got, ref, [(0, 0)], {(0, 0): pre})["token_ratio"] <= 1.0
