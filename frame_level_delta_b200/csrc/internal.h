@@ -126,6 +126,7 @@ enum KernelId {
   K_SCAN_TC,
   K_COMPOSE_TC,
   K_SOLVE_CHOL_TC,
+  K_WINDOW_ATTN_TC,
   K_NUM_KERNELS
 };
 const char* kernel_name(int id);
@@ -157,5 +158,11 @@ bool scan_tc_supported(const Problem& p);
 cudaError_t launch_scan_tc(const Problem& p, cudaStream_t s, bool chunked);
 cudaError_t launch_compose_tc(const Problem& p, cudaStream_t s);
 cudaError_t launch_readout_tc(const Problem& p, const void* gate, void* O, cudaStream_t s);
+
+// Softmax branch: window + anchor attention with the sigmoid gate (bf16, D in {64, 128}).
+// Q, K, V, gate and O are advanced to the problem's first head (rows of Ht * D values).
+bool window_attn_tc_supported(const Problem& p);
+cudaError_t launch_window_attn_tc(const Problem& p, const void* Q, const void* K, const void* V, const void* gate,
+                                  void* O, cudaStream_t s);
 
 }  // namespace vda

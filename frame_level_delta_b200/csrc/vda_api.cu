@@ -20,7 +20,7 @@ const char* kernel_name(int id) {
   static const char* names[K_NUM_KERNELS] = {
       "prep_video", "prep_text", "gram_simt", "gram_tc", "solve_simt",
       "scan_simt", "readout_simt", "readout_tc", "zero_anchors", "solve_tc", "scan_tc", "compose_tc",
-      "solve_chol_tc"};
+      "solve_chol_tc", "window_attn_tc"};
   return (id >= 0 && id < K_NUM_KERNELS) ? names[id] : "?";
 }
 
@@ -56,6 +56,7 @@ struct vda_ctx {
   std::vector<EventPair> pool;
   int prof_launches[K_NUM_KERNELS] = {};
   double prof_ms[K_NUM_KERNELS] = {};
+  uint32_t* attn_status = nullptr;  // status word of the last vda_window_attention call
 };
 
 namespace {
@@ -455,18 +456,51 @@ vda_status vda_readout(vda_ctx* ctx, const void* gate, void* O, void* stream) {
 
 vda_status vda_poll_device_status(vda_ctx* ctx, void* stream) {
   if (!ctx) return VDA_ERR_INVALID_ARG;
-  if (!ctx->p.status) return fail(ctx, VDA_ERR_STATE, "no workspace bound yet");
+  if (!ctx->p.status && !ctx->attn_status) return fail(ctx, VDA_ERR_STATE, "no workspace bound yet");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint32_t word = 0;
-  cudaError_t e = cudaMemcpyAsync(&word, ctx->p.status, sizeof(word), cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) return cuda_fail(ctx, e, "status read");
-  if (word != 0) {
-    e = cudaMemsetAsync(ctx->p.status, 0, sizeof(word), s);
-    if (e != cudaSuccess) return cuda_fail(ctx, e, "status clear");
-    return fail(ctx, VDA_ERR_TIMEOUT, "a bounded device-side wait gave up");
+  bool timeout = false;
+  for (uint32_t* w : {ctx->p.status, ctx->attn_status}) {
+    if (!w) continue;
+    uint32_t word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, w, sizeof(word), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "status read");
+    if (word != 0) {
+      e = cudaMemsetAsync(w, 0, sizeof(word), s);
+      if (e != cudaSuccess) return cuda_fail(ctx, e, "status clear");
+      timeout = true;
+    }
   }
+  if (timeout) return fail(ctx, VDA_ERR_TIMEOUT, "a bounded device-side wait gave up");
   return VDA_OK;
+}
+
+vda_status vda_window_attention(vda_ctx* ctx, const void* Q, const void* K, const void* V, const void* gate,
+                                void* O, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!ctx) return VDA_ERR_INVALID_ARG;
+  const vda_config& c = ctx->cfg;
+  if (!Q || !K || !V || !O || !workspace) return fail(ctx, VDA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || (gate && !aligned16(gate)))
+    return fail(ctx, VDA_ERR_ALIGNMENT, "Q, K, V, gate and O must be 16-byte aligned");
+  if (((uintptr_t)workspace & 255) != 0) return fail(ctx, VDA_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  if (workspace_bytes < 256) return fail(ctx, VDA_ERR_WORKSPACE_TOO_SMALL, "the attention needs 256 bytes of workspace");
+  Problem p{};
+  p.B = c.B; p.H = c.H; p.T = c.T; p.U = c.U; p.L = c.L; p.D = c.d_k; p.c = c.chunk; p.J = J_of(c);
+  p.gh = c.grid_h; p.gw = c.grid_w; p.Ht = heads_total(c);
+  p.bf16 = c.dtype == VDA_BF16;
+  p.flags = c.flags;
+  p.status = static_cast<uint32_t*>(workspace);
+  p.spin_limit = 2000000000ull;
+  if (use_simt_only(c) || !window_attn_tc_supported(p))
+    return fail(ctx, VDA_ERR_UNSUPPORTED, "the window attention needs bf16 storage and d in {64, 128}");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(p.status, 0, sizeof(uint32_t), s);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "status reset");
+  ctx->attn_status = p.status;
+  return run_kernel(ctx, K_WINDOW_ATTN_TC, s, [&] {
+    return launch_window_attn_tc(p, head_slice(c, Q), head_slice(c, K), head_slice(c, V), head_slice(c, gate),
+                                 head_slice(c, O), s);
+  });
 }
 
 vda_status vda_profile_enable(vda_ctx* ctx, int enable) {

@@ -149,3 +149,31 @@ def split_conv_w(conv_w: torch.Tensor, H: int, d: int):
     parts = torch.split(conv_w, sizes)
     return (parts[0].reshape(H, d, 5, 5), parts[1].reshape(H, d, 5),
             parts[2].reshape(H, d, 5, 5), parts[3].reshape(H, d, 5))
+
+
+def make_attention_inputs(cfg: VDAConfig, logit_std: float = 1.0, seed: Optional[int] = None,
+                          gate: bool = True) -> Dict[str, torch.Tensor]:
+    """Seeded inputs of the softmax branch in the layouts the C ABI takes: Q, K,
+    V [B, T*U, H, d] and the branch's gate logits g [B, T*U, H, d] (storage dtype).
+
+    K rows are unit vectors and Q rows have N(0, logit_std^2 d) entries, so the
+    logits q.k / sqrt(d) are roughly N(0, logit_std^2): 1 gives the nearly flat
+    weights of normalised features, larger values sharply peaked ones. V ~ N(0, 1),
+    gate logits ~ N(0, 1). Draw order: Q, K, V, gate.
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed((cfg.seed if seed is None else seed) + 1000)
+    B, H, d, T, U = cfg.B, cfg.H, cfg.d, cfg.T, cfg.U
+    sd = storage_dtype(cfg)
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=g, dtype=torch.float32)
+
+    Q = randn(B, T * U, H, d) * (logit_std * d ** 0.5)
+    K = _unit_rows(randn(B, T * U, H, d))
+    V = randn(B, T * U, H, d)
+    out = {"Q": Q.to(sd).contiguous(), "K": K.to(sd).contiguous(),
+           "V": V.to(sd).contiguous()}
+    if gate:
+        out["gate"] = randn(B, T * U, H, d).to(sd).contiguous()
+    return out

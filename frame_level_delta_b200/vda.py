@@ -31,7 +31,7 @@ REGIONS = {"status": 0, "A": 1, "B": 2, "M": 3, "C": 4, "S_fwd": 5, "S_rev": 6,
 
 # Exported symbols, in the order include/vda.h declares them.
 EXPORTS = ["vda_create", "vda_destroy", "vda_workspace_size", "vda_prepare", "vda_scan_bidir",
-           "vda_readout", "vda_poll_device_status", "vda_workspace_region", "vda_status_string",
+           "vda_readout", "vda_poll_device_status", "vda_window_attention", "vda_workspace_region", "vda_status_string",
            "vda_last_error", "vda_profile_enable", "vda_num_kernels", "vda_profile_read",
            "vda_launch_count", "vda_describe", "vda_selftest_bounded_wait",
            "vda_selftest_recip", "vda_static_workspace_capacity", "vda_run_static_workspace",
@@ -72,6 +72,7 @@ def lib() -> ctypes.CDLL:
         L.vda_scan_bidir.argtypes = [vp, vp]
         L.vda_readout.argtypes = [vp, vp, vp, vp]
         L.vda_poll_device_status.argtypes = [vp, vp]
+        L.vda_window_attention.argtypes = [vp] * 7 + [sz, vp]
         L.vda_workspace_region.argtypes = [cfgp, i, ctypes.POINTER(sz), ctypes.POINTER(sz)]
         L.vda_status_string.argtypes = [st]
         L.vda_status_string.restype = ctypes.c_char_p
@@ -169,6 +170,7 @@ class VDA:
         self.ws_bytes = workspace_size(self.c)
         self.device = torch.device(device)
         self.workspace: Optional[torch.Tensor] = None
+        self._attn_ws: Optional[torch.Tensor] = None
         self._keep = None
 
     def __del__(self):
@@ -244,7 +246,10 @@ class VDA:
         cfg = self.cfg
         out = dict(inp)
         for k in ("alpha", "beta", "beta_txt"):
-            out[k] = inp[k][:, h0:h0 + n].contiguous()
+            t = inp[k][:, h0:h0 + n]
+            if not t.is_contiguous() or t.data_ptr() % 16:
+                t = t.clone(memory_format=torch.contiguous_format)  # the C ABI takes 16-byte aligned rows
+            out[k] = t
         if cfg.prep_conv:
             hd, d = cfg.H * cfg.d, cfg.d
             w = inp["conv_w"]
@@ -288,6 +293,29 @@ class VDA:
             self._prepare(inp, stream)
             self._check(lib().vda_scan_bidir(self._ctx, _stream_handle(stream)), "vda_scan_bidir")
             self._check(lib().vda_readout(self._ctx, _ptr(gate), _ptr(O), _stream_handle(stream)), "vda_readout")
+        return O
+
+    def window_attention(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                         gate: Optional[torch.Tensor] = None, O: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+        """The softmax branch (window + anchor attention, optional sigmoid gate)
+        over the same token tensors as the linear branch."""
+        cfg = self.cfg
+        sd = torch.float32 if cfg.dtype == "f32" else torch.bfloat16
+        shape = (cfg.B, cfg.T * cfg.U, cfg.H, cfg.d)
+        for name, t in (("Q", Q), ("K", K), ("V", V)):
+            self._expect(name, t, shape, sd)
+        if gate is not None:
+            self._expect("gate", gate, shape, sd)
+        if O is None:
+            O = self.new_output()
+        self._expect("O", O, shape, sd)
+        if self._attn_ws is None:
+            self._attn_ws = torch.zeros(256, dtype=torch.uint8, device=self.device)
+        with self._on_device():
+            self._check(lib().vda_window_attention(self._ctx, _ptr(Q), _ptr(K), _ptr(V), _ptr(gate), _ptr(O),
+                                                   _ptr(self._attn_ws), 256, _stream_handle(stream)),
+                        "vda_window_attention")
         return O
 
     def poll_device_status(self, stream=None) -> int:

@@ -170,11 +170,35 @@ vda_status vda_scan_bidir(vda_ctx* ctx, void* stream);
 vda_status vda_readout(vda_ctx* ctx, const void* gate, void* O, void* stream);
 
 /*
- * Synchronise `stream`, read the device status word in the workspace, clear it
- * and return VDA_ERR_TIMEOUT if a bounded device-side wait gave up since the last
- * poll, VDA_OK otherwise (VDA_ERR_STATE before any vda_prepare).
+ * Synchronise `stream`, read the device status words of the last vda_prepare
+ * workspace and of the last vda_window_attention workspace, clear them and return
+ * VDA_ERR_TIMEOUT if a bounded device-side wait gave up since the last poll,
+ * VDA_OK otherwise (VDA_ERR_STATE before any vda_prepare or vda_window_attention).
  */
 vda_status vda_poll_device_status(vda_ctx* ctx, void* stream);
+
+/*
+ * The softmax half of the hybrid attention layer, on the same Q, K, V as the
+ * linear branch (Video DeltaNet summary, onedev.kr/papers/80, section "how it
+ * works": each query chunk attends densely to chunks j-1 .. j+1 and to the
+ * boundary anchors; section "how it differs": its own sigmoid output gate; VDN-H3
+ * post, section "hybrid attention structure": the four-way anchor links).
+ * For every token of frame t (chunk j = floor(t / c)), every head:
+ *   o = softmax(q K_vis^T / sqrt(d)) V_vis,  then  o <- o * sigmoid(g)  (gate given)
+ * where the visible keys are every token of frames max(0, c(j-1)) .. min(T-1,
+ * c(j+2)-1) and of frames 0 and T-1 when t is not an anchor, and every video
+ * token when t is 0 or T-1 (text tokens are not part of this branch).
+ *   Q, K, V, gate, O  [B, T*U, H_total, d] storage dtype (this context's heads
+ *                     h0 .. h0 + H - 1 are read and written); gate may be NULL.
+ *   workspace         >= 256 bytes of device memory, 256-byte aligned; its first
+ *                     word is this call's device status word (cleared here, read
+ *                     by vda_poll_device_status). Separate calls that may run at
+ *                     the same time need separate workspaces.
+ * Needs bf16 storage and d in {64, 128} (tensor-core kernel), else
+ * VDA_ERR_UNSUPPORTED. Independent of vda_prepare; only enqueues work.
+ */
+vda_status vda_window_attention(vda_ctx* ctx, const void* Q, const void* K, const void* V, const void* gate,
+                                void* O, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Regions of the workspace, for staged parity checks and debugging. Every

@@ -81,6 +81,24 @@ def window_softmax_head(Q: np.ndarray, K: np.ndarray, V: np.ndarray, T: int, U: 
     return O
 
 
+def window_softmax_rows(Q: np.ndarray, K: np.ndarray, V: np.ndarray, T: int, U: int, c: int,
+                        rows, scale: float = None) -> np.ndarray:
+    """The same attention as window_softmax_head for selected query tokens only
+    (token indices into the frame-major [T U] axis), for spot checks of large
+    clips. Returns [len(rows), d_v]."""
+    d_k = Q.shape[1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d_k)
+    out = np.zeros((len(rows), V.shape[1]))
+    for n, row in enumerate(rows):
+        t = int(row) // U
+        keys = np.concatenate([np.arange(f * U, (f + 1) * U) for f in visible_frames(t, c, T)])
+        logits = (K[keys] @ Q[row]) * scale
+        w = np.exp(logits - logits.max())
+        out[n] = (w / w.sum()) @ V[keys]
+    return out
+
+
 def softmax_gate(O: np.ndarray, g: np.ndarray) -> np.ndarray:
     """O~S = O^S * sigmoid(g^S), elementwise."""
     return O * (1.0 / (1.0 + np.exp(-g)))

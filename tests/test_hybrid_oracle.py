@@ -59,6 +59,18 @@ def test_window_softmax_matches_token_pair_mask(T, U, c, d, mod=ho):
     np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
 
 
+@pytest.mark.parametrize("T,U,c,d", [(9, 3, 2, 4), (13, 2, 3, 5), (20, 1, 5, 2)])
+def test_sampled_rows_match_the_token_pair_mask(T, U, c, d, mod=ho):
+    """The spot-check form (selected query tokens) against the dense masked
+    softmax over the token-pair mask, on every row and on a shuffled subset."""
+    Q, K, V = _rand(T * 7 + U, T, U, d)
+    want = _dense_masked(Q, K, V, _pair_mask(T, U, c), 1.0 / np.sqrt(d))
+    rows = np.random.default_rng(3).permutation(T * U)[: max(3, T * U // 3)]
+    np.testing.assert_allclose(mod.window_softmax_rows(Q, K, V, T, U, c, rows), want[rows], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(mod.window_softmax_rows(Q, K, V, T, U, c, range(T * U)), want, rtol=1e-12,
+                               atol=1e-12)
+
+
 def test_window_spanning_the_clip_is_dense_attention(mod=ho):
     T, U, c, d = 6, 3, 3, 4  # two chunks: every window covers both
     Q, K, V = _rand(7, T, U, d)
@@ -140,6 +152,7 @@ MUTATIONS = {
     "anchor_rows_windowed": ("    if t in anchor_frames(T):\n        return list(range(T))\n", ""),
     "scale_one_over_d": ("scale = 1.0 / np.sqrt(d_k)", "scale = 1.0 / d_k"),
     "softmax_over_queries": ("w = w / w.sum(axis=1, keepdims=True)", "w = w / w.sum(axis=0, keepdims=True)"),
+    "rows_keys_of_wrong_frame": ("        t = int(row) // U\n", "        t = int(row) // U + 1\n"),
     "gate_sign": ("return O * (1.0 / (1.0 + np.exp(-g)))", "return O * (1.0 / (1.0 + np.exp(g)))"),
     "merge_drops_linear": ("return Ot_S.reshape(N, -1) @ W_S + Ot_L.reshape(N, -1) @ W_L",
                            "return Ot_S.reshape(N, -1) @ W_S"),
@@ -153,7 +166,7 @@ MUTATIONS = {
 def _mutant(name):
     src = inspect.getsource(ho)
     old, new = MUTATIONS[name]
-    assert src.count(old) == 1, name
+    assert src.count(old) >= 1, name  # a systematic mistake: planted wherever the text occurs
     mod = types.ModuleType("hybrid_oracle_mutant_" + name)
     exec(compile(src.replace(old, new), mod.__name__, "exec"), mod.__dict__)
     return mod
@@ -165,6 +178,7 @@ def _checks(mod):
         (test_anchor_density_matches_the_printed_figure, ()),
         (test_window_softmax_matches_token_pair_mask, (9, 3, 2, 4)),
         (test_window_softmax_matches_token_pair_mask, (13, 2, 3, 5)),
+        (test_sampled_rows_match_the_token_pair_mask, (13, 2, 3, 5)),
         (test_window_spanning_the_clip_is_dense_attention, ()),
         (test_outputs_are_convex_combinations_of_visible_values, ()),
         (test_key_order_within_a_frame_does_not_matter, ()),
