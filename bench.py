@@ -465,6 +465,174 @@ def run_reference(args, cfg, rank, world):
 
 
 # ----------------------------------------------------------------------------
+# Softmax branch and the whole hybrid layer (--path softmax / hybrid)
+# ----------------------------------------------------------------------------
+def attention_pairs(cfg) -> int:
+    """(query, visible key) token pairs of the window + anchor softmax per (b, h)."""
+    from frame_level_delta_b200.inputs import CONFIGS  # noqa: F401 (keeps the import style of the module)
+    c, T, U = cfg.chunk, cfg.T, cfg.U
+    n = 0
+    for t in range(T):
+        if t in (0, T - 1):
+            n += T
+        else:
+            j = t // c
+            lo, hi = max(0, c * (j - 1)), min(T - 1, c * (j + 2) - 1)
+            n += (hi - lo + 1) + (1 if lo > 0 else 0) + (1 if hi < T - 1 else 0)
+    return n * U * U
+
+
+def attention_flops(cfg) -> float:
+    """Two d-deep products (Q K^T and P V) per visible pair: 4 d flops."""
+    return 4.0 * cfg.d * attention_pairs(cfg) * cfg.B * cfg.H
+
+
+def attention_bytes(cfg) -> float:
+    """Q, K, V, gate read once and O written once (bf16)."""
+    return 5.0 * cfg.B * cfg.T * cfg.U * cfg.H * cfg.d * 2
+
+
+def merge_flops(cfg, n_model: int) -> float:
+    return 2.0 * cfg.B * cfg.T * cfg.U * (2 * cfg.H * cfg.d) * n_model
+
+
+def time_attention_oracle(cfg, inp, budget_s: float):
+    """The float64 oracle's window softmax on query tokens of head 0, frame by
+    frame from the middle of the clip, until the budget is spent."""
+    import numpy as np
+    from oracle.hybrid_oracle import softmax_gate, window_softmax_rows
+    Q, K, V, g = (inp[k][0, :, 0].double().numpy() for k in ("Q", "K", "V", "gate"))
+    done, t0 = 0, time.perf_counter()
+    rows = list(range((cfg.T // 2) * cfg.U, cfg.T * cfg.U)) + list(range(0, (cfg.T // 2) * cfg.U))
+    step = 64
+    while time.perf_counter() - t0 < budget_s and done < len(rows):
+        r = rows[done:done + step]
+        softmax_gate(window_softmax_rows(Q, K, V, cfg.T, cfg.U, cfg.chunk, r), g[r])
+        done += len(r)
+    return done, time.perf_counter() - t0
+
+
+def run_attention_path(args, cfg, rank, world, local, dist, dev):
+    """One step = the softmax branch (--path softmax) or the whole hybrid layer's
+    attention (--path hybrid: linear branch, softmax branch and the merge by the
+    two output projections, model width H d) over one synthetic batch."""
+    from frame_level_delta_b200 import vda as V
+    from frame_level_delta_b200.inputs import make_attention_inputs, make_merge_inputs
+    hybrid = args.path == "hybrid"
+    inp_cpu = make_inputs(cfg, seed=rank_seed(cfg, rank)) if hybrid else {}
+    att = make_attention_inputs(cfg, seed=rank_seed(cfg, rank))
+    if hybrid:
+        att = {k: att[k] for k in ("gate",)}
+        att.update({k: inp_cpu[k] for k in ("Q", "K", "V")})
+    n_model = cfg.H * cfg.d
+    W = make_merge_inputs(1, n_model, cfg.H * cfg.d, seed=rank) if hybrid else {}
+    host = {k: v.pin_memory() for k, v in {**inp_cpu, **att}.items()}
+    dinp = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
+    Wd = {k: W[k].to(dev) for k in ("W_soft", "W_lin")} if hybrid else {}
+    ctx = V.VDA(cfg, device=dev)
+    O_soft = ctx.new_output()
+    O_lin = ctx.new_output() if hybrid else None
+    M = cfg.B * cfg.T * cfg.U
+    Y = torch.empty(M, n_model, dtype=torch.bfloat16, device=dev) if hybrid else None
+    mstat = torch.zeros(256, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(d, o_soft, o_lin, y):
+        if hybrid:
+            ctx.run(d, o_lin)
+        ctx.window_attention(d["Q"], d["K"], d["V"], d["gate"], o_soft)
+        if hybrid:
+            V.hybrid_merge(o_soft, Wd["W_soft"], o_lin, Wd["W_lin"], y, status=mstat)
+
+    for _ in range(args.warmup):
+        step(dinp, O_soft, O_lin, Y)
+    torch.cuda.synchronize(dev)
+    if ctx.poll_device_status() != 0:
+        raise RuntimeError("device status reported a timeout during warm-up")
+    n0 = ctx.launch_count()
+    clocks = ClockSampler(local)
+    ctx.profile_enable(True)
+    barrier(dist)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step(dinp, O_soft, O_lin, Y)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.stop()
+    barrier(dist)
+    ms = ev0.elapsed_time(ev1)
+    prof = ctx.profile_read()
+    ctx.profile_enable(False)
+    launches = ctx.launch_count() - n0 + (args.steps if hybrid else 0)  # + one merge launch per step
+    if ctx.poll_device_status() != 0 or int(mstat[:4].view(torch.int32).item()) != 0:
+        raise RuntimeError("device status reported a timeout in the timed region")
+    ms_max = max_over_ranks(dist, ms, dev)
+    value = whole_job_rate(world, cfg, args.steps, ms_max)
+
+    # End to end: pinned host inputs up, the step, the result back, every step (serial).
+    out_host = torch.empty((M, n_model) if hybrid else tuple(O_soft.shape), dtype=torch.bfloat16, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * 2
+    ke = max(1, min(args.e2e_steps, args.steps, 5))
+    barrier(dist)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(ke):
+        for k, v in host.items():
+            dinp[k].copy_(v, non_blocking=True)
+        step(dinp, O_soft, O_lin, Y)
+        out_host.copy_(Y if hybrid else O_soft, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dist)
+    e2e_value = whole_job_rate(world, cfg, ke, max_over_ranks(dist, e0.elapsed_time(e1), dev))
+
+    peaks, peak_src = load_peaks()
+    att_n, att_ms = prof["window_attn_tc"]
+    att_s = att_ms / att_n / 1e3
+    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    achieved = attention_flops(cfg) / att_s / 1e12
+    step_s = ms_max / 1e3 / args.steps
+    kernels = {k: {"launches": n, "avg_us": tot / n * 1e3} for k, (n, tot) in prof.items()}
+    if rank == 0:
+        metric = ("hybrid attention layer (VDA linear branch + window softmax + merge) head-tokens/s"
+                  if hybrid else "window + anchor softmax branch head-tokens/s; % of B200 bf16 tensor peak")
+        line = {
+            "metric": metric, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "vda",
+            "config": {"workload": workload_desc(cfg) + ("" if hybrid else ", softmax branch, logit std 1"),
+                       "path": args.path, "model_width": n_model if hybrid else None,
+                       "l2": "no flush: each step reads > 1 GB of tokens, far above the 126 MB L2"},
+            "roofline": {"bound": "tensor", "kernel": "window_attn_tc", "achieved": achieved, "peak": peak,
+                         "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                         "peak_source": f"bf16_tflops_sustained of {peak_src} (each launch runs for tens of ms)",
+                         "frac_of_burst": achieved / float(peaks["bf16_tflops"]),
+                         "algorithmic_flops_per_launch": attention_flops(cfg),
+                         "algorithmic_bytes_per_launch": attention_bytes(cfg)},
+            "step_tflops": (attention_flops(cfg) + (merge_flops(cfg, n_model) + path_flops(cfg) if hybrid else 0))
+                           / step_s / 1e12,
+            "kernels": kernels, "gpu_launches": launches, "clocks": clocks.summary(),
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": ke, "note": "serial copies: inputs up, step, result down"},
+        }
+        if world == 1 and args.cpu_budget > 0:
+            done, dt = time_attention_oracle(cfg, att, args.cpu_budget)
+            line["cpu_baseline"] = {
+                "value": done / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                "blas": blas_library(),
+                "sample": f"float64 oracle window softmax (+gate) of {done} query tokens of head 0, {dt:.2f} s"
+                          + ("; the linear branch's oracle is timed by --path linear" if hybrid else "")}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -480,6 +648,9 @@ def main():
                     help="tensor-core scan frame by frame (default) or over composed chunk maps")
     ap.add_argument("--heads", type=int, default=0,
                     help="override H (a smaller case of the same workload, e.g. for profiler captures)")
+    ap.add_argument("--path", default="linear", choices=["linear", "softmax", "hybrid"],
+                    help="linear: the VDA linear branch (the headline); softmax: the window + anchor "
+                         "softmax branch; hybrid: both branches and the merge")
     ap.add_argument("--shard", default="batch", choices=["batch", "heads"],
                     help="N > 1: a batch per rank (weak scaling) or one batch's heads split over the ranks")
     args = ap.parse_args()
@@ -502,6 +673,8 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     dist = init_ranks(world, dev)
+    if args.path != "linear":
+        return run_attention_path(args, cfg, rank, world, local, dist, dev)
 
     # Each rank draws its own batch (independent problems), or all draw the one
     # batch whose heads they split.

@@ -127,6 +127,7 @@ enum KernelId {
   K_COMPOSE_TC,
   K_SOLVE_CHOL_TC,
   K_WINDOW_ATTN_TC,
+  K_MERGE_TC,
   K_NUM_KERNELS
 };
 const char* kernel_name(int id);
@@ -164,5 +165,8 @@ cudaError_t launch_readout_tc(const Problem& p, const void* gate, void* O, cudaS
 bool window_attn_tc_supported(const Problem& p);
 cudaError_t launch_window_attn_tc(const Problem& p, const void* Q, const void* K, const void* V, const void* gate,
                                   void* O, cudaStream_t s);
+// Hybrid merge Y = A1 B1^T + A2 B2^T (bf16, K-major rows; Y [M, N] bf16).
+cudaError_t launch_merge_tc(const void* A1, const void* B1, const void* A2, const void* B2, void* Y, int M, int N,
+                            int K1, int K2, uint32_t* status, unsigned long long wait_ns, cudaStream_t s);
 
 }  // namespace vda

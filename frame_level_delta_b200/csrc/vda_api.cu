@@ -20,7 +20,7 @@ const char* kernel_name(int id) {
   static const char* names[K_NUM_KERNELS] = {
       "prep_video", "prep_text", "gram_simt", "gram_tc", "solve_simt",
       "scan_simt", "readout_simt", "readout_tc", "zero_anchors", "solve_tc", "scan_tc", "compose_tc",
-      "solve_chol_tc", "window_attn_tc"};
+      "solve_chol_tc", "window_attn_tc", "merge_tc"};
   return (id >= 0 && id < K_NUM_KERNELS) ? names[id] : "?";
 }
 
@@ -534,6 +534,23 @@ vda_status vda_launch_count(const vda_ctx* ctx, uint64_t* launches) {
 vda_status vda_selftest_bounded_wait(uint32_t* status_dev, uint64_t spins, void* stream) {
   if (!status_dev || !aligned16(status_dev)) return VDA_ERR_INVALID_ARG;
   cudaError_t e = launch_selftest_wait(status_dev, spins, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? VDA_OK : VDA_ERR_CUDA;
+}
+
+vda_status vda_hybrid_merge(const void* O_soft, const void* W_soft, const void* O_lin, const void* W_lin, void* Y,
+                            int M, int N, int K, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!O_soft || !W_soft || !O_lin || !W_lin || !Y || !workspace) return VDA_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 1 || N % 8 != 0 || K % 8 != 0) return VDA_ERR_INVALID_ARG;
+  if ((long long)M * N >= (1LL << 40) || (long long)M * K >= (1LL << 40)) return VDA_ERR_INVALID_ARG;
+  const void* ptrs[] = {O_soft, W_soft, O_lin, W_lin, Y};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return VDA_ERR_ALIGNMENT;
+  if (((uintptr_t)workspace & 255) != 0) return VDA_ERR_ALIGNMENT;
+  if (workspace_bytes < 256) return VDA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  if (cudaMemsetAsync(status, 0, sizeof(uint32_t), s) != cudaSuccess) return VDA_ERR_CUDA;
+  cudaError_t e = launch_merge_tc(O_soft, W_soft, O_lin, W_lin, Y, M, N, K, K, status, 2000000000ull, s);
   return e == cudaSuccess ? VDA_OK : VDA_ERR_CUDA;
 }
 

@@ -177,3 +177,18 @@ def make_attention_inputs(cfg: VDAConfig, logit_std: float = 1.0, seed: Optional
     if gate:
         out["gate"] = randn(B, T * U, H, d).to(sd).contiguous()
     return out
+
+
+def make_merge_inputs(M: int, N: int, K: int, seed: int = 0) -> Dict[str, torch.Tensor]:
+    """Seeded inputs of the hybrid merge: the two gated branch outputs O_soft, O_lin
+    [M, K] ~ N(0, 1) and the output projections W_soft, W_lin [N, K] ~ N(0, 1/K)
+    (the [out, in] layout of a linear layer), all bf16. Draw order: O_soft, O_lin,
+    W_soft, W_lin."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed + 2000)
+
+    def randn(*shape, scale=1.0):
+        return (torch.randn(*shape, generator=g, dtype=torch.float32) * scale).to(torch.bfloat16).contiguous()
+
+    return {"O_soft": randn(M, K), "O_lin": randn(M, K), "W_soft": randn(N, K, scale=K ** -0.5),
+            "W_lin": randn(N, K, scale=K ** -0.5)}

@@ -31,7 +31,8 @@ REGIONS = {"status": 0, "A": 1, "B": 2, "M": 3, "C": 4, "S_fwd": 5, "S_rev": 6,
 
 # Exported symbols, in the order include/vda.h declares them.
 EXPORTS = ["vda_create", "vda_destroy", "vda_workspace_size", "vda_prepare", "vda_scan_bidir",
-           "vda_readout", "vda_poll_device_status", "vda_window_attention", "vda_workspace_region", "vda_status_string",
+           "vda_readout", "vda_poll_device_status", "vda_window_attention", "vda_hybrid_merge",
+           "vda_workspace_region", "vda_status_string",
            "vda_last_error", "vda_profile_enable", "vda_num_kernels", "vda_profile_read",
            "vda_launch_count", "vda_describe", "vda_selftest_bounded_wait",
            "vda_selftest_recip", "vda_static_workspace_capacity", "vda_run_static_workspace",
@@ -73,6 +74,7 @@ def lib() -> ctypes.CDLL:
         L.vda_readout.argtypes = [vp, vp, vp, vp]
         L.vda_poll_device_status.argtypes = [vp, vp]
         L.vda_window_attention.argtypes = [vp] * 7 + [sz, vp]
+        L.vda_hybrid_merge.argtypes = [vp] * 5 + [i, i, i, vp, sz, vp]
         L.vda_workspace_region.argtypes = [cfgp, i, ctypes.POINTER(sz), ctypes.POINTER(sz)]
         L.vda_status_string.argtypes = [st]
         L.vda_status_string.restype = ctypes.c_char_p
@@ -395,6 +397,31 @@ def run_static_workspace(cfg: VDAConfig, inp: Dict[str, torch.Tensor], O: torch.
         ctypes.byref(c), _ptr(inp["Q"]), _ptr(inp["K"]), _ptr(inp["V"]), _ptr(inp["K_txt"]), _ptr(inp["V_txt"]),
         _ptr(inp["alpha"]), _ptr(inp["beta"]), _ptr(inp["beta_txt"]), _ptr(inp.get("conv_w")),
         _ptr(inp.get("gate")), _ptr(O), _stream_handle(stream))
+
+
+def hybrid_merge(O_soft: torch.Tensor, W_soft: torch.Tensor, O_lin: torch.Tensor, W_lin: torch.Tensor,
+                 Y: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """Y = O_soft W_soft^T + O_lin W_lin^T through vda_hybrid_merge. The branch
+    outputs may be [B, T*U, H, d] (viewed as [B*T*U, H*d]); the projections are
+    [N, H*d] bf16. ``status`` (256 device bytes) receives the call's status word."""
+    M = O_soft.numel() // O_soft.shape[-1] // (O_soft.shape[-2] if O_soft.dim() == 4 else 1)
+    K = W_soft.shape[1]
+    N = W_soft.shape[0]
+    for name, t in (("O_soft", O_soft), ("O_lin", O_lin), ("W_soft", W_soft), ("W_lin", W_lin)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CUDA tensor")
+    if O_soft.numel() != M * K or O_lin.numel() != M * K or tuple(W_lin.shape) != (N, K):
+        raise ValueError("O_soft, O_lin must hold M x K values and W_soft, W_lin be N x K")
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=O_soft.device)
+    if status is None:
+        status = torch.zeros(256, dtype=torch.uint8, device=O_soft.device)
+    st = lib().vda_hybrid_merge(_ptr(O_soft), _ptr(W_soft), _ptr(O_lin), _ptr(W_lin), _ptr(Y), M, N, K,
+                                _ptr(status), status.numel(), _stream_handle(stream))
+    if st != VDA_OK:
+        raise VDAError(st, "vda_hybrid_merge")
+    return Y
 
 
 def static_workspace_poll(stream=None) -> int:

@@ -201,6 +201,25 @@ vda_status vda_window_attention(vda_ctx* ctx, const void* Q, const void* K, cons
                                 void* O, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The hybrid merge of the two gated branch outputs (Video DeltaNet summary,
+ * section "how it differs": each branch has its own output projection and the
+ * two are summed; VDN-H3 post, section "hybrid attention structure"):
+ *   Y = O_soft W_soft^T + O_lin W_lin^T
+ *   O_soft, O_lin  [M, K] bf16: the gated branch outputs with the heads
+ *                  concatenated (a [B, T*U, H, d] output is [M = B*T*U, K = H*d])
+ *   W_soft, W_lin  [N, K] bf16: the output projections, [out, in] as a linear
+ *                  layer stores them
+ *   Y              [M, N] bf16 (fp32 accumulation on the tensor cores)
+ *   workspace      >= 256 bytes of device memory, 256-byte aligned: the call's
+ *                  device status word (cleared here; non-zero after a bounded
+ *                  device-side wait gave up)
+ * N and K must be multiples of 8 and every pointer 16-byte aligned, else
+ * VDA_ERR_INVALID_ARG / VDA_ERR_ALIGNMENT before any launch. Only enqueues work.
+ */
+vda_status vda_hybrid_merge(const void* O_soft, const void* W_soft, const void* O_lin, const void* W_lin, void* Y,
+                            int M, int N, int K, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Regions of the workspace, for staged parity checks and debugging. Every
  * float32 d x d matrix below (one per slot, chunk or direction) is stored in
  * column quads: element (i, j) at float index ((j / 4) * d + i) * 4 + j % 4 of

@@ -302,3 +302,49 @@ def vda_reference(inp: Dict, cfg, heads: Optional[Iterable[Tuple[int, int]]] = N
             inter[(b, h)] = dict(A=A, B=Bm, M=M, C=C, S_T=S_T, F=F, R=R,
                                  S_fwd=S_fwd, S_rev=S_rev, o_pre_norm=o_pre_norm)
     return {"O": O, "inter": inter, "heads": heads}
+
+
+# ----------------------------------------------------------------------------
+# Backward of one frame step (for training)  [P1 "assumptions and limits": the
+# frame-level update is trained end to end (stages A1/A2/B); the pages print no
+# backward, so this is the plain chain rule of the forward step above]
+# ----------------------------------------------------------------------------
+
+
+def frame_step(S_prev: np.ndarray, Kf: np.ndarray, Vf: np.ndarray, beta: np.ndarray,
+               alpha: np.ndarray) -> np.ndarray:
+    """One frame of the scan: S_t = S_{t-1} M_t + C_t with M_t, C_t from frame_solve."""
+    A, B = frame_stats(Kf, Vf, beta)
+    M, C = frame_solve(A, B, alpha)
+    return S_prev @ M + C
+
+
+def frame_step_backward(S_prev: np.ndarray, Kf: np.ndarray, Vf: np.ndarray, beta: np.ndarray,
+                        alpha: np.ndarray, dS: np.ndarray) -> Dict[str, np.ndarray]:
+    """Vector-Jacobian product of frame_step: given dS = dL/dS_t, the gradients of
+    L with respect to S_{t-1}, K_t, V_t, beta_t and alpha_t.
+
+    With P = (I + A)^-1 (symmetric), X = S_{t-1} Diag(alpha) + B and S_t = X P:
+      dL/dX = dS P^T = dS P =: Gx           (so dL/dB = Gx, dL/dS_{t-1} = Gx Diag(alpha))
+      dL/dP = X^T dS,  dL/dA = -P^T (X^T dS) P^T = -S_t^T Gx =: GA
+      dL/dalpha_k = sum_i S_{t-1}[i, k] Gx[i, k]
+    and through A = sum_u beta_u k_u k_u^T, B = sum_u beta_u v_u k_u^T:
+      dL/dk_u = beta_u ((GA + GA^T) k_u + Gx^T v_u)
+      dL/dv_u = beta_u Gx k_u
+      dL/dbeta_u = k_u^T GA k_u + v_u^T Gx k_u.
+    """
+    A, B = frame_stats(Kf, Vf, beta)
+    d_k = A.shape[0]
+    P = np.linalg.solve(np.eye(d_k) + A, np.eye(d_k))
+    X = S_prev * alpha[None, :] + B
+    S = X @ P
+    Gx = dS @ P.T
+    GA = -(S.T @ Gx)
+    out = {
+        "dS_prev": Gx * alpha[None, :],
+        "dalpha": np.sum(S_prev * Gx, axis=0),
+        "dK": beta[:, None] * (Kf @ (GA + GA.T).T + Vf @ Gx),
+        "dV": beta[:, None] * (Kf @ Gx.T),
+        "dbeta": np.einsum("uk,kl,ul->u", Kf, GA, Kf) + np.einsum("uv,vk,uk->u", Vf, Gx, Kf),
+    }
+    return out

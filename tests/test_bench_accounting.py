@@ -52,3 +52,12 @@ def test_alu_peak_and_prep_count():
     # every input frame's 25-tap spatial sum, amortised over the F outputs, plus 5 temporal taps
     per_value = 25 * 40 / F + 5
     assert bench.kernel_alu_flops("prep_video", cfg) == pytest.approx(H * 2 * F * U * d * 2 * per_value)
+
+
+def test_attention_pair_count_matches_the_oracles_visible_sets():
+    from oracle.hybrid_oracle import visible_frames
+    for name, kw in (("h3", {}), ("small", {}), ("small", dict(T=13, chunk=5)), ("small", dict(T=7, chunk=1))):
+        cfg = CONFIGS[name].with_(**kw)
+        want = sum(len(visible_frames(t, cfg.chunk, cfg.T)) for t in range(cfg.T)) * cfg.U * cfg.U
+        assert bench.attention_pairs(cfg) == want
+        assert bench.attention_flops(cfg) == 4 * cfg.d * want * cfg.B * cfg.H

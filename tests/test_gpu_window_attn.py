@@ -15,7 +15,7 @@ import pytest
 import torch
 
 from frame_level_delta_b200 import vda as V
-from frame_level_delta_b200.inputs import CONFIGS, make_attention_inputs
+from frame_level_delta_b200.inputs import CONFIGS, make_attention_inputs, make_merge_inputs
 from oracle import hybrid_oracle as ho
 from tests.parity import TOL_O, local_output_errors, rel_fro
 
@@ -143,3 +143,64 @@ def test_window_attention_h3_full_size_sampled_rows(spread):
         rn = np.linalg.norm(want, axis=1)
         floor = 0.05 * np.sqrt(np.mean(rn * rn))
         assert (en <= tol * np.maximum(rn, floor)).all(), float((en / np.maximum(rn, floor)).max())
+
+
+# ---------------------------------------------------------------------------
+# Hybrid merge Y = O~S W_S^T + O~L W_L^T (vda_hybrid_merge)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("M,N,K", [(300, 136, 200), (128, 256, 64), (1000, 520, 1032), (7, 8, 8)])
+def test_hybrid_merge_matches_oracle(M, N, K):
+    x = make_merge_inputs(M, N, K, seed=M + N + K)
+    Os, Ol, Ws, Wl = x["O_soft"], x["O_lin"], x["W_soft"], x["W_lin"]
+    Y = V.hybrid_merge(*(t.cuda() for t in (Os, Ws, Ol, Wl)))
+    torch.cuda.synchronize()
+    want = ho.hybrid_output(Os.double().numpy()[:, None, :], Ol.double().numpy()[:, None, :],
+                            Ws.double().numpy().T, Wl.double().numpy().T)
+    got = Y.double().cpu().numpy()
+    assert rel_fro(got, want) <= 5e-3
+    en, rn = np.linalg.norm(got - want, axis=1), np.linalg.norm(want, axis=1)
+    assert (en <= 1e-2 * np.maximum(rn, 0.05 * np.sqrt(np.mean(rn * rn)))).all()
+
+
+def test_hybrid_merge_h3_projection_sampled_rows():
+    """The H3-like clip's merge: 62400 tokens, 24 heads x 128 channels per branch,
+    a 3072-wide model dimension; sampled output rows against the oracle."""
+    cfg = CONFIGS["h3"]
+    M, K, N = cfg.B * cfg.T * cfg.U, cfg.H * cfg.d, cfg.H * cfg.d
+    x = make_merge_inputs(M, N, K, seed=5)
+    Os, Ol, Ws, Wl = x["O_soft"], x["O_lin"], x["W_soft"], x["W_lin"]
+    Y = V.hybrid_merge(*(t.cuda() for t in (Os, Ws, Ol, Wl))).cpu()
+    rows = np.random.default_rng(1).integers(0, M, 300)
+    rows = np.unique(np.concatenate([rows, [0, 127, 128, M - 1]]))
+    want = ho.hybrid_output(Os[rows].double().numpy()[:, None, :], Ol[rows].double().numpy()[:, None, :],
+                            Ws.double().numpy().T, Wl.double().numpy().T)
+    assert rel_fro(Y[rows].double().numpy(), want) <= 5e-3
+
+
+def test_hybrid_layer_end_to_end():
+    """Both branches of one attention layer on the same Q, K, V through the C ABI
+    (the softmax branch with its gate, the linear branch with conv prep, RMSNorm
+    and its gate), merged by the two output projections, against the oracles."""
+    from oracle.vda_oracle import vda_reference
+    from frame_level_delta_b200.inputs import make_inputs
+    cfg = CONFIGS["hires"].with_(H=2, T=9, grid_h=6, grid_w=10, L=5, chunk=2)
+    inp = make_inputs(cfg)
+    ga = make_attention_inputs(cfg)["gate"]  # the softmax branch's own gate logits
+    dev = torch.device("cuda:0")
+    d = {k: v.to(dev) for k, v in inp.items()}
+    ctx = V.VDA(cfg, device=dev)
+    O_lin = ctx.run(d)
+    O_soft = ctx.window_attention(d["Q"], d["K"], d["V"], ga.to(dev))
+    K = cfg.H * cfg.d
+    w = make_merge_inputs(1, 96, K, seed=9)
+    Ws, Wl = w["W_soft"], w["W_lin"]
+    Y = V.hybrid_merge(O_soft, Ws.to(dev), O_lin, Wl.to(dev))
+    torch.cuda.synchronize()
+    assert ctx.poll_device_status() == 0
+    Q, Kk, Vv = (inp[k].double().numpy() for k in ("Q", "K", "V"))
+    o_soft = ho.window_softmax_layer(Q, Kk, Vv, ga.double().numpy(), cfg.T, cfg.U, cfg.chunk)
+    o_lin = vda_reference(inp, cfg, keep=False)["O"]
+    N = cfg.B * cfg.T * cfg.U
+    want = ho.hybrid_output(o_soft.reshape(N, cfg.H, cfg.d), o_lin.reshape(N, cfg.H, cfg.d),
+                            Ws.double().numpy().T, Wl.double().numpy().T)
+    assert rel_fro(Y.double().cpu().numpy(), want) <= TOL_O["bf16"]
