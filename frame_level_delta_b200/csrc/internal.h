@@ -128,6 +128,7 @@ enum KernelId {
   K_SOLVE_CHOL_TC,
   K_WINDOW_ATTN_TC,
   K_MERGE_TC,
+  K_FRAME_BWD_SIMT,
   K_NUM_KERNELS
 };
 const char* kernel_name(int id);
@@ -142,6 +143,11 @@ cudaError_t launch_scan_simt(const Problem& p, cudaStream_t s);
 cudaError_t launch_readout_simt(const Problem& p, const void* gate, void* O, cudaStream_t s);
 cudaError_t launch_zero_anchors(const Problem& p, void* O, cudaStream_t s);
 cudaError_t launch_selftest_wait(uint32_t* status, unsigned long long spins, cudaStream_t s);
+// Backward of the frame step for frames 1..T-2 (after the statistics kernel has
+// written A_t, B_t): writes dS_prev, dalpha, dbeta, dK, dV (and Gx, Gsym into the
+// workspace's M and C slots). Two launches.
+cudaError_t launch_frame_bwd_simt(const Problem& p, const float* S_prev, const float* dS, float* dS_prev,
+                                  float* dalpha, float* dbeta, void* dK, void* dV, cudaStream_t s);
 // The sweep solve's pivot reciprocal applied to x[0..n) (for an error bound test).
 cudaError_t launch_recip_selftest(const float* x, float* y, int n, cudaStream_t s);
 

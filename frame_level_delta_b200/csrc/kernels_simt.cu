@@ -516,6 +516,218 @@ __global__ void selftest_wait_kernel(uint32_t* status, unsigned long long spins)
 }
 
 // ---------------------------------------------------------------------------
+// Backward of one frame step S_t = (S_{t-1} Diag(alpha_t) + B_t)(I + A_t)^-1 for
+// every (b, h, frame t in 1..T-2), given dS_t = dL/dS_t. With P = (I + A)^-1,
+// X = S_{t-1} Diag(alpha) + B, S_t = X P:
+//   Gx = dS P, dS_{t-1} = Gx Diag(alpha), dalpha_k = sum_i S_{t-1}[i,k] Gx[i,k],
+//   GA = -S_t^T Gx (= dL/dA), Gsym = GA + GA^T,
+// and per token u of the frame (k_u, v_u its key and value):
+//   dk_u = beta_u (Gsym k_u + Gx^T v_u),  dv_u = beta_u Gx k_u,
+//   dbeta_u = k_u^T GA k_u + v_u^T Gx k_u = (k_u . (Gsym k_u + Gx^T v_u) + v_u . Gx k_u) / 2
+// (the last form because k.Gx^T v = v.Gx k).
+// solve_bwd_simt_kernel: one CTA per (frame, head, batch), (D/8)^2 threads with
+// 8 x 8 register tiles: the sweep for P (as in the forward solve), then S_t, Gx,
+// GA through shared memory. Writes dS_{t-1}, dalpha and, into the workspace
+// (row-major), Gx and Gsym for the token kernel.
+// ---------------------------------------------------------------------------
+struct BwdArgs {
+  const float* S_prev;  // [B,H,T,D,D] row-major: entry t = S_{t-1}
+  const float* dS;      // [B,H,T,D,D] row-major: dL/dS_t
+  float* dS_prev;       // [B,H,T,D,D]
+  float* dalpha;        // [B,H,T,D]
+  float* dbeta;         // [B,H,T,U]
+  void* dK;             // token tensors [B, T*U, Ht, D] (advanced to the first head)
+  void* dV;
+};
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kSmemFloats = 2 * SweepCfg<D>::kPv + 3 * D * D;
+};
+
+template <int D>
+__global__ void __launch_bounds__(SweepCfg<D>::kThreads) solve_bwd_simt_kernel(Problem p, BwdArgs g) {
+  using C = SweepCfg<D>;
+  extern __shared__ float smem[];
+  float* pv = smem;               // [2][kPv]: pivot vectors, then the dalpha sums
+  float* sP = smem + 2 * C::kPv;  // P, then GA (row-major)
+  float* sS = sP + D * D;         // X, then S_t
+  float* sG = sS + D * D;         // dS, then Gx
+  const int t = blockIdx.x + 1, h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, ti = tid / C::NT, tj = tid % C::NT;
+  const long long off = slot_off(p, b, h, t);
+  const long long uo = ((((long long)b * p.H + h) * p.T) + t) * D * D;
+  const float* alpha = p.alpha + (((long long)b * p.H + h) * p.T + t) * D;
+  for (int e = tid; e < D * D; e += C::kThreads) {
+    const int i = e / D, k = e % D;
+    sS[e] = fmaf(g.S_prev[uo + e], alpha[k], p.Bm[off + quad_off(D, i, k)]);
+    sG[e] = g.dS[uo + e];
+  }
+  // X = I + A in registers, swept to -P.
+  float x[8][8];
+  const float4* A4 = reinterpret_cast<const float4*>(p.A + off);
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int i = 8 * ti + r;
+    const float4 w0 = A4[(2 * tj) * D + i], w1 = A4[(2 * tj + 1) * D + i];
+    x[r][0] = w0.x; x[r][1] = w0.y; x[r][2] = w0.z; x[r][3] = w0.w;
+    x[r][4] = w1.x; x[r][5] = w1.y; x[r][6] = w1.z; x[r][7] = w1.w;
+  }
+  if (ti == tj) {
+#pragma unroll
+    for (int r = 0; r < 8; ++r) x[r][r] += 1.f;
+  }
+  if (ti == 0) sweep_publish<D, 0>(pv, x, ti, tj);
+  __syncthreads();
+#pragma unroll 1
+  for (int K = 0; K < C::NT; ++K) {
+    sweep_simt_step<D, 0>(x, pv, K, ti, tj);
+    sweep_simt_step<D, 1>(x, pv, K, ti, tj);
+    sweep_simt_step<D, 2>(x, pv, K, ti, tj);
+    sweep_simt_step<D, 3>(x, pv, K, ti, tj);
+    sweep_simt_step<D, 4>(x, pv, K, ti, tj);
+    sweep_simt_step<D, 5>(x, pv, K, ti, tj);
+    sweep_simt_step<D, 6>(x, pv, K, ti, tj);
+    sweep_simt_step<D, 7>(x, pv, K, ti, tj);
+  }
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    float4* dst = reinterpret_cast<float4*>(sP + (8 * ti + r) * D + 8 * tj);
+    dst[0] = make_float4(-x[r][0], -x[r][1], -x[r][2], -x[r][3]);
+    dst[1] = make_float4(-x[r][4], -x[r][5], -x[r][6], -x[r][7]);
+  }
+  __syncthreads();
+  // S_t = X P and Gx = dS P: this thread's 8 x 8 tiles.
+  float gx[8][8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) x[r][c] = gx[r][c] = 0.f;
+#pragma unroll 2
+  for (int k = 0; k < D; ++k) {
+    const float4 p0 = reinterpret_cast<const float4*>(sP + k * D + 8 * tj)[0];
+    const float4 p1 = reinterpret_cast<const float4*>(sP + k * D + 8 * tj)[1];
+    const float pc[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const float xs = sS[(8 * ti + r) * D + k], gs = sG[(8 * ti + r) * D + k];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        x[r][c] = fmaf(xs, pc[c], x[r][c]);
+        gx[r][c] = fmaf(gs, pc[c], gx[r][c]);
+      }
+    }
+  }
+  for (int e = tid; e < D; e += C::kThreads) pv[e] = 0.f;
+  __syncthreads();  // X, dS and P are no longer read
+  float part[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) part[c] = 0.f;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int i = 8 * ti + r;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int k = 8 * tj + c;
+      sS[i * D + k] = x[r][c];
+      sG[i * D + k] = gx[r][c];
+      g.dS_prev[uo + i * D + k] = gx[r][c] * alpha[k];
+      p.M[off + i * D + k] = gx[r][c];  // Gx for the token kernel
+      part[c] = fmaf(g.S_prev[uo + i * D + k], gx[r][c], part[c]);
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < 8; ++c) atomicAdd(&pv[8 * tj + c], part[c]);
+  __syncthreads();
+  // GA = -S_t^T Gx: rows a = 8 ti.., columns 8 tj..
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) x[r][c] = 0.f;
+#pragma unroll 2
+  for (int i = 0; i < D; ++i) {
+    const float4 q0 = reinterpret_cast<const float4*>(sG + i * D + 8 * tj)[0];
+    const float4 q1 = reinterpret_cast<const float4*>(sG + i * D + 8 * tj)[1];
+    const float gc[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    const float4 s0 = reinterpret_cast<const float4*>(sS + i * D + 8 * ti)[0];
+    const float4 s1 = reinterpret_cast<const float4*>(sS + i * D + 8 * ti)[1];
+    const float sr[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) x[r][c] = fmaf(-sr[r], gc[c], x[r][c]);
+  }
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) sP[(8 * ti + r) * D + 8 * tj + c] = x[r][c];
+  for (int e = tid; e < D; e += C::kThreads) g.dalpha[(((long long)b * p.H + h) * p.T + t) * D + e] = pv[e];
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int a = 8 * ti + r, bb = 8 * tj + c;
+      p.C[off + a * D + bb] = sP[a * D + bb] + sP[bb * D + a];  // Gsym
+    }
+}
+
+// token_bwd_simt_kernel: grid (ceil(U / 32), T-2, B*H), 256 threads: eight per
+// token of a 32-token tile, each producing D/8 of the token's outputs from Gsym
+// and Gx in shared memory (rows padded to D + 1 floats).
+template <int D>
+__global__ void __launch_bounds__(256) token_bwd_simt_kernel(Problem p, BwdArgs g) {
+  constexpr int LD = D + 1, TT = 32;
+  extern __shared__ float smem[];
+  float* sGs = smem;            // [D][LD]
+  float* sGx = sGs + D * LD;    // [D][LD]
+  float* sK = sGx + D * LD;     // [TT][LD]
+  float* sV = sK + TT * LD;     // [TT][LD]
+  const int t = blockIdx.y + 1, bh = blockIdx.z, b = bh / p.H, h = bh % p.H;
+  const int u0 = blockIdx.x * TT;
+  const long long off = slot_off(p, b, h, t);
+  for (int e = threadIdx.x; e < D * D; e += blockDim.x) {
+    sGs[(e / D) * LD + e % D] = p.C[off + e];
+    sGx[(e / D) * LD + e % D] = p.M[off + e];
+  }
+  const long long kb = b * p.Kv.s_b + h * p.Kv.s_h + t * p.Kv.s_t;
+  const long long vb = b * p.Vv.s_b + h * p.Vv.s_h + t * p.Vv.s_t;
+  for (int e = threadIdx.x; e < TT * D; e += blockDim.x) {
+    const int uu = e / D, k = e % D, u = u0 + uu;
+    sK[uu * LD + k] = u < p.U ? ld_tok(p.Kv.p, kb + u * p.Kv.s_u + k, p.bf16) : 0.f;
+    sV[uu * LD + k] = u < p.U ? ld_tok(p.Vv.p, vb + u * p.Vv.s_u + k, p.bf16) : 0.f;
+  }
+  __syncthreads();
+  const int uu = threadIdx.x / 8, q = threadIdx.x % 8, u = u0 + uu;
+  const bool live = u < p.U;
+  const float beta = live ? p.beta[(((long long)b * p.H + h) * p.T + t) * p.U + u] : 0.f;
+  const long long row = (((long long)b * p.T * p.U) + (long long)t * p.U + (live ? u : 0)) * p.Ht + h;
+  float db = 0.f;
+#pragma unroll 1
+  for (int m = 0; m < D / 8; ++m) {
+    const int n = q + 8 * m;
+    float w = 0.f, y = 0.f, z = 0.f;
+#pragma unroll 8
+    for (int k = 0; k < D; ++k) {
+      const float kk = sK[uu * LD + k], vv = sV[uu * LD + k];
+      w = fmaf(sGs[n * LD + k], kk, w);
+      y = fmaf(sGx[k * LD + n], vv, y);
+      z = fmaf(sGx[n * LD + k], kk, z);
+    }
+    const float a1 = w + y;
+    db = fmaf(sK[uu * LD + n], a1, fmaf(sV[uu * LD + n], z, db));
+    if (live) {
+      st_tok(g.dK, row * D + n, beta * a1, p.bf16);
+      st_tok(g.dV, row * D + n, beta * z, p.bf16);
+    }
+  }
+  db += __shfl_xor_sync(0xffffffffu, db, 1);
+  db += __shfl_xor_sync(0xffffffffu, db, 2);
+  db += __shfl_xor_sync(0xffffffffu, db, 4);
+  if (live && q == 0) g.dbeta[(((long long)b * p.H + h) * p.T + t) * p.U + u] = 0.5f * db;
+}
+
+// ---------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------
 template <typename F>
@@ -585,6 +797,25 @@ cudaError_t launch_prep_text(const Problem& p, const void* Kt, const void* Vt, c
   const int blocks = (int)((warps * 32 + 255) / 256);
   prep_text_kernel<<<blocks, 256, 0, s>>>(p, Kt, Vt);
   return cudaGetLastError();
+}
+
+cudaError_t launch_frame_bwd_simt(const Problem& p, const float* S_prev, const float* dS, float* dS_prev,
+                                  float* dalpha, float* dbeta, void* dK, void* dV, cudaStream_t s) {
+  if (p.T < 3) return cudaSuccess;
+  const BwdArgs g{S_prev, dS, dS_prev, dalpha, dbeta, dK, dV};
+  return dispatch_d(p.D, [&](auto dc) {
+    constexpr int D = decltype(dc)::value;
+    const size_t sm1 = (size_t)BwdCfg<D>::kSmemFloats * sizeof(float);
+    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(solve_bwd_simt_kernel<D>), (int)sm1);
+    if (e != cudaSuccess) return e;
+    solve_bwd_simt_kernel<D><<<dim3(p.T - 2, p.H, p.B), SweepCfg<D>::kThreads, sm1, s>>>(p, g);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const size_t sm2 = (size_t)(2 * D + 2 * 32) * (D + 1) * sizeof(float);
+    e = set_max_dynamic_smem(reinterpret_cast<const void*>(token_bwd_simt_kernel<D>), (int)sm2);
+    if (e != cudaSuccess) return e;
+    token_bwd_simt_kernel<D><<<dim3((p.U + 31) / 32, p.T - 2, p.B * p.H), 256, sm2, s>>>(p, g);
+    return cudaGetLastError();
+  });
 }
 
 cudaError_t launch_selftest_wait(uint32_t* status, unsigned long long spins, cudaStream_t s) {

@@ -20,7 +20,7 @@ const char* kernel_name(int id) {
   static const char* names[K_NUM_KERNELS] = {
       "prep_video", "prep_text", "gram_simt", "gram_tc", "solve_simt",
       "scan_simt", "readout_simt", "readout_tc", "zero_anchors", "solve_tc", "scan_tc", "compose_tc",
-      "solve_chol_tc", "window_attn_tc", "merge_tc"};
+      "solve_chol_tc", "window_attn_tc", "merge_tc", "frame_bwd_simt"};
   return (id >= 0 && id < K_NUM_KERNELS) ? names[id] : "?";
 }
 
@@ -535,6 +535,66 @@ vda_status vda_selftest_bounded_wait(uint32_t* status_dev, uint64_t spins, void*
   if (!status_dev || !aligned16(status_dev)) return VDA_ERR_INVALID_ARG;
   cudaError_t e = launch_selftest_wait(status_dev, spins, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? VDA_OK : VDA_ERR_CUDA;
+}
+
+vda_status vda_frame_solve_backward(vda_ctx* ctx, const void* K, const void* V, const float* alpha,
+                                    const float* beta, const float* S_prev, const float* dS, void* dK, void* dV,
+                                    float* dalpha, float* dbeta, float* dS_prev, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  if (!ctx) return VDA_ERR_INVALID_ARG;
+  const vda_config& c = ctx->cfg;
+  if (c.flags & VDA_PREP_CONV)
+    return fail(ctx, VDA_ERR_UNSUPPORTED, "the frame-step backward takes prepared keys and values (no conv prep)");
+  const void* ptrs[] = {K, V, alpha, beta, S_prev, dS, dK, dV, dalpha, dbeta, dS_prev};
+  for (const void* q : ptrs)
+    if (!q) return fail(ctx, VDA_ERR_INVALID_ARG, "a required pointer is NULL");
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return fail(ctx, VDA_ERR_ALIGNMENT, "every tensor must be 16-byte aligned");
+  if (!workspace) return fail(ctx, VDA_ERR_INVALID_ARG, "workspace is NULL");
+  if (((uintptr_t)workspace & 255) != 0) return fail(ctx, VDA_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  const Layout L = make_layout(c);
+  if (workspace_bytes < L.total) return fail(ctx, VDA_ERR_WORKSPACE_TOO_SMALL, "workspace smaller than vda_workspace_size()");
+  char* ws = static_cast<char*>(workspace);
+  Problem p{};
+  p.B = c.B; p.H = c.H; p.T = c.T; p.U = c.U; p.D = c.d_k; p.c = c.chunk; p.J = J_of(c);
+  p.gh = c.grid_h; p.gw = c.grid_w; p.Ht = heads_total(c);
+  p.bf16 = c.dtype == VDA_BF16;
+  p.flags = c.flags;
+  p.alpha = alpha;
+  p.beta = beta;
+  p.status = reinterpret_cast<uint32_t*>(ws + L.off[VDA_REGION_STATUS]);
+  p.A = reinterpret_cast<float*>(ws + L.off[VDA_REGION_A]);
+  p.Bm = reinterpret_cast<float*>(ws + L.off[VDA_REGION_B]);
+  p.M = reinterpret_cast<float*>(ws + L.off[VDA_REGION_M]);
+  p.C = reinterpret_cast<float*>(ws + L.off[VDA_REGION_C]);
+  p.spin_limit = 2000000000ull;
+  const long long D = p.D, T = p.T, U = p.U, Ht = p.Ht;
+  K = head_slice(c, K);
+  V = head_slice(c, V);
+  dK = head_slice(c, dK);
+  dV = head_slice(c, dV);
+  p.Kv = TokView{K, T * U * Ht * D, D, U * Ht * D, Ht * D};
+  p.Vv = TokView{V, T * U * Ht * D, D, U * Ht * D, Ht * D};
+  // The statistics kernels also form a text slot (slot 0), which the backward
+  // does not use: point it at one token of the video keys.
+  p.L = 1;
+  p.Kt = TokView{K, Ht * D, D, 0, Ht * D};
+  p.Vt = TokView{V, Ht * D, D, 0, Ht * D};
+  p.beta_txt = beta;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(p.status, 0, L.bytes[VDA_REGION_STATUS], s);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "status reset");
+  ctx->p.status = p.status;  // for vda_poll_device_status
+  vda_status st;
+  if (!use_simt_only(c) && gram_tc_supported(p))
+    st = run_kernel(ctx, K_GRAM_TC, s, [&] { return launch_gram_tc(p, s); });
+  else
+    st = run_kernel(ctx, K_GRAM_SIMT, s, [&] { return launch_gram_simt(p, s); });
+  if (st != VDA_OK) return st;
+  ctx->prepared = ctx->scanned = false;  // the workspace no longer holds a forward pass
+  return run_kernel(ctx, K_FRAME_BWD_SIMT, s, [&] {
+    return launch_frame_bwd_simt(p, S_prev, dS, dS_prev, dalpha, dbeta, dK, dV, s);
+  });
 }
 
 vda_status vda_hybrid_merge(const void* O_soft, const void* W_soft, const void* O_lin, const void* W_lin, void* Y,

@@ -192,3 +192,15 @@ def make_merge_inputs(M: int, N: int, K: int, seed: int = 0) -> Dict[str, torch.
 
     return {"O_soft": randn(M, K), "O_lin": randn(M, K), "W_soft": randn(N, K, scale=K ** -0.5),
             "W_lin": randn(N, K, scale=K ** -0.5)}
+
+
+def make_backward_inputs(cfg: VDAConfig, seed: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """Seeded inputs of the frame-step backward on top of make_inputs(cfg): the
+    state before each frame S_prev and the upstream gradient dS, both
+    [B, H, T, d, d] float32 ~ N(0, 1) (row-major d_v x d_k per frame). Draw order:
+    S_prev, dS."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed((cfg.seed if seed is None else seed) + 3000)
+    shape = (cfg.B, cfg.H, cfg.T, cfg.d, cfg.d)
+    return {"S_prev": torch.randn(*shape, generator=g).contiguous(),
+            "dS": torch.randn(*shape, generator=g).contiguous()}

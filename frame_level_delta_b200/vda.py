@@ -31,7 +31,8 @@ REGIONS = {"status": 0, "A": 1, "B": 2, "M": 3, "C": 4, "S_fwd": 5, "S_rev": 6,
 
 # Exported symbols, in the order include/vda.h declares them.
 EXPORTS = ["vda_create", "vda_destroy", "vda_workspace_size", "vda_prepare", "vda_scan_bidir",
-           "vda_readout", "vda_poll_device_status", "vda_window_attention", "vda_hybrid_merge",
+           "vda_readout", "vda_poll_device_status", "vda_window_attention", "vda_frame_solve_backward",
+           "vda_hybrid_merge",
            "vda_workspace_region", "vda_status_string",
            "vda_last_error", "vda_profile_enable", "vda_num_kernels", "vda_profile_read",
            "vda_launch_count", "vda_describe", "vda_selftest_bounded_wait",
@@ -75,6 +76,7 @@ def lib() -> ctypes.CDLL:
         L.vda_poll_device_status.argtypes = [vp, vp]
         L.vda_window_attention.argtypes = [vp] * 7 + [sz, vp]
         L.vda_hybrid_merge.argtypes = [vp] * 5 + [i, i, i, vp, sz, vp]
+        L.vda_frame_solve_backward.argtypes = [vp] * 13 + [sz, vp]
         L.vda_workspace_region.argtypes = [cfgp, i, ctypes.POINTER(sz), ctypes.POINTER(sz)]
         L.vda_status_string.argtypes = [st]
         L.vda_status_string.restype = ctypes.c_char_p
@@ -319,6 +321,34 @@ class VDA:
                                                    _ptr(self._attn_ws), 256, _stream_handle(stream)),
                         "vda_window_attention")
         return O
+
+    def frame_solve_backward(self, K: torch.Tensor, V: torch.Tensor, alpha: torch.Tensor, beta: torch.Tensor,
+                             S_prev: torch.Tensor, dS: torch.Tensor, stream=None) -> Dict[str, torch.Tensor]:
+        """Backward of the frame step for frames 1..T-2 (vda_frame_solve_backward).
+        Returns dK, dV (storage dtype) and dS_prev, dalpha, dbeta (float32), zero
+        on the anchor frames."""
+        cfg = self.cfg
+        sd = torch.float32 if cfg.dtype == "f32" else torch.bfloat16
+        B, H, T, U, d = cfg.B, self.c.H, cfg.T, cfg.U, cfg.d
+        tok = (cfg.B, T * U, cfg.H, d)
+        self._expect("K", K, tok, sd)
+        self._expect("V", V, tok, sd)
+        p = self._head_params({"alpha": alpha, "beta": beta, "beta_txt": beta[:, :, 0]}) if self.heads else \
+            {"alpha": alpha, "beta": beta}
+        self._expect("alpha", p["alpha"], (B, H, T, d), torch.float32)
+        self._expect("beta", p["beta"], (B, H, T, U), torch.float32)
+        self._expect("S_prev", S_prev, (B, H, T, d, d), torch.float32)
+        self._expect("dS", dS, (B, H, T, d, d), torch.float32)
+        out = {"dK": torch.zeros(tok, dtype=sd, device=self.device), "dV": torch.zeros(tok, dtype=sd, device=self.device),
+               "dS_prev": torch.zeros_like(S_prev), "dalpha": torch.zeros_like(p["alpha"]),
+               "dbeta": torch.zeros_like(p["beta"])}
+        ws = self.ensure_workspace()
+        with self._on_device():
+            self._check(lib().vda_frame_solve_backward(
+                self._ctx, _ptr(K), _ptr(V), _ptr(p["alpha"]), _ptr(p["beta"]), _ptr(S_prev), _ptr(dS),
+                _ptr(out["dK"]), _ptr(out["dV"]), _ptr(out["dalpha"]), _ptr(out["dbeta"]), _ptr(out["dS_prev"]),
+                _ptr(ws), ws.numel(), _stream_handle(stream)), "vda_frame_solve_backward")
+        return out
 
     def poll_device_status(self, stream=None) -> int:
         with self._on_device():

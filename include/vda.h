@@ -201,6 +201,33 @@ vda_status vda_window_attention(vda_ctx* ctx, const void* Q, const void* K, cons
                                 void* O, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Backward of one frame step of the scan, for training: for every head and every
+ * non-anchor frame t = 1 .. T-2, the vector-Jacobian product of
+ *   S_t = (S_{t-1} Diag(alpha_t) + B_t)(I + A_t)^-1,  A_t = K_t^T Diag(beta_t) K_t,
+ *   B_t = V_t^T Diag(beta_t) K_t
+ * (Video DeltaNet summary, onedev.kr/papers/80, section "how to use": the frame
+ * solve; section "assumptions and limits": the update is trained end to end; the
+ * pages print no backward, so this is the chain rule of the forward step). Given
+ * dS = dL/dS_t it returns dL/dS_{t-1}, dL/dK_t, dL/dV_t, dL/dbeta_t, dL/dalpha_t.
+ *   K, V           [B, T*U, H_total, d] storage dtype (prepared keys and values)
+ *   alpha, beta    [B, H, T, d_k], [B, H, T, U] float32, as for vda_prepare
+ *   S_prev, dS     [B, H, T, d_v, d_k] float32 row-major: entry t is S_{t-1} and
+ *                  dL/dS_t (entries of anchor frames 0 and T-1 are not read)
+ *   dK, dV         [B, T*U, H_total, d] storage dtype; dS_prev [B, H, T, d_v, d_k],
+ *   dalpha, dbeta  [B, H, T, d_k], [B, H, T, U] float32: written for frames
+ *                  1 .. T-2 only, every other entry is left as it was
+ *   workspace      >= vda_workspace_size(cfg) bytes, 256-byte aligned (its A, B,
+ *                  M and C regions are overwritten; a later vda_scan_bidir needs a
+ *                  new vda_prepare)
+ * Not with VDA_PREP_CONV (VDA_ERR_UNSUPPORTED). Only enqueues work; device-side
+ * timeouts are read with vda_poll_device_status.
+ */
+vda_status vda_frame_solve_backward(vda_ctx* ctx, const void* K, const void* V, const float* alpha,
+                                    const float* beta, const float* S_prev, const float* dS, void* dK, void* dV,
+                                    float* dalpha, float* dbeta, float* dS_prev, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+
+/*
  * The hybrid merge of the two gated branch outputs (Video DeltaNet summary,
  * section "how it differs": each branch has its own output projection and the
  * two are summed; VDN-H3 post, section "hybrid attention structure"):

@@ -43,9 +43,11 @@ MUTATIONS = {
 def _mutant(name):
     src = inspect.getsource(vo)
     old, new = MUTATIONS[name]
-    assert src.count(old) == 1, name
+    assert src.count(old) >= 1, name
     mod = types.ModuleType("vda_oracle_mutant_" + name)
-    exec(compile(src.replace(old, new), mod.__name__, "exec"), mod.__dict__)
+    # The first occurrence is the forward path's (the frame-step backward, further
+    # down, repeats some lines and has pins of its own).
+    exec(compile(src.replace(old, new, 1), mod.__name__, "exec"), mod.__dict__)
     return mod
 
 
