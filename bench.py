@@ -161,8 +161,10 @@ def kernel_bytes(name: str, cfg) -> float:
         return BH * ((F * U + L) * (2 * d * esz + 4) + 2 * NS * dd4)
     if name == "solve_simt":
         return BH * (4 * NS * dd4 + F * d * 4)
-    if name == "solve_tc" and inject_in_scan(cfg):  # A read, P's hi/lo images written; B, C of the text slot
-        return BH * (NS * dd4 + F * dd4 + 2 * dd4)
+    if name == "solve_tc" and inject_in_scan(cfg):  # the text grid: A and B read, C = S_T written
+        return BH * 3 * dd4
+    if name == "solve_tc_frames":  # the frame grid: A read, P's hi/lo images written
+        return BH * F * 2 * dd4
     if name in ("solve_tc", "solve_chol_tc"):  # A, B, alpha read; C (fp32) and M's hi/lo operand images written
         return BH * (3 * NS * dd4 + F * dd4 + F * d * 4)
     if name == "scan_tc":  # per step: a (chunk) map's hi/lo images + its C; S_T; readout states
@@ -198,8 +200,10 @@ def kernel_flops(name: str, cfg) -> float:
     F, NS, J = T - 2, T - 1, cfg.J
     if name.startswith("gram"):
         return B * H * (F * U + L) * 4 * d * d
-    if name == "solve_tc" and inject_in_scan(cfg):  # the inverse d^3 per slot; C = B P for S_T only
-        return B * H * (NS * d ** 3 + 2 * d ** 3)
+    if name == "solve_tc" and inject_in_scan(cfg):  # text grid: the inverse d^3 and C = B P (2 d^3)
+        return B * H * 3 * d ** 3
+    if name == "solve_tc_frames":  # frame grid: the inverse, d^3 per slot
+        return B * H * F * d ** 3
     if name.startswith("solve"):  # Cholesky d^3/3, L^-1 d^3/3, P d^3/3, C = B P 2 d^3
         return B * H * NS * 3 * d ** 3
     if name == "compose_tc":  # two d x d x d products per absorbed frame
@@ -225,12 +229,15 @@ TENSOR_BOUND = ("solve_chol_tc", "solve_simt")
 # separable conv prep takes a 5x5 spatial sum of every input frame and a 5-tap
 # temporal sum per output: (25 T / (T-2) + 5) FMAs per prepared K or V value.
 # Peak: 148 SMs x 128 fp32 lanes x 2 flop per FMA x the SM clock.
-ALU_BOUND = ("solve_tc", "prep_video")
+ALU_BOUND = ("solve_tc", "solve_tc_frames", "prep_video")
 
 
 def kernel_alu_flops(name: str, cfg) -> float:
     if name == "solve_tc":
-        return cfg.B * cfg.H * (cfg.T - 1) * 2 * cfg.d ** 3
+        slots = 1 if inject_in_scan(cfg) else cfg.T - 1  # the text grid alone in the P form
+        return cfg.B * cfg.H * slots * 2 * cfg.d ** 3
+    if name == "solve_tc_frames":
+        return cfg.B * cfg.H * (cfg.T - 2) * 2 * cfg.d ** 3
     if name == "prep_video":
         F = cfg.T - 2
         return cfg.B * cfg.H * 2 * F * cfg.U * cfg.d * 2 * (25 * cfg.T / F + 5)
@@ -268,6 +275,7 @@ def path_flops(cfg) -> float:
 
 def source_digest(kernel: str):
     files = {"gram_tc": "gram_tc.cu", "readout_tc": "readout_tc.cu", "solve_tc": "solve_tc.cu",
+             "solve_tc_frames": "solve_tc.cu", "window_attn_tc": "window_attn_tc.cu", "merge_tc": "merge_tc.cu",
              "scan_tc": "scan_tc.cu", "compose_tc": "compose_tc.cu", "solve_chol_tc": "solve_chol_tc.cu",
              "prep_video": "prep_video.cu"}
     fn = files.get(kernel, "kernels_simt.cu")

@@ -34,7 +34,10 @@ template <int D>
 struct GramCfg {
   static constexpr int kBoxes = D / 64;                     // boxes per operand tile
   static constexpr int kStageBytes = 2 * kBoxes * kBoxBytes;  // K and V token tiles
-  static constexpr int kStages = D == 128 ? 6 : 12;         // HBM reads in flight per SM
+  // HBM reads in flight per SM. At d = 128 five 32 KB stages leave ~32 KB of the
+  // SM's shared memory and ~42k registers free, room for two compact frame-solve
+  // CTAs beside this one.
+  static constexpr int kStages = D == 128 ? 5 : 12;
   static constexpr int kBkSlots = 2;                        // beta*K ring, released by the MMAs
   static constexpr int kBkBytes = kBoxes * kBoxBytes;
   static constexpr int kTmemCols = D == 128 ? 256 : 64;

@@ -129,6 +129,7 @@ enum KernelId {
   K_WINDOW_ATTN_TC,
   K_MERGE_TC,
   K_FRAME_BWD_SIMT,
+  K_SOLVE_TC_FRAMES,
   K_NUM_KERNELS
 };
 const char* kernel_name(int id);
@@ -159,7 +160,9 @@ bool solve_tc_supported(const Problem& p);
 // Raise `func`'s dynamic shared-memory limit to `bytes` on the current device,
 // once per (function, device): the attribute belongs to the device's context.
 cudaError_t set_max_dynamic_smem(const void* func, int bytes);
-cudaError_t launch_solve_tc(const Problem& p, cudaStream_t s);
+// part 0: the text slots (or, unless the P form is used, every slot); part 1:
+// the frame slots of the P form (compact CTAs). Nothing for part 1 otherwise.
+cudaError_t launch_solve_tc(const Problem& p, cudaStream_t s, int part);
 cudaError_t launch_solve_chol_tc(const Problem& p, cudaStream_t s);
 bool scan_tc_supported(const Problem& p);
 cudaError_t launch_scan_tc(const Problem& p, cudaStream_t s, bool chunked);

@@ -43,6 +43,11 @@ constexpr int kPvStride = D + 4;            // floats per pivot buffer (16-byte 
 constexpr int kBarOff = kPvOff + 2 * kPvStride * 4;
 constexpr int kSmemBytes = kBarOff + 64 + 1024;  // + room to align the base to 1024 bytes
 static_assert(3 * (kSmemBytes + 1024) <= 228 * 1024, "three CTAs per SM");
+// A grid of frame slots whose scan forms the injections (P form) needs neither
+// the operand images nor TMEM: only the pivot vectors and the barrier block.
+constexpr int kCompactPvOff = 0;
+constexpr int kCompactBarOff = 2 * kPvStride * 4;
+constexpr int kCompactSmemBytes = kCompactBarOff + 64 + 1024;
 constexpr uint32_t kTmemCols = 128;         // the C accumulator; three CTAs use 384 of 512
 constexpr uint32_t kIdKM = sm100::idesc_bf16_f32(128, 128, false, true);  // A K-major, B MN-major
 
@@ -59,6 +64,8 @@ struct SolveArgs {
   uint32_t* status;
   unsigned long long wait_ns;
   int pform;  // frames write P_t's images and no C_t (the scan forms the injection)
+  int key0;     // key index of this grid's first CTA (0, or B*H for a grid of frame slots)
+  int compact;  // shared memory holds only the pivot vectors and barriers (P-form frame slots)
 };
 
 // Byte offset of element (row, col) in a bf16 image with 128-byte rows of 64
@@ -182,8 +189,8 @@ __global__ void __launch_bounds__(kThreads, 3) solve_tc_kernel(const SolveArgs a
   uint8_t* smem = sm100::align_smem_1024(smem_raw);
   uint8_t* pimg = smem + kPOff;
   uint8_t* bimg = smem + kBOff;
-  float* pv = reinterpret_cast<float*>(smem + kPvOff);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kBarOff);  // [2]: the two halves' MMAs
+  float* pv = reinterpret_cast<float*>(smem + (a.compact ? kCompactPvOff : kPvOff));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + (a.compact ? kCompactBarOff : kBarOff));  // [2]: the two halves' MMAs
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -192,7 +199,7 @@ __global__ void __launch_bounds__(kThreads, 3) solve_tc_kernel(const SolveArgs a
   // scans reach last, and the scans, launched while that wave runs, advance on
   // everything before them.
   int bh, slot;
-  key_slot(blockIdx.x, a.B * a.H, a.T - 1, bh, slot);
+  key_slot(a.key0 + blockIdx.x, a.B * a.H, a.T - 1, bh, slot);
   const long long off = ((long long)bh * (a.T - 1) + slot) * (long long)D * D;
   const bool active = tid < kTiles;
   // C = B P on tcgen05: for every slot, or only for the text slot (S_T) when
@@ -445,18 +452,28 @@ cudaError_t launch_recip_selftest(const float* x, float* y, int n, cudaStream_t 
   return cudaGetLastError();
 }
 
-cudaError_t launch_solve_tc(const Problem& p, cudaStream_t s) {
+cudaError_t launch_solve_tc(const Problem& p, cudaStream_t s, int part) {
   cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void*>(solve_tc_kernel), kSmemBytes);
   if (e != cudaSuccess) return e;
+  const long long BH = (long long)p.B * p.H;
+  // In the P form the solve runs as two grids: the text slots (S_T = B P on
+  // tcgen05, operand images in shared memory), then the frame slots in compact
+  // CTAs (about 2 KB of shared memory, no TMEM) that fit beside the statistics
+  // kernel's CTAs on the same SM and start as soon as their slot's statistics
+  // are stored. Otherwise one grid takes every slot.
+  const bool split = p.pform != 0;
+  const int key0 = (split && part == 1) ? (int)BH : 0;
+  const int compact = (split && part == 1) ? 1 : 0;
+  const long long n = split ? (part == 0 ? BH : BH * (p.T - 2)) : BH * (p.T - 1);
+  if (n == 0) return cudaSuccess;
   SolveArgs a{p.B, p.H, p.T, p.ready, p.gready, p.A, p.Bm, p.alpha, p.M, p.C, static_cast<uint8_t*>(p.Msplit),
-              p.status, p.spin_limit, p.pform};
-  const long long n = (long long)p.B * p.H * (p.T - 1);
-  // After the tensor-core statistics kernel, launch as its programmatic
-  // dependent: CTAs start on the SMs its finished CTAs leave.
+              p.status, p.spin_limit, p.pform, key0, compact};
+  // After the tensor-core statistics kernel (or the text grid), launch as its
+  // programmatic dependent: CTAs start on the SMs its CTAs leave room on.
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3((unsigned)n);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.dynamicSmemBytes = compact ? kCompactSmemBytes : kSmemBytes;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -20,7 +20,7 @@ const char* kernel_name(int id) {
   static const char* names[K_NUM_KERNELS] = {
       "prep_video", "prep_text", "gram_simt", "gram_tc", "solve_simt",
       "scan_simt", "readout_simt", "readout_tc", "zero_anchors", "solve_tc", "scan_tc", "compose_tc",
-      "solve_chol_tc", "window_attn_tc", "merge_tc", "frame_bwd_simt"};
+      "solve_chol_tc", "window_attn_tc", "merge_tc", "frame_bwd_simt", "solve_tc_frames"};
   return (id >= 0 && id < K_NUM_KERNELS) ? names[id] : "?";
 }
 
@@ -404,7 +404,9 @@ vda_status vda_prepare(vda_ctx* ctx, const void* Q, const void* K, const void* V
   else if (sweep_tc) {
     p.ready = p.status + 64;
     p.pform = pform_of(c, p) ? 1 : 0;
-    st = run_kernel(ctx, K_SOLVE_TC, s, [&] { return launch_solve_tc(p, s); });
+    st = run_kernel(ctx, K_SOLVE_TC, s, [&] { return launch_solve_tc(p, s, 0); });
+    if (st == VDA_OK && p.pform && p.T > 2)
+      st = run_kernel(ctx, K_SOLVE_TC_FRAMES, s, [&] { return launch_solve_tc(p, s, 1); });
   }
   else
     st = run_kernel(ctx, K_SOLVE_SIMT, s, [&] { return launch_solve_simt(p, s); });

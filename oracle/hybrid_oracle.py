@@ -89,13 +89,17 @@ def window_softmax_rows(Q: np.ndarray, K: np.ndarray, V: np.ndarray, T: int, U: 
     d_k = Q.shape[1]
     if scale is None:
         scale = 1.0 / np.sqrt(d_k)
+    rows = np.asarray(list(rows), dtype=np.int64)
     out = np.zeros((len(rows), V.shape[1]))
-    for n, row in enumerate(rows):
-        t = int(row) // U
-        keys = np.concatenate([np.arange(f * U, (f + 1) * U) for f in visible_frames(t, c, T)])
-        logits = (K[keys] @ Q[row]) * scale
-        w = np.exp(logits - logits.max())
-        out[n] = (w / w.sum()) @ V[keys]
+    frames = rows // U
+    for t in np.unique(frames):  # the rows of one frame share their visible keys
+        sel = np.nonzero(frames == t)[0]
+        keys = np.concatenate([np.arange(f * U, (f + 1) * U) for f in visible_frames(int(t), c, T)])
+        logits = (Q[rows[sel]] @ K[keys].T) * scale
+        logits = logits - logits.max(axis=1, keepdims=True)
+        w = np.exp(logits)
+        w = w / w.sum(axis=1, keepdims=True)
+        out[sel] = w @ V[keys]
     return out
 
 

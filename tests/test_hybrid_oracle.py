@@ -152,7 +152,7 @@ MUTATIONS = {
     "anchor_rows_windowed": ("    if t in anchor_frames(T):\n        return list(range(T))\n", ""),
     "scale_one_over_d": ("scale = 1.0 / np.sqrt(d_k)", "scale = 1.0 / d_k"),
     "softmax_over_queries": ("w = w / w.sum(axis=1, keepdims=True)", "w = w / w.sum(axis=0, keepdims=True)"),
-    "rows_keys_of_wrong_frame": ("        t = int(row) // U\n", "        t = int(row) // U + 1\n"),
+    "rows_keys_of_wrong_frame": ("    frames = rows // U\n", "    frames = rows // U + 1\n"),
     "gate_sign": ("return O * (1.0 / (1.0 + np.exp(-g)))", "return O * (1.0 / (1.0 + np.exp(g)))"),
     "merge_drops_linear": ("return Ot_S.reshape(N, -1) @ W_S + Ot_L.reshape(N, -1) @ W_L",
                            "return Ot_S.reshape(N, -1) @ W_S"),
