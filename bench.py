@@ -538,6 +538,10 @@ def run_attention_path(args, cfg, rank, world, local, dist, dev):
     dinp = {k: v.to(dev, non_blocking=True) for k, v in host.items()}
     Wd = {k: W[k].to(dev) for k in ("W_soft", "W_lin")} if hybrid else {}
     ctx = V.VDA(cfg, device=dev)
+    # The linear branch runs on a side stream next to the softmax branch (its
+    # middle kernels are latency-bound and fill the SMs the attention leaves).
+    lin = V.VDA(cfg, device=dev) if hybrid else None
+    side = torch.cuda.Stream(dev) if hybrid else None
     O_soft = ctx.new_output()
     O_lin = ctx.new_output() if hybrid else None
     M = cfg.B * cfg.T * cfg.U
@@ -547,9 +551,11 @@ def run_attention_path(args, cfg, rank, world, local, dist, dev):
 
     def step(d, o_soft, o_lin, y):
         if hybrid:
-            ctx.run(d, o_lin)
+            side.wait_stream(stream)
+            lin.run(d, o_lin, stream=side)
         ctx.window_attention(d["Q"], d["K"], d["V"], d["gate"], o_soft)
         if hybrid:
+            stream.wait_stream(side)
             V.hybrid_merge(o_soft, Wd["W_soft"], o_lin, Wd["W_lin"], y, status=mstat)
 
     for _ in range(args.warmup):
@@ -557,7 +563,7 @@ def run_attention_path(args, cfg, rank, world, local, dist, dev):
     torch.cuda.synchronize(dev)
     if ctx.poll_device_status() != 0:
         raise RuntimeError("device status reported a timeout during warm-up")
-    n0 = ctx.launch_count()
+    n0 = ctx.launch_count() + (lin.launch_count() if hybrid else 0)
     clocks = ClockSampler(local)
     ctx.profile_enable(True)
     barrier(dist)
@@ -574,7 +580,9 @@ def run_attention_path(args, cfg, rank, world, local, dist, dev):
     ms = ev0.elapsed_time(ev1)
     prof = ctx.profile_read()
     ctx.profile_enable(False)
-    launches = ctx.launch_count() - n0 + (args.steps if hybrid else 0)  # + one merge launch per step
+    launches = ctx.launch_count() + (lin.launch_count() if hybrid else 0) - n0 + (args.steps if hybrid else 0)
+    if hybrid and lin.poll_device_status() != 0:
+        raise RuntimeError("device status reported a timeout in the linear branch")
     if ctx.poll_device_status() != 0 or int(mstat[:4].view(torch.int32).item()) != 0:
         raise RuntimeError("device status reported a timeout in the timed region")
     ms_max = max_over_ranks(dist, ms, dev)
@@ -615,6 +623,8 @@ def run_attention_path(args, cfg, rank, world, local, dist, dev):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "vda",
             "config": {"workload": workload_desc(cfg) + ("" if hybrid else ", softmax branch, logit std 1"),
                        "path": args.path, "model_width": n_model if hybrid else None,
+                       "streams": ("linear branch on a side stream beside the softmax kernel; merge after both"
+                                   if hybrid else "one stream"),
                        "l2": "no flush: each step reads > 1 GB of tokens, far above the 126 MB L2"},
             "roofline": {"bound": "tensor", "kernel": "window_attn_tc", "achieved": achieved, "peak": peak,
                          "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
@@ -641,6 +651,74 @@ def run_attention_path(args, cfg, rank, world, local, dist, dev):
     return 0
 
 
+def run_ulysses(args, cfg, rank, world, local, dist, dev):
+    """--shard ulysses: the batch arrives sequence-sharded (rank r holds tokens
+    r n .. (r+1) n - 1 of every head, n = T U / world); one step is the all-to-all
+    of Q, K, V to head shards (every token of this rank's heads), the linear
+    branch on those heads, and the all-to-all of O back to sequence shards. The
+    per-head parameters (alpha, beta, text tokens) are this rank's heads' (they
+    are small; their own exchange is the same operation). Strong scaling."""
+    from frame_level_delta_b200 import vda as V
+    from frame_level_delta_b200.shard import head_partition, heads_to_seq, seq_to_heads
+    full = make_inputs(cfg)
+    N = cfg.T * cfg.U
+    if N % world:
+        raise SystemExit(f"--shard ulysses needs T*U ({N}) divisible by the rank count ({world})")
+    n = N // world
+    parts = head_partition(cfg.H, world)
+    h0, k = parts[rank]
+    seq = {x: full[x][:, rank * n:(rank + 1) * n].contiguous().to(dev) for x in ("Q", "K", "V")}
+    par = {x: full[x][:, :, h0:h0 + k].contiguous().to(dev) for x in ("K_txt", "V_txt")}
+    par.update({x: full[x][:, h0:h0 + k].contiguous().to(dev) for x in ("alpha", "beta", "beta_txt")})
+    lcfg = cfg.with_(H=k)
+    lib = V.VDA(lcfg, device=dev)
+    O = lib.new_output()
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        if world > 1:
+            heads = {x: seq_to_heads(seq[x], parts) for x in ("Q", "K", "V")}
+        else:
+            heads = seq
+        lib.run({**heads, **par}, O)
+        return heads_to_seq(O, parts) if world > 1 else O
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    n0 = lib.launch_count()
+    clocks = ClockSampler(local)
+    barrier(dist)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.stop()
+    barrier(dist)
+    ms_max = max_over_ranks(dist, e0.elapsed_time(e1), dev)
+    if lib.poll_device_status() != 0:
+        raise RuntimeError("device status reported a timeout in the timed region")
+    value = cfg.head_tokens * args.steps / (ms_max / 1e3)
+    xbytes = 4 * cfg.B * n * cfg.H * cfg.d * (2 if cfg.dtype == "bf16" else 4) * (world - 1) / max(world, 1)
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic",
+                "config": {"workload": workload_desc(cfg), "global_batch": cfg.B,
+                           "parallelism": f"ulysses{world}: sequence shards -> all-to-all -> heads {parts} "
+                                          f"-> all-to-all back (NCCL)"},
+                "exchange_bytes_per_rank_per_step": xbytes, "gpu_launches": lib.launch_count() - n0,
+                "clocks": clocks.summary()}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -659,8 +737,9 @@ def main():
     ap.add_argument("--path", default="linear", choices=["linear", "softmax", "hybrid"],
                     help="linear: the VDA linear branch (the headline); softmax: the window + anchor "
                          "softmax branch; hybrid: both branches and the merge")
-    ap.add_argument("--shard", default="batch", choices=["batch", "heads"],
-                    help="N > 1: a batch per rank (weak scaling) or one batch's heads split over the ranks")
+    ap.add_argument("--shard", default="batch", choices=["batch", "heads", "ulysses"],
+                    help="N > 1: a batch per rank (weak scaling), one batch's heads split over the ranks, "
+                         "or sequence-sharded inputs exchanged to head shards and back (all-to-all)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -683,6 +762,8 @@ def main():
     dist = init_ranks(world, dev)
     if args.path != "linear":
         return run_attention_path(args, cfg, rank, world, local, dist, dev)
+    if args.shard == "ulysses":
+        return run_ulysses(args, cfg, rank, world, local, dist, dev)
 
     # Each rank draws its own batch (independent problems), or all draw the one
     # batch whose heads they split.

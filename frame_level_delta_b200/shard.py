@@ -41,3 +41,45 @@ def head_partition(H: int, world: int, weights: Optional[Sequence[float]] = None
         out.append((h0, n))
         h0 += n
     return out
+
+
+def seq_to_heads(x_seq, parts, group=None):
+    """Ulysses exchange, sequence shards to head shards: every rank holds its
+    contiguous token range of all heads, x_seq [B, n, H, d] (the same n on every
+    rank); afterwards each rank holds every token of its own heads,
+    [B, world * n, n_r, d] with (h0_r, n_r) = parts[rank] (uneven splits allowed).
+    One all_to_all_single over the process group (NCCL between GPUs)."""
+    import torch
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    B, n, H, d = x_seq.shape
+    send = torch.cat([x_seq[:, :, h0:h0 + k].reshape(-1) for (h0, k) in parts])
+    n_r = parts[rank][1]
+    recv = torch.empty(world * B * n * n_r * d, dtype=x_seq.dtype, device=x_seq.device)
+    dist.all_to_all_single(recv, send, output_split_sizes=[B * n * n_r * d] * world,
+                           input_split_sizes=[B * n * k * d for (_, k) in parts], group=group)
+    # recv holds, source rank by source rank, [B, n, n_r, d]: token order is rank order.
+    return recv.view(world, B, n, n_r, d).permute(1, 0, 2, 3, 4).reshape(B, world * n, n_r, d)
+
+
+def heads_to_seq(x_heads, parts, group=None):
+    """The inverse exchange: [B, world * n, n_r, d] (every token, this rank's
+    heads) back to [B, n, H, d] (this rank's tokens, every head)."""
+    import torch
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    B, N, n_r, d = x_heads.shape
+    n = N // world
+    H = sum(k for _, k in parts)
+    send = x_heads.view(B, world, n, n_r, d).permute(1, 0, 2, 3, 4).reshape(-1)
+    recv = torch.empty(B * n * H * d, dtype=x_heads.dtype, device=x_heads.device)
+    dist.all_to_all_single(recv, send, output_split_sizes=[B * n * k * d for (_, k) in parts],
+                           input_split_sizes=[B * n * n_r * d] * world, group=group)
+    out = torch.empty(B, n, H, d, dtype=x_heads.dtype, device=x_heads.device)
+    off = 0
+    for (h0, k) in parts:
+        sz = B * n * k * d
+        out[:, :, h0:h0 + k] = recv[off:off + sz].view(B, n, k, d)
+        off += sz
+    return out

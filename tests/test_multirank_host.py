@@ -114,6 +114,57 @@ def _rank_heads(rank, world, port, out_dir):
             json.dump({"parts": [list(p) for p in parts], "equal": bool(np.array_equal(got, whole))}, f)
 
 
+def _rank_ulysses(rank, world, port, out_dir):
+    """Sequence-sharded ranks: each holds a contiguous token range of every head;
+    the Ulysses all-to-all hands each rank every token of its heads (uneven 5:3
+    split), the oracle stands in for the library on CPU, and the inverse exchange
+    brings each rank its tokens of every head back."""
+    sys.path.insert(0, ROOT)
+    _set_env(rank, world, port)
+    import numpy as np
+
+    import bench
+    from frame_level_delta_b200.inputs import CONFIGS, make_inputs
+    from frame_level_delta_b200.shard import head_partition, heads_to_seq, seq_to_heads
+    from oracle.vda_oracle import vda_reference
+
+    r, w, _ = bench.rank_env()
+    dist = bench.init_ranks(w, torch.device("cpu"), timeout_s=60)
+    cfg = CONFIGS["small"].with_(H=5, T=8, grid_h=4, grid_w=4, L=6, d=16, dtype="f32")
+    full = make_inputs(cfg)  # drawn identically on every rank; each keeps only its shard
+    N = cfg.T * cfg.U
+    n = N // w
+    parts = head_partition(cfg.H, w, (5, 3))
+    h0, k = parts[r]
+    mine = {}
+    for name in ("Q", "K", "V"):
+        shard = full[name][:, r * n:(r + 1) * n].contiguous()
+        mine[name] = seq_to_heads(shard, parts)
+    ok_layout = all(torch.equal(mine[x], full[x][:, :, h0:h0 + k]) for x in mine)
+    local = dict(full)
+    local.update(mine)
+    for name in ("K_txt", "V_txt"):
+        local[name] = full[name][:, :, h0:h0 + k].contiguous()
+    for name in ("alpha", "beta", "beta_txt"):
+        local[name] = full[name][:, h0:h0 + k].contiguous()
+    O_heads = torch.from_numpy(vda_reference(local, cfg.with_(H=k), keep=False)["O"])
+    O_seq = heads_to_seq(O_heads, parts)
+    want = vda_reference(full, cfg, keep=False)["O"][:, r * n:(r + 1) * n]
+    dist.destroy_process_group()
+    with open(os.path.join(out_dir, f"ulysses{r}.json"), "w") as f:
+        json.dump({"layout": ok_layout, "equal": bool(np.array_equal(O_seq.numpy(), want)),
+                   "shape": list(O_seq.shape)}, f)
+
+
+def test_two_gloo_ranks_ulysses_exchange_round_trip(tmp_path):
+    world = 2
+    mp.start_processes(_rank_ulysses, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    for r in range(world):
+        d = json.loads((tmp_path / f"ulysses{r}.json").read_text())
+        assert d["layout"] and d["equal"], d
+
+
 def test_two_gloo_ranks_head_slices_reassemble_the_output(tmp_path):
     world = 2
     mp.start_processes(_rank_heads, args=(world, _free_port(), str(tmp_path)), nprocs=world,
