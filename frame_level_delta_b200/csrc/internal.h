@@ -130,6 +130,8 @@ enum KernelId {
   K_MERGE_TC,
   K_FRAME_BWD_SIMT,
   K_SOLVE_TC_FRAMES,
+  K_READOUT_FP8_TC,
+  K_GRAM_FP8_TC,
   K_NUM_KERNELS
 };
 const char* kernel_name(int id);
@@ -174,6 +176,16 @@ cudaError_t launch_readout_tc(const Problem& p, const void* gate, void* O, cudaS
 bool window_attn_tc_supported(const Problem& p);
 cudaError_t launch_window_attn_tc(const Problem& p, const void* Q, const void* K, const void* V, const void* gate,
                                   void* O, cudaStream_t s);
+// Readout from e4m3 queries with per-(token, head) scales (D = 128, no conv
+// prep or gate); Q8 and q_scale advanced to the problem's first head.
+bool readout_fp8_tc_supported(const Problem& p);
+cudaError_t launch_readout_fp8_tc(const Problem& p, const void* Q8, const float* q_scale, void* O, cudaStream_t s);
+// Statistics from e4m3 keys and values with per-(token, head) scales shared by
+// the token's key and value (D = 128): a pre-pass writes each slot's exponent to
+// unit_exp, then the tensor-core kernel writes A, B. Two launches.
+cudaError_t launch_gram_fp8_tc(const Problem& p, const void* K8, const void* V8, const float* kv_scale,
+                               const void* Kt8, const void* Vt8, const float* kvt_scale, int* unit_exp,
+                               cudaStream_t s);
 // Hybrid merge Y = A1 B1^T + A2 B2^T (bf16, K-major rows; Y [M, N] bf16).
 cudaError_t launch_merge_tc(const void* A1, const void* B1, const void* A2, const void* B2, void* Y, int M, int N,
                             int K1, int K2, uint32_t* status, unsigned long long wait_ns, cudaStream_t s);

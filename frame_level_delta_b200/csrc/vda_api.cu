@@ -20,7 +20,8 @@ const char* kernel_name(int id) {
   static const char* names[K_NUM_KERNELS] = {
       "prep_video", "prep_text", "gram_simt", "gram_tc", "solve_simt",
       "scan_simt", "readout_simt", "readout_tc", "zero_anchors", "solve_tc", "scan_tc", "compose_tc",
-      "solve_chol_tc", "window_attn_tc", "merge_tc", "frame_bwd_simt", "solve_tc_frames"};
+      "solve_chol_tc", "window_attn_tc", "merge_tc", "frame_bwd_simt", "solve_tc_frames", "readout_fp8_tc",
+      "gram_fp8_tc"};
   return (id >= 0 && id < K_NUM_KERNELS) ? names[id] : "?";
 }
 
@@ -415,6 +416,81 @@ vda_status vda_prepare(vda_ctx* ctx, const void* Q, const void* K, const void* V
   return VDA_OK;
 }
 
+vda_status vda_prepare_fp8(vda_ctx* ctx, const void* K8, const void* V8, const float* kv_scale, const void* Kt8,
+                           const void* Vt8, const float* kvt_scale, const float* alpha, const float* beta,
+                           const float* beta_txt, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!ctx) return VDA_ERR_INVALID_ARG;
+  ctx->prepared = ctx->scanned = false;
+  const vda_config& c = ctx->cfg;
+  if (!K8 || !V8 || !kv_scale || !Kt8 || !Vt8 || !kvt_scale || !alpha || !beta || !beta_txt || !workspace)
+    return fail(ctx, VDA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (c.d_k != 128 || c.dtype != VDA_BF16 || (c.flags & (VDA_PREP_CONV | VDA_FORCE_SIMT)))
+    return fail(ctx, VDA_ERR_UNSUPPORTED, "the FP8 statistics need d = 128, bf16 outputs and no conv prep");
+  const void* a16[] = {K8, V8, Kt8, Vt8, alpha, beta, beta_txt};
+  for (const void* q : a16)
+    if (!aligned16(q)) return fail(ctx, VDA_ERR_ALIGNMENT, "token tensors, alpha and beta must be 16-byte aligned");
+  if (((uintptr_t)kv_scale & 3) || ((uintptr_t)kvt_scale & 3))
+    return fail(ctx, VDA_ERR_ALIGNMENT, "the scales must be 4-byte aligned");
+  if (((uintptr_t)workspace & 255) != 0) return fail(ctx, VDA_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  const Layout L = make_layout(c);
+  if (workspace_bytes < L.total) return fail(ctx, VDA_ERR_WORKSPACE_TOO_SMALL, "workspace smaller than vda_workspace_size()");
+  char* ws = static_cast<char*>(workspace);
+  Problem& p = ctx->p;
+  p = Problem{};
+  p.B = c.B; p.H = c.H; p.T = c.T; p.U = c.U; p.L = c.L; p.D = c.d_k; p.c = c.chunk; p.J = J_of(c);
+  p.gh = c.grid_h; p.gw = c.grid_w; p.Ht = heads_total(c);
+  p.bf16 = 1;
+  p.flags = c.flags;
+  p.l2_eps = c.l2_eps;
+  p.rms_eps = c.rms_eps;
+  p.alpha = alpha; p.beta = beta; p.beta_txt = beta_txt; p.Q = nullptr;
+  p.status = reinterpret_cast<uint32_t*>(ws + L.off[VDA_REGION_STATUS]);
+  p.A = reinterpret_cast<float*>(ws + L.off[VDA_REGION_A]);
+  p.Bm = reinterpret_cast<float*>(ws + L.off[VDA_REGION_B]);
+  p.M = reinterpret_cast<float*>(ws + L.off[VDA_REGION_M]);
+  p.C = reinterpret_cast<float*>(ws + L.off[VDA_REGION_C]);
+  p.Sf = reinterpret_cast<float*>(ws + L.off[VDA_REGION_S_FWD]);
+  p.Sr = reinterpret_cast<float*>(ws + L.off[VDA_REGION_S_REV]);
+  p.Msplit = ws + L.off[VDA_REGION_M_SPLIT];
+  p.CMi = ws + L.off[VDA_REGION_CHUNK_M];
+  p.CC = reinterpret_cast<float*>(ws + L.off[VDA_REGION_CHUNK_C]);
+  p.spin_limit = 2000000000ull;
+  // One byte per channel: advance the e4m3 tensors to head h0 by h0 * d bytes,
+  // the scales by h0 floats.
+  const size_t hb = (size_t)c.h0 * c.d_k;
+  K8 = static_cast<const char*>(K8) + hb;
+  V8 = static_cast<const char*>(V8) + hb;
+  Kt8 = static_cast<const char*>(Kt8) + hb;
+  Vt8 = static_cast<const char*>(Vt8) + hb;
+  kv_scale += c.h0;
+  kvt_scale += c.h0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(p.status, 0, L.bytes[VDA_REGION_STATUS], s);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "status reset");
+  const bool sweep_tc = solve_tc_supported(p) && !(c.flags & VDA_SOLVE_CHOLESKY);
+  const size_t words = align_up((size_t)p.B * p.H * (p.T - 1) * 4, 256) / 4;
+  if (sweep_tc) p.gready = p.status + 64 + words;
+  // The slot exponents live in the M region (the tensor-core solves do not use it).
+  int* exps = reinterpret_cast<int*>(p.M);
+  vda_status st = run_kernel(ctx, K_GRAM_FP8_TC, s, [&] {
+    return launch_gram_fp8_tc(p, K8, V8, kv_scale, Kt8, Vt8, kvt_scale, exps, s);
+  });
+  if (st != VDA_OK) return st;
+  ctx->launches += 1;  // the exponent pre-pass
+  if (c.flags & VDA_SOLVE_CHOLESKY)
+    st = run_kernel(ctx, K_SOLVE_CHOL_TC, s, [&] { return launch_solve_chol_tc(p, s); });
+  else {
+    p.ready = p.status + 64;
+    p.pform = pform_of(c, p) ? 1 : 0;
+    st = run_kernel(ctx, K_SOLVE_TC, s, [&] { return launch_solve_tc(p, s, 0); });
+    if (st == VDA_OK && p.pform && p.T > 2)
+      st = run_kernel(ctx, K_SOLVE_TC_FRAMES, s, [&] { return launch_solve_tc(p, s, 1); });
+  }
+  if (st != VDA_OK) return st;
+  ctx->prepared = true;
+  return VDA_OK;
+}
+
 vda_status vda_scan_bidir(vda_ctx* ctx, void* stream) {
   if (!ctx) return VDA_ERR_INVALID_ARG;
   if (!ctx->prepared) return fail(ctx, VDA_ERR_STATE, "vda_scan_bidir before a successful vda_prepare");
@@ -454,6 +530,22 @@ vda_status vda_readout(vda_ctx* ctx, const void* gate, void* O, void* stream) {
   vda_status st = run_kernel(ctx, K_ZERO_ANCHORS, s, [&] { return launch_zero_anchors(p, O, s); });
   if (st != VDA_OK) return st;
   return run_kernel(ctx, K_READOUT_SIMT, s, [&] { return launch_readout_simt(p, gate, O, s); });
+}
+
+vda_status vda_readout_fp8(vda_ctx* ctx, const void* Q8, const float* q_scale, void* O, void* stream) {
+  if (!ctx) return VDA_ERR_INVALID_ARG;
+  if (!ctx->scanned) return fail(ctx, VDA_ERR_STATE, "vda_readout_fp8 before a successful vda_scan_bidir");
+  if (!Q8 || !q_scale || !O) return fail(ctx, VDA_ERR_INVALID_ARG, "a required pointer is NULL");
+  if (!aligned16(Q8) || !aligned16(O) || ((uintptr_t)q_scale & 3) != 0)
+    return fail(ctx, VDA_ERR_ALIGNMENT, "Q8 and O must be 16-byte aligned, q_scale 4-byte aligned");
+  const vda_config& c = ctx->cfg;
+  if (use_simt_only(c) || !readout_fp8_tc_supported(ctx->p) || c.dtype != VDA_BF16)
+    return fail(ctx, VDA_ERR_UNSUPPORTED, "the FP8 readout needs d = 128, bf16 output and no conv prep or gate");
+  const char* q8 = static_cast<const char*>(Q8) + (size_t)c.h0 * c.d_k;  // one byte per channel
+  const float* qs = q_scale + c.h0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return run_kernel(ctx, K_READOUT_FP8_TC, s,
+                    [&] { return launch_readout_fp8_tc(ctx->p, q8, qs, head_slice(c, O), s); });
 }
 
 vda_status vda_poll_device_status(vda_ctx* ctx, void* stream) {

@@ -204,3 +204,46 @@ def make_backward_inputs(cfg: VDAConfig, seed: Optional[int] = None) -> Dict[str
     shape = (cfg.B, cfg.H, cfg.T, cfg.d, cfg.d)
     return {"S_prev": torch.randn(*shape, generator=g).contiguous(),
             "dS": torch.randn(*shape, generator=g).contiguous()}
+
+
+def quantize_e4m3(x: torch.Tensor):
+    """Per-row e4m3 quantisation of [..., d] values: scale = max|row| / 448 (1 for
+    an all-zero row), x8 = round-to-nearest e4m3 of x / scale. Returns (x8, scale
+    [...] float32); x8 * scale is what a consumer of the FP8 form sees. A storage
+    format of the inputs, not part of the method."""
+    xf = x.float()
+    amax = xf.abs().amax(dim=-1)
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    x8 = (xf / scale.unsqueeze(-1)).to(torch.float8_e4m3fn)
+    return x8.contiguous(), scale.contiguous()
+
+
+def quantize_e4m3_pair(k: torch.Tensor, v: torch.Tensor):
+    """e4m3 form of a key and a value sharing one scale per row:
+    scale = max(max|k_row|, max|v_row|) / 448. Returns (k8, v8, scale)."""
+    kf, vf = k.float(), v.float()
+    amax = torch.maximum(kf.abs().amax(dim=-1), vf.abs().amax(dim=-1))
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    s = scale.unsqueeze(-1)
+    return ((kf / s).to(torch.float8_e4m3fn).contiguous(), (vf / s).to(torch.float8_e4m3fn).contiguous(),
+            scale.contiguous())
+
+
+def make_fp8_inputs(cfg: VDAConfig, seed: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """The FP8 storage form of make_inputs(cfg): Q8 with q_scale (per token and
+    head), K8 and V8 sharing kv_scale, Kt8 and Vt8 sharing kvt_scale; alpha,
+    beta, beta_txt as drawn by make_inputs. Also returns the exact stored values
+    in float64 under Q, K, V, K_txt, V_txt (scale times e4m3 value), for the
+    oracle."""
+    inp = make_inputs(cfg, seed)
+    Q8, qs = quantize_e4m3(inp["Q"])
+    K8, V8, kvs = quantize_e4m3_pair(inp["K"], inp["V"])
+    Kt8, Vt8, kvts = quantize_e4m3_pair(inp["K_txt"], inp["V_txt"])
+    out = {"Q8": Q8, "q_scale": qs, "K8": K8, "V8": V8, "kv_scale": kvs, "Kt8": Kt8, "Vt8": Vt8,
+           "kvt_scale": kvts, "alpha": inp["alpha"], "beta": inp["beta"], "beta_txt": inp["beta_txt"]}
+    out["Q"] = Q8.double() * qs.double().unsqueeze(-1)
+    out["K"] = K8.double() * kvs.double().unsqueeze(-1)
+    out["V"] = V8.double() * kvs.double().unsqueeze(-1)
+    out["K_txt"] = Kt8.double() * kvts.double().unsqueeze(-1)
+    out["V_txt"] = Vt8.double() * kvts.double().unsqueeze(-1)
+    return out

@@ -31,7 +31,8 @@ REGIONS = {"status": 0, "A": 1, "B": 2, "M": 3, "C": 4, "S_fwd": 5, "S_rev": 6,
 
 # Exported symbols, in the order include/vda.h declares them.
 EXPORTS = ["vda_create", "vda_destroy", "vda_workspace_size", "vda_prepare", "vda_scan_bidir",
-           "vda_readout", "vda_poll_device_status", "vda_window_attention", "vda_frame_solve_backward",
+           "vda_readout", "vda_prepare_fp8", "vda_readout_fp8", "vda_poll_device_status", "vda_window_attention",
+           "vda_frame_solve_backward",
            "vda_hybrid_merge",
            "vda_workspace_region", "vda_status_string",
            "vda_last_error", "vda_profile_enable", "vda_num_kernels", "vda_profile_read",
@@ -76,6 +77,8 @@ def lib() -> ctypes.CDLL:
         L.vda_poll_device_status.argtypes = [vp, vp]
         L.vda_window_attention.argtypes = [vp] * 7 + [sz, vp]
         L.vda_hybrid_merge.argtypes = [vp] * 5 + [i, i, i, vp, sz, vp]
+        L.vda_readout_fp8.argtypes = [vp] * 5
+        L.vda_prepare_fp8.argtypes = [vp] * 11 + [sz, vp]
         L.vda_frame_solve_backward.argtypes = [vp] * 13 + [sz, vp]
         L.vda_workspace_region.argtypes = [cfgp, i, ctypes.POINTER(sz), ctypes.POINTER(sz)]
         L.vda_status_string.argtypes = [st]
@@ -280,6 +283,45 @@ class VDA:
         self.check_output(O, gate)
         with self._on_device():
             self._check(lib().vda_readout(self._ctx, _ptr(gate), _ptr(O), _stream_handle(stream)), "vda_readout")
+
+    def prepare_fp8(self, inp8: Dict[str, torch.Tensor], stream=None):
+        """Statistics and solve from e4m3 keys and values (vda_prepare_fp8). inp8
+        holds K8, V8 [B, T*U, H, d] and Kt8, Vt8 [B, L, H, d] (float8_e4m3fn),
+        kv_scale [B, T*U, H], kvt_scale [B, L, H] (float32), and alpha, beta,
+        beta_txt as for prepare."""
+        cfg = self.cfg
+        f8, f32 = torch.float8_e4m3fn, torch.float32
+        B, H, T, U, L, d = cfg.B, cfg.H, cfg.T, cfg.U, cfg.L, cfg.d
+        spec = {"K8": ((B, T * U, H, d), f8), "V8": ((B, T * U, H, d), f8), "Kt8": ((B, L, H, d), f8),
+                "Vt8": ((B, L, H, d), f8), "kv_scale": ((B, T * U, H), f32), "kvt_scale": ((B, L, H), f32),
+                "alpha": ((B, H, T, d), f32), "beta": ((B, H, T, U), f32), "beta_txt": ((B, H, L), f32)}
+        for name, (shape, dt) in spec.items():
+            if name not in inp8:
+                raise ValueError(f"missing input {name}")
+            self._expect(name, inp8[name], shape, dt)
+        par = self._head_params(inp8)
+        ws = self.ensure_workspace()
+        self._keep = (inp8, par)
+        with self._on_device():
+            self._check(lib().vda_prepare_fp8(
+                self._ctx, _ptr(inp8["K8"]), _ptr(inp8["V8"]), _ptr(inp8["kv_scale"]), _ptr(inp8["Kt8"]),
+                _ptr(inp8["Vt8"]), _ptr(inp8["kvt_scale"]), _ptr(par["alpha"]), _ptr(par["beta"]),
+                _ptr(par["beta_txt"]), _ptr(ws), ws.numel(), _stream_handle(stream)), "vda_prepare_fp8")
+
+    def readout_fp8(self, Q8: torch.Tensor, q_scale: torch.Tensor, O: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+        """The readout from e4m3 queries with per-(token, head) float32 scales
+        (vda_readout_fp8), after prepare and scan_bidir."""
+        cfg = self.cfg
+        self._expect("Q8", Q8, (cfg.B, cfg.T * cfg.U, cfg.H, cfg.d), torch.float8_e4m3fn)
+        self._expect("q_scale", q_scale, (cfg.B, cfg.T * cfg.U, cfg.H), torch.float32)
+        if O is None:
+            O = self.new_output()
+        self._expect("O", O, (cfg.B, cfg.T * cfg.U, cfg.H, cfg.d), torch.bfloat16)
+        with self._on_device():
+            self._check(lib().vda_readout_fp8(self._ctx, _ptr(Q8), _ptr(q_scale), _ptr(O), _stream_handle(stream)),
+                        "vda_readout_fp8")
+        return O
 
     def new_output(self) -> torch.Tensor:
         cfg = self.cfg

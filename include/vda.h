@@ -170,6 +170,44 @@ vda_status vda_scan_bidir(vda_ctx* ctx, void* stream);
 vda_status vda_readout(vda_ctx* ctx, const void* gate, void* O, void* stream);
 
 /*
+ * Stage 1 with FP8 keys and values (NEXT to vda_readout_fp8 in the FP8 form of
+ * the path): the frame statistics and the frame solve of vda_prepare, from keys
+ * and values stored as e4m3 with one float32 scale per (token, head) shared by
+ * the token's key and value, k = s K8, v = s V8, read at one byte per channel
+ * (Video DeltaNet summary, section "assumptions and limits": FP8 / MXFP8 for the
+ * large products). The write operand beta s^2 K8 enters the tensor cores as two
+ * e4m3 parts under a power-of-two scale per (b, h, slot) (about 2^-8 relative).
+ *   K8, V8          [B, T*U, H_total, d] e4m3      kv_scale   [B, T*U, H_total] float32
+ *   Kt8, Vt8        [B, L, H_total, d] e4m3        kvt_scale  [B, L, H_total] float32
+ *   alpha, beta, beta_txt, workspace: as for vda_prepare.
+ * Needs d = 128, bf16 storage of the other tensors, no VDA_PREP_CONV or
+ * VDA_FORCE_SIMT (else VDA_ERR_UNSUPPORTED). Then vda_scan_bidir and vda_readout
+ * or vda_readout_fp8 as after vda_prepare (vda_readout needs the bf16 Q; this
+ * call has none, so use vda_readout_fp8).
+ */
+vda_status vda_prepare_fp8(vda_ctx* ctx, const void* K8, const void* V8, const float* kv_scale, const void* Kt8,
+                           const void* Vt8, const float* kvt_scale, const float* alpha, const float* beta,
+                           const float* beta_txt, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Stage 3 with FP8 queries (the pages run their large products in FP8 / MXFP8:
+ * Video DeltaNet summary, section "assumptions and limits"; VDN-H3 post, section
+ * "compared with existing methods"): the readout of vda_readout for queries
+ * given as e4m3 values with one float32 scale per (token, head),
+ * q = q_scale * Q8, read at one byte per channel.
+ *   Q8       [B, T*U, H_total, d] e4m3 (OCP FP8, 4 exponent and 3 mantissa bits)
+ *   q_scale  [B, T*U, H_total] float32
+ *   O        [B, T*U, H_total, d_v] bf16; anchor frames written as zeros
+ * The gathered state S->_j + S<-_j enters the tensor cores as two e4m3 parts
+ * under a power-of-two scale per (b, h, chunk) (about 2^-8 relative), products
+ * accumulate in fp32. Needs d = 128, bf16 storage, and neither VDA_PREP_CONV nor
+ * VDA_READOUT_NORM_GATE (else VDA_ERR_UNSUPPORTED); VDA_ERR_STATE unless
+ * vda_scan_bidir succeeded after the last vda_prepare. The Q given to
+ * vda_prepare is not read by this call.
+ */
+vda_status vda_readout_fp8(vda_ctx* ctx, const void* Q8, const float* q_scale, void* O, void* stream);
+
+/*
  * Synchronise `stream`, read the device status words of the last vda_prepare
  * workspace and of the last vda_window_attention workspace, clear them and return
  * VDA_ERR_TIMEOUT if a bounded device-side wait gave up since the last poll,
