@@ -130,6 +130,9 @@ def whole_job_rate(world: int, cfg, steps: int, ms_max: float, shard: str = "bat
 SCAN_CHUNKED = False
 # Whether the Cholesky solve is selected (VDA_SOLVE_CHOLESKY); set from --solve.
 SOLVE_CHOLESKY = False
+# Whether the path runs from e4m3 keys, values and queries (--fp8).
+FP8 = False
+FP8_KEYS = ("Q8", "q_scale", "K8", "V8", "kv_scale", "Kt8", "Vt8", "kvt_scale", "alpha", "beta", "beta_txt")
 
 
 def inject_in_scan(cfg) -> bool:
@@ -159,6 +162,10 @@ def kernel_bytes(name: str, cfg) -> float:
     dd4 = d * d * 4
     if name in ("gram_tc", "gram_simt"):
         return BH * ((F * U + L) * (2 * d * esz + 4) + 2 * NS * dd4)
+    if name == "gram_fp8_tc":  # e4m3 K, V (one byte per channel), beta, the shared scale; A, B out
+        return BH * ((F * U + L) * (2 * d + 4 + 4) + 2 * NS * dd4)
+    if name == "readout_fp8_tc":  # e4m3 Q and its scale in, bf16 O out, the states, anchor zeros
+        return BH * (F * U * (d + 4 + 2 * d) + 2 * J * dd4 + 2 * U * d * 2)
     if name == "solve_simt":
         return BH * (4 * NS * dd4 + F * d * 4)
     if name == "solve_tc" and inject_in_scan(cfg):  # the text grid: A and B read, C = S_T written
@@ -200,6 +207,8 @@ def kernel_flops(name: str, cfg) -> float:
     F, NS, J = T - 2, T - 1, cfg.J
     if name.startswith("gram"):
         return B * H * (F * U + L) * 4 * d * d
+    if name == "readout_fp8_tc":
+        return B * H * F * U * 2 * d * d
     if name == "solve_tc" and inject_in_scan(cfg):  # text grid: the inverse d^3 and C = B P (2 d^3)
         return B * H * 3 * d ** 3
     if name == "solve_tc_frames":  # frame grid: the inverse, d^3 per slot
@@ -256,6 +265,8 @@ def path_bytes(cfg) -> float:
     esz = 4 if cfg.dtype == "f32" else 2
     F = T - 2
     per_head = F * U * (4 * d * esz + 4) + L * (2 * d * esz + 4) + F * d * 4 + 2 * U * d * esz
+    if FP8:  # Q8, K8, V8 at one byte per channel with their scales; O in bf16
+        per_head = F * U * (3 * d + 2 * d + 4 + 4 + 4) + L * (2 * d + 4 + 4) + F * d * 4 + 2 * U * d * 2
     if cfg.prep_conv:
         per_head += 2 * 2 * U * d * esz + F * U * d * esz  # anchor-frame K, V for the conv; gate
     return B * H * per_head
@@ -275,6 +286,7 @@ def path_flops(cfg) -> float:
 
 def source_digest(kernel: str):
     files = {"gram_tc": "gram_tc.cu", "readout_tc": "readout_tc.cu", "solve_tc": "solve_tc.cu",
+             "gram_fp8_tc": "gram_fp8_tc.cu", "readout_fp8_tc": "readout_fp8_tc.cu",
              "solve_tc_frames": "solve_tc.cu", "window_attn_tc": "window_attn_tc.cu", "merge_tc": "merge_tc.cu",
              "scan_tc": "scan_tc.cu", "compose_tc": "compose_tc.cu", "solve_chol_tc": "solve_chol_tc.cu",
              "prep_video": "prep_video.cu"}
@@ -651,6 +663,111 @@ def run_attention_path(args, cfg, rank, world, local, dist, dev):
     return 0
 
 
+def backward_flops(cfg) -> dict:
+    """Per launch: the statistics (4 d^2 flops per token), the per-frame adjoints
+    (the sweep's d^3 FMAs and three d x d x d products, S_t, Gx and GA, at 2 d^3
+    flops each) and the per-token products (three d x d matrix-vector products,
+    6 d^2 flops per token)."""
+    B, H, d, T, U, L = cfg.B, cfg.H, cfg.d, cfg.T, cfg.U, cfg.L
+    F = T - 2
+    return {"gram": B * H * (F * U + L) * 4 * d * d,
+            "frame": B * H * F * (2 * d ** 3 + 3 * 2 * d ** 3),
+            "token": B * H * F * U * 6 * d * d}
+
+
+def backward_bytes(cfg) -> float:
+    """K, V, beta read and dK, dV, dbeta written per token; S_prev, dS read and
+    dS_prev written per frame; alpha and dalpha."""
+    B, H, d, T, U = cfg.B, cfg.H, cfg.d, cfg.T, cfg.U
+    esz = 4 if cfg.dtype == "f32" else 2
+    F = T - 2
+    return B * H * F * (U * (4 * d * esz + 8) + 3 * d * d * 4 + 2 * d * 4)
+
+
+def run_backward_path(args, cfg, rank, world, local, dist, dev):
+    """--path backward: one step = vda_frame_solve_backward over every head and
+    frame of one batch (the statistics recomputed, the per-frame adjoints, the
+    per-token gradients)."""
+    from frame_level_delta_b200 import vda as V
+    from frame_level_delta_b200.inputs import make_backward_inputs
+    inp = {k: v.to(dev) for k, v in make_inputs(cfg, seed=rank_seed(cfg, rank)).items()}
+    bw = {k: v.to(dev) for k, v in make_backward_inputs(cfg, seed=rank_seed(cfg, rank)).items()}
+    ctx = V.VDA(cfg, device=dev)
+    out = None
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return ctx.frame_solve_backward(inp["K"], inp["V"], inp["alpha"], inp["beta"], bw["S_prev"], bw["dS"],
+                                        out=out)
+
+    out = step()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    n0 = ctx.launch_count()
+    ctx.profile_enable(True)
+    clocks = ClockSampler(local)
+    barrier(dist)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.stop()
+    barrier(dist)
+    ms_max = max_over_ranks(dist, e0.elapsed_time(e1), dev)
+    prof = ctx.profile_read()
+    ctx.profile_enable(False)
+    if ctx.poll_device_status() != 0:
+        raise RuntimeError("device status reported a timeout in the timed region")
+    launches = ctx.launch_count() - n0 + args.steps  # frame_bwd_simt is two launches per step
+    value = whole_job_rate(world, cfg, args.steps, ms_max)
+    fl = backward_flops(cfg)
+    bn, bms = prof["frame_bwd_simt"]
+    b_s = bms / bn / 1e3
+    sm_mhz = float(clocks.summary().get("sm_mhz") or 1965.0)
+    peak = alu_peak_tflops(sm_mhz)
+    achieved = (fl["frame"] + fl["token"]) / b_s / 1e12
+    if rank == 0:
+        line = {"metric": "frame-step backward head-tokens/s (dK, dV, dbeta, dalpha, dS_prev)", "value": value,
+                "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic", "impl": "vda",
+                "config": {"workload": workload_desc(cfg), "path": "backward"},
+                "roofline": {"bound": "alu", "kernel": "frame_bwd_simt", "achieved": achieved, "peak": peak,
+                             "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                             "peak_source": f"fp32 FMA peak derived: 148 SMs x 128 lanes x 2 flop x {sm_mhz:.0f} MHz",
+                             "algorithmic_flops_per_launch": fl["frame"] + fl["token"],
+                             "algorithmic_bytes_per_launch": backward_bytes(cfg)},
+                "kernels": {k: {"launches": n, "avg_us": tot / n * 1e3} for k, (n, tot) in prof.items()},
+                "gpu_launches": launches, "clocks": clocks.summary()}
+        if world == 1 and args.cpu_budget > 0:
+            from oracle.vda_oracle import frame_step_backward
+            n, t0 = 0, time.perf_counter()
+            U = cfg.U
+            while time.perf_counter() - t0 < args.cpu_budget:
+                h, t = n % cfg.H, 1 + (n // cfg.H) % (cfg.T - 2)
+                frame_step_backward(bw["S_prev"][0, h, t].double().cpu().numpy(),
+                                    inp["K"][0, t * U:(t + 1) * U, h].double().cpu().numpy(),
+                                    inp["V"][0, t * U:(t + 1) * U, h].double().cpu().numpy(),
+                                    inp["beta"][0, h, t].double().cpu().numpy(),
+                                    inp["alpha"][0, h, t].double().cpu().numpy(),
+                                    bw["dS"][0, h, t].double().cpu().numpy())
+                n += 1
+            dt = time.perf_counter() - t0
+            line["cpu_baseline"] = {"value": n * U / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                                    "blas": blas_library(),
+                                    "sample": f"float64 oracle frame_step_backward on {n} (head, frame) pairs, "
+                                              f"{dt:.2f} s"}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
 def run_ulysses(args, cfg, rank, world, local, dist, dev):
     """--shard ulysses: the batch arrives sequence-sharded (rank r holds tokens
     r n .. (r+1) n - 1 of every head, n = T U / world); one step is the all-to-all
@@ -734,9 +851,11 @@ def main():
                     help="tensor-core scan frame by frame (default) or over composed chunk maps")
     ap.add_argument("--heads", type=int, default=0,
                     help="override H (a smaller case of the same workload, e.g. for profiler captures)")
-    ap.add_argument("--path", default="linear", choices=["linear", "softmax", "hybrid"],
+    ap.add_argument("--path", default="linear", choices=["linear", "softmax", "hybrid", "backward"],
                     help="linear: the VDA linear branch (the headline); softmax: the window + anchor "
                          "softmax branch; hybrid: both branches and the merge")
+    ap.add_argument("--fp8", action="store_true",
+                    help="linear path from e4m3 keys, values and queries with per-token scales")
     ap.add_argument("--shard", default="batch", choices=["batch", "heads", "ulysses"],
                     help="N > 1: a batch per rank (weak scaling), one batch's heads split over the ranks, "
                          "or sequence-sharded inputs exchanged to head shards and back (all-to-all)")
@@ -760,6 +879,8 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     dist = init_ranks(world, dev)
+    if args.path == "backward":
+        return run_backward_path(args, cfg, rank, world, local, dist, dev)
     if args.path != "linear":
         return run_attention_path(args, cfg, rank, world, local, dist, dev)
     if args.shard == "ulysses":
@@ -767,7 +888,12 @@ def main():
 
     # Each rank draws its own batch (independent problems), or all draw the one
     # batch whose heads they split.
-    inp_cpu = make_inputs(cfg, seed=rank_seed(cfg, rank, args.shard))
+    if args.fp8:
+        from frame_level_delta_b200.inputs import make_fp8_inputs
+        x8 = make_fp8_inputs(cfg, seed=rank_seed(cfg, rank, args.shard))
+        inp_cpu = {k: x8[k] for k in FP8_KEYS}
+    else:
+        inp_cpu = make_inputs(cfg, seed=rank_seed(cfg, rank, args.shard))
     heads = None
     if args.shard == "heads" and world > 1:
         from frame_level_delta_b200.shard import head_partition
@@ -782,6 +908,17 @@ def main():
     kcfg = cfg if heads is None else cfg.with_(H=heads[1])
     O = lib.new_output()
     stream = torch.cuda.current_stream(dev)
+    if args.fp8:
+        global FP8
+        FP8 = True
+
+        def run_fp8(inp, out, stream=None):
+            lib.prepare_fp8(inp, stream=stream)
+            lib.scan_bidir(stream=stream)
+            lib.readout_fp8(inp["Q8"], inp["q_scale"], out, stream=stream)
+            return out
+
+        lib.run = run_fp8  # every step below goes through the FP8 entry points
     for _ in range(args.warmup):
         lib.run(inp_dev, O)
     torch.cuda.synchronize(dev)
@@ -915,7 +1052,9 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-            "scaling": "weak" if args.shard == "batch" else "strong", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32",
+            "scaling": "weak" if args.shard == "batch" else "strong", "vs_baseline": None,
+            "dtype": ("e4m3 operands, fp32 accumulation and state, bf16 O" if FP8 else
+                      "bf16" if cfg.dtype == "bf16" else "f32"),
             "data": "synthetic",
             "config": {"workload": workload_desc(cfg), "global_batch": cfg.B * (world if args.shard == "batch" else 1),
                        "parallelism": (f"dp{world} (independent batches, no collective)" if args.shard == "batch"
@@ -945,7 +1084,7 @@ def main():
                     "steps": ke},
         }
         if world == 1 and args.cpu_budget > 0:
-            line["cpu_baseline"] = cpu_baseline(cfg, inp_cpu, budget_s=args.cpu_budget)
+            line["cpu_baseline"] = cpu_baseline(cfg, x8 if args.fp8 else inp_cpu, budget_s=args.cpu_budget)
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()

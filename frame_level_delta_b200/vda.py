@@ -365,10 +365,11 @@ class VDA:
         return O
 
     def frame_solve_backward(self, K: torch.Tensor, V: torch.Tensor, alpha: torch.Tensor, beta: torch.Tensor,
-                             S_prev: torch.Tensor, dS: torch.Tensor, stream=None) -> Dict[str, torch.Tensor]:
+                             S_prev: torch.Tensor, dS: torch.Tensor, stream=None,
+                             out: Optional[Dict[str, torch.Tensor]] = None) -> Dict[str, torch.Tensor]:
         """Backward of the frame step for frames 1..T-2 (vda_frame_solve_backward).
         Returns dK, dV (storage dtype) and dS_prev, dalpha, dbeta (float32), zero
-        on the anchor frames."""
+        on the anchor frames (``out``, from an earlier call, is written again)."""
         cfg = self.cfg
         sd = torch.float32 if cfg.dtype == "f32" else torch.bfloat16
         B, H, T, U, d = cfg.B, self.c.H, cfg.T, cfg.U, cfg.d
@@ -381,9 +382,11 @@ class VDA:
         self._expect("beta", p["beta"], (B, H, T, U), torch.float32)
         self._expect("S_prev", S_prev, (B, H, T, d, d), torch.float32)
         self._expect("dS", dS, (B, H, T, d, d), torch.float32)
-        out = {"dK": torch.zeros(tok, dtype=sd, device=self.device), "dV": torch.zeros(tok, dtype=sd, device=self.device),
-               "dS_prev": torch.zeros_like(S_prev), "dalpha": torch.zeros_like(p["alpha"]),
-               "dbeta": torch.zeros_like(p["beta"])}
+        if out is None:
+            out = {"dK": torch.zeros(tok, dtype=sd, device=self.device),
+                   "dV": torch.zeros(tok, dtype=sd, device=self.device),
+                   "dS_prev": torch.zeros_like(S_prev), "dalpha": torch.zeros_like(p["alpha"]),
+                   "dbeta": torch.zeros_like(p["beta"])}
         ws = self.ensure_workspace()
         with self._on_device():
             self._check(lib().vda_frame_solve_backward(
