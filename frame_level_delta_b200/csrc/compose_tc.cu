@@ -58,15 +58,16 @@ __device__ __forceinline__ uint32_t img_off(int row, int col) {
 }
 
 __device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
-  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&hi);
-  __nv_bfloat162* l = reinterpret_cast<__nv_bfloat162*>(&lo);
+  uint32_t h[4], l[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * q], x[2 * q + 1]);
     const float2 hf = __bfloat1622float2(hh);
-    h[q] = hh;
-    l[q] = __floats2bfloat162_rn(x[2 * q] - hf.x, x[2 * q + 1] - hf.y);
+    h[q] = sm100::bf162_bits(hh);
+    l[q] = sm100::bf162_bits(__floats2bfloat162_rn(x[2 * q] - hf.x, x[2 * q + 1] - hf.y));
   }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
 // 32 consecutive values of a row as 16 hi and 16 lo bf16 pairs (lower column

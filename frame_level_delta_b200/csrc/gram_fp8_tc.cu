@@ -88,7 +88,7 @@ __device__ __forceinline__ uint16_t to_e4m3x2(float lo, float hi) {
 }
 __device__ __forceinline__ float2 from_e4m3x2(uint16_t v) {
   const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)v, __NV_E4M3);
-  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+  return __half22float2(__half2(h));
 }
 
 // Pre-pass: E per (b, h, slot) with 2^E max_u(beta_u s_u^2) 448 <= 240, so every
@@ -275,21 +275,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = c0; c < c0 + 4; ++c) {
           const int pc = c ^ (row & 7);
           const uint4 v = *reinterpret_cast<const uint4*>(src + pc * 16);
-          const uint16_t* e = reinterpret_cast<const uint16_t*>(&v);
-          uint4 hv, lv;
-          uint16_t* hp = reinterpret_cast<uint16_t*>(&hv);
-          uint16_t* lp = reinterpret_cast<uint16_t*>(&lv);
+          const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+          // Pairs unpacked and packed by shifts (no type-punned accesses).
+          uint32_t hw[4], lw[4];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            const float2 f = from_e4m3x2(e[q]);
+            const uint16_t e = (uint16_t)(vw[q >> 1] >> ((q & 1) * 16));
+            const float2 f = from_e4m3x2(e);
             const float r0 = f.x * sc, r1 = f.y * sc;
             const uint16_t hh = to_e4m3x2(r0, r1);
             const float2 hf = from_e4m3x2(hh);
-            hp[q] = hh;
-            lp[q] = to_e4m3x2(r0 - hf.x, r1 - hf.y);
+            const uint16_t ll = to_e4m3x2(r0 - hf.x, r1 - hf.y);
+            if (q & 1) {
+              hw[q >> 1] |= (uint32_t)hh << 16;
+              lw[q >> 1] |= (uint32_t)ll << 16;
+            } else {
+              hw[q >> 1] = hh;
+              lw[q >> 1] = ll;
+            }
           }
-          *reinterpret_cast<uint4*>(dh + pc * 16) = hv;
-          *reinterpret_cast<uint4*>(dl + pc * 16) = lv;
+          *reinterpret_cast<uint4*>(dh + pc * 16) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(dl + pc * 16) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
         fence_proxy_async_smem();
         __syncwarp();

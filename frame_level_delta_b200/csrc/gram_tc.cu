@@ -271,14 +271,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* dst = bkring + bs * C::kBkBytes + box * kBoxBytes + row * 128;
         for (int c = c0; c < c1; ++c) {
           const int pc = c ^ (row & 7);  // any chunk order works; this one avoids bank conflicts
-          uint4 v = *reinterpret_cast<const uint4*>(src + pc * 16);
-          __nv_bfloat162* e = reinterpret_cast<__nv_bfloat162*>(&v);
+          const uint4 v = *reinterpret_cast<const uint4*>(src + pc * 16);
+          uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            float2 f = __bfloat1622float2(e[q]);
-            e[q] = __floats2bfloat162_rn(f.x * bb, f.y * bb);
+            const float2 f = __bfloat1622float2(bits_bf162(w[q]));
+            w[q] = bf162_bits(__floats2bfloat162_rn(f.x * bb, f.y * bb));
           }
-          *reinterpret_cast<uint4*>(dst + pc * 16) = v;
+          *reinterpret_cast<uint4*>(dst + pc * 16) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async_smem();
         __syncwarp();

@@ -47,8 +47,7 @@ struct MergeArgs {
 };
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&v);
+  return sm100::bf162_bits(__floats2bfloat162_rn(a, b));
 }
 
 __global__ void __launch_bounds__(kThreads, 1)

@@ -65,8 +65,8 @@ struct PrepIO<__nv_bfloat16> {
   static __device__ __forceinline__ void store4(__nv_bfloat16* dst, float4 v) {
     __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
     uint2 u;
-    u.x = *reinterpret_cast<uint32_t*>(&a);
-    u.y = *reinterpret_cast<uint32_t*>(&b);
+    u.x = sm100::bf162_bits(a);
+    u.y = sm100::bf162_bits(b);
     *reinterpret_cast<uint2*>(dst) = u;
   }
 };

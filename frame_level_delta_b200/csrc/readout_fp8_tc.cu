@@ -117,12 +117,11 @@ __device__ __forceinline__ uint16_t to_e4m3x2(float lo, float hi) {
 }
 __device__ __forceinline__ float2 from_e4m3x2(uint16_t v) {
   const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)v, __NV_E4M3);
-  return __half22float2(*reinterpret_cast<const __half2*>(&h));
+  return __half22float2(__half2(h));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&v);
+  return sm100::bf162_bits(__floats2bfloat162_rn(a, b));
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -287,16 +286,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             x[4 * q + 2] = (f.z + g.z) * sc;
             x[4 * q + 3] = (f.w + g.w) * sc;
           }
-          uint4 hv, lv;
-          uint16_t* hp = reinterpret_cast<uint16_t*>(&hv);
-          uint16_t* lp = reinterpret_cast<uint16_t*>(&lv);
+          // Pairs packed into 32-bit words by shifts (no type-punned stores).
+          uint32_t hw[4], lw[4];
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const uint16_t hh = to_e4m3x2(x[2 * q], x[2 * q + 1]);
             const float2 hf = from_e4m3x2(hh);
-            hp[q] = hh;
-            lp[q] = to_e4m3x2(x[2 * q] - hf.x, x[2 * q + 1] - hf.y);
+            const uint16_t ll = to_e4m3x2(x[2 * q] - hf.x, x[2 * q + 1] - hf.y);
+            if (q & 1) {
+              hw[q >> 1] |= (uint32_t)hh << 16;
+              lw[q >> 1] |= (uint32_t)ll << 16;
+            } else {
+              hw[q >> 1] = hh;
+              lw[q >> 1] = ll;
+            }
           }
+          const uint4 hv = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          const uint4 lv = make_uint4(lw[0], lw[1], lw[2], lw[3]);
           const int boff = i * 128 + ((c16 ^ (i & 7)) << 4);
           *reinterpret_cast<uint4*>(sHi + boff) = hv;
           *reinterpret_cast<uint4*>(sLo + boff) = lv;

@@ -326,16 +326,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float4 r0 = pr[(2 * c8) * D + i], r1 = pr[(2 * c8 + 1) * D + i];
           x[0] = f0.x + r0.x; x[1] = f0.y + r0.y; x[2] = f0.z + r0.z; x[3] = f0.w + r0.w;
           x[4] = f1.x + r1.x; x[5] = f1.y + r1.y; x[6] = f1.z + r1.z; x[7] = f1.w + r1.w;
-          uint4 hv, lv;
-          __nv_bfloat162* hp = reinterpret_cast<__nv_bfloat162*>(&hv);
-          __nv_bfloat162* lp = reinterpret_cast<__nv_bfloat162*>(&lv);
+          uint32_t hp[4], lp[4];
 #pragma unroll
           for (int k2 = 0; k2 < 4; ++k2) {
             const __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * k2], x[2 * k2 + 1]);
             const float2 hf = __bfloat1622float2(hh);
-            hp[k2] = hh;
-            lp[k2] = __floats2bfloat162_rn(x[2 * k2] - hf.x, x[2 * k2 + 1] - hf.y);
+            hp[k2] = bf162_bits(hh);
+            lp[k2] = bf162_bits(__floats2bfloat162_rn(x[2 * k2] - hf.x, x[2 * k2 + 1] - hf.y));
           }
+          const uint4 hv = make_uint4(hp[0], hp[1], hp[2], hp[3]);
+          const uint4 lv = make_uint4(lp[0], lp[1], lp[2], lp[3]);
           const int atom = c8 / 8, chunk = c8 % 8;
           const int boff = atom * C::kSAtomBytes + i * 128 + ((chunk ^ (i & 7)) * 16);
           *reinterpret_cast<uint4*>(sShi + boff) = hv;
@@ -374,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < kChunks; ++c) {
             const int gc = hf * kChunks + c;  // chunk of the whole row (swizzled order: the sum needs none)
             const uint4 v = *reinterpret_cast<const uint4*>(qrow + (gc / 8) * (kTileM * 128) + (gc % 8) * 16);
-            const __nv_bfloat162* e = reinterpret_cast<const __nv_bfloat162*>(&v);
+            const __nv_bfloat162 e[4] = {bits_bf162(v.x), bits_bf162(v.y), bits_bf162(v.z), bits_bf162(v.w)};
 #pragma unroll
             for (int k2 = 0; k2 < 4; ++k2) {
               const float2 f = __bfloat1622float2(e[k2]);
@@ -441,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float g8[8];
           if constexpr (GATE) {
             const uint4 gv = gr[2 * cc + half];
-            const __nv_bfloat162* ge = reinterpret_cast<const __nv_bfloat162*>(&gv);
+            const __nv_bfloat162 ge[4] = {bits_bf162(gv.x), bits_bf162(gv.y), bits_bf162(gv.z), bits_bf162(gv.w)};
 #pragma unroll
             for (int k2 = 0; k2 < 4; ++k2) {  // rn * sigmoid(g) = hr + hr * tanh(g / 2), hr = rn / 2
               const float2 f = __bfloat1622float2(ge[k2]);
@@ -452,11 +452,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < 8; ++k) g8[k] = 1.f;
           }
-          __nv_bfloat162* op = reinterpret_cast<__nv_bfloat162*>(&outs[2 * cc + half]);
+          uint32_t op[4];
 #pragma unroll
           for (int k2 = 0; k2 < 4; ++k2)
-            op[k2] = __floats2bfloat162_rn(vf[half * 8 + 2 * k2] * scale * g8[2 * k2],
-                                           vf[half * 8 + 2 * k2 + 1] * scale * g8[2 * k2 + 1]);
+            op[k2] = bf162_bits(__floats2bfloat162_rn(vf[half * 8 + 2 * k2] * scale * g8[2 * k2],
+                                                      vf[half * 8 + 2 * k2 + 1] * scale * g8[2 * k2 + 1]));
+          outs[2 * cc + half] = make_uint4(op[0], op[1], op[2], op[3]);
         }
       }
       if constexpr (!GATE) {

@@ -77,17 +77,18 @@ struct ScanArgs {
 };
 
 __device__ __forceinline__ void split8(const float* x, uint4& hi, uint4& lo) {
-  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&hi);
-  __nv_bfloat162* l = reinterpret_cast<__nv_bfloat162*>(&lo);
+  uint32_t h[4], l[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     const __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * q], x[2 * q + 1]);
     const float2 hf = __bfloat1622float2(hh);
-    h[q] = hh;
+    h[q] = sm100::bf162_bits(hh);
     // x - hi is exact in fp32; one packed add for the pair.
     const float2 d = __fadd2_rn(make_float2(x[2 * q], x[2 * q + 1]), make_float2(-hf.x, -hf.y));
-    l[q] = __floats2bfloat162_rn(d.x, d.y);
+    l[q] = sm100::bf162_bits(__floats2bfloat162_rn(d.x, d.y));
   }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
 // 16 consecutive values of a state row as 8 hi and 8 lo bf16 pairs (lower

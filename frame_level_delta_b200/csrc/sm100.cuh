@@ -7,13 +7,28 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <string.h>
 
 #include "../../include/vda.h"
 
 namespace vda {
 namespace sm100 {
+
+// Bit moves between a bf16 pair and a 32-bit word (memcpy, not a type-punned
+// pointer, so the compiler sees every write of the word).
+__device__ __forceinline__ uint32_t bf162_bits(__nv_bfloat162 v) {
+  uint32_t u;
+  memcpy(&u, &v, sizeof(u));
+  return u;
+}
+__device__ __forceinline__ __nv_bfloat162 bits_bf162(uint32_t u) {
+  __nv_bfloat162 v;
+  memcpy(&v, &u, sizeof(v));
+  return v;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

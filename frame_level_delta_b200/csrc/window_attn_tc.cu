@@ -194,8 +194,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&v);
+  return sm100::bf162_bits(__floats2bfloat162_rn(a, b));
 }
 
 template <int D>
@@ -451,7 +450,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           float g8[8];
           if (gsrc) {
             const uint4 gv = gsrc[c4 * 4 + q8];
-            const __nv_bfloat162* ge = reinterpret_cast<const __nv_bfloat162*>(&gv);
+            const __nv_bfloat162 ge[4] = {sm100::bits_bf162(gv.x), sm100::bits_bf162(gv.y), sm100::bits_bf162(gv.z),
+                                          sm100::bits_bf162(gv.w)};
 #pragma unroll
             for (int k2 = 0; k2 < 4; ++k2) {
               const float2 f = __bfloat1622float2(ge[k2]);
@@ -462,13 +462,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < 8; ++k) g8[k] = 1.f;
           }
-          uint4 ov;
-          uint32_t* op = reinterpret_cast<uint32_t*>(&ov);
+          uint32_t op[4];
 #pragma unroll
           for (int k2 = 0; k2 < 4; ++k2)
             op[k2] = pack_bf16(__uint_as_float(v[q8 * 8 + 2 * k2]) * inv * g8[2 * k2],
                                __uint_as_float(v[q8 * 8 + 2 * k2 + 1]) * inv * g8[2 * k2 + 1]);
-          dst[c4 * 4 + q8] = ov;
+          dst[c4 * 4 + q8] = make_uint4(op[0], op[1], op[2], op[3]);
         }
       }
     }
