@@ -14,8 +14,9 @@
 //   acc = Q8 hi^T + Q8 lo^T        (M = 128 tokens, N = d_v, K = d_k, fp32 in TMEM)
 // and the epilogue writes o = s_q 2^-E acc as bf16. Persistent CTAs walk the
 // same (head, token segment) tile lists as the bf16 readout.
-// Warp roles: 0 = TMA producer, 1 = TMEM owner + MMA issuer, 2..5 = prologue
-// and epilogue (one token row per thread).
+// Warp roles: 0 = TMA producer, 1 = TMEM owner + MMA issuer, 2..9 = prologue
+// and epilogue (two warps per TMEM lane quadrant, one per half of the output
+// columns); full tiles leave through a staging tile and TMA stores.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
@@ -31,13 +32,15 @@ namespace {
 
 constexpr int D = 128;
 constexpr int kTileM = 128;
-constexpr int kThreads = 192;
-constexpr int kEpi = 128;
+constexpr int kThreads = 320;  // TMA warp, MMA warp, eight epilogue warps
+constexpr int kEpi = 256;
 constexpr int kStages = 6;
 constexpr int kTileBytes = kTileM * D;  // one e4m3 tile of 128 tokens (16 KB)
 constexpr int kSBytes = D * D;          // one e4m3 image of S (16 KB)
 constexpr int kSHiOff = 0, kSLoOff = kSBytes, kQOff = 2 * kSBytes;
-constexpr int kBarOff = kQOff + kStages * kTileBytes;
+constexpr int kOOff = kQOff + kStages * kTileBytes;  // bf16 output tile staged for the TMA store (32 KB)
+constexpr int kOBox = kTileM * 128;                      // one 64-column box of it
+constexpr int kBarOff = kOOff + 2 * kOBox;
 constexpr int kSmemBytes = kBarOff + 256 + 1024;
 // kind::f8f6f4: D f32, A and B e4m3, both K-major, M = 128, N = 128.
 constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(D >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
@@ -120,18 +123,30 @@ __device__ __forceinline__ float2 from_e4m3x2(uint16_t v) {
   return __half22float2(__half2(h));
 }
 
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(sm100::smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return sm100::bf162_bits(__floats2bfloat162_rn(a, b));
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    readout_fp8_tc_kernel(const __grid_constant__ CUtensorMap mQ, const Ro8Args a) {
+    readout_fp8_tc_kernel(const __grid_constant__ CUtensorMap mQ, const __grid_constant__ CUtensorMap mO,
+                          const Ro8Args a) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   uint8_t* sHi = smem + kSHiOff;
   uint8_t* sLo = smem + kSLoOff;
   uint8_t* sQ = smem + kQOff;
+  uint8_t* sO = smem + kOOff;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOff);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
@@ -141,8 +156,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* epibar = drain + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epibar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* sred = reinterpret_cast<float*>(tmem_slot + 4);  // [4] per-warp maxima
-  static_assert((2 * kStages + 7) * 8 + 32 <= 256, "barrier block overflows its allowance");
+  float* sred = reinterpret_cast<float*>(tmem_slot + 4);  // [8] per-warp maxima
+  static_assert((2 * kStages + 7) * 8 + 16 + 32 <= 256, "barrier block overflows its allowance");
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   int tiles_per_head = 0;
@@ -160,14 +175,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4);
+      mbar_init(&tempty[i], 8);
     }
-    mbar_init(sready, 4);
+    mbar_init(sready, 8);
     mbar_init(drain, 1);
     mbar_init(epibar, kEpi);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&mQ);
+    prefetch_tmap(&mO);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 256);
@@ -223,8 +239,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(drain);
     }
   } else {
-    const int et = threadIdx.x - 64;  // 0..127
+    const int et = threadIdx.x - 64;  // 0..255
     const int quad = warp % 4;
+    const int hf = (warp - 2) / 4;    // output columns 64 hf .. 64 hf + 63
     const int r = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     // Anchor frames 0 and T-1 read zero: this CTA's share of their rows (per batch
@@ -267,9 +284,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        if (lane == 0) sred[quad] = mx;
+        if (lane == 0) sred[warp - 2] = mx;
         if (!epi_sync()) break;
-        mx = fmaxf(fmaxf(sred[0], sred[1]), fmaxf(sred[2], sred[3]));
+#pragma unroll
+        for (int w = 0; w < 8; ++w) mx = fmaxf(mx, sred[w]);
         // 2^E with max |S| 2^E <= 240 (an exact power of two; 0 when S is zero)
         const int E = mx > 0.f ? max(-100, min(100, (int)floorf(log2f(240.f / mx)))) : 0;
         const float sc = ldexpf(1.f, E);
@@ -319,30 +337,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool live = r < ti.nvalid;
       const long long tok = ti.tok0 + (live ? r : 0);
       const float scale = (live ? a.q_scale[tok * a.Ht + h] : 0.f) * inv_scale;
-      uint4* dst = reinterpret_cast<uint4*>(a.O + (tok * a.Ht + h) * (long long)D);
+      // This warp's half row: 64 columns as eight 16-byte chunks of bf16.
+      uint4 outs[8];
 #pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
+      for (int c = 0; c < 4; ++c) {
         uint32_t v[16];
-        tmem_ld16(tmem + lane_off + tb * D + c * 16, v);
+        tmem_ld16(tmem + lane_off + tb * D + hf * 64 + c * 16, v);
         tmem_ld_wait();
-        if (live) {
-          uint4 w0, w1;
-          w0.x = pack_bf16(__uint_as_float(v[0]) * scale, __uint_as_float(v[1]) * scale);
-          w0.y = pack_bf16(__uint_as_float(v[2]) * scale, __uint_as_float(v[3]) * scale);
-          w0.z = pack_bf16(__uint_as_float(v[4]) * scale, __uint_as_float(v[5]) * scale);
-          w0.w = pack_bf16(__uint_as_float(v[6]) * scale, __uint_as_float(v[7]) * scale);
-          w1.x = pack_bf16(__uint_as_float(v[8]) * scale, __uint_as_float(v[9]) * scale);
-          w1.y = pack_bf16(__uint_as_float(v[10]) * scale, __uint_as_float(v[11]) * scale);
-          w1.z = pack_bf16(__uint_as_float(v[12]) * scale, __uint_as_float(v[13]) * scale);
-          w1.w = pack_bf16(__uint_as_float(v[14]) * scale, __uint_as_float(v[15]) * scale);
-          dst[2 * c] = w0;
-          dst[2 * c + 1] = w1;
-        }
+        uint32_t w[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) w[k] = pack_bf16(__uint_as_float(v[2 * k]) * scale, __uint_as_float(v[2 * k + 1]) * scale);
+        outs[2 * c] = make_uint4(w[0], w[1], w[2], w[3]);
+        outs[2 * c + 1] = make_uint4(w[4], w[5], w[6], w[7]);
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[tb]);
+      if (lane == 0) mbar_arrive(&tempty[tb]);  // accumulator read: the MMAs may reuse it
+      const bool partial = ti.nvalid < kTileM;
+      // The staging tile must have been read by the previous tile's TMA store.
+      if (et == 0) bulk_wait_read0();
+      if (!epi_sync()) break;
+      if (!partial) {
+        uint8_t* orow = sO + hf * kOBox + r * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(orow + ((c ^ (r & 7)) << 4)) = outs[c];
+      } else if (live) {
+        uint4* dst = reinterpret_cast<uint4*>(a.O + (tok * a.Ht + h) * (long long)D) + hf * 8;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) dst[c] = outs[c];
+      }
+      fence_proxy_async_smem();
+      if (!epi_sync()) break;
+      if (et == 0 && !partial) {
+        tma_store_3d(&mO, sO, 0, h, (int)ti.tok0);
+        tma_store_3d(&mO, sO + kOBox, 64, h, (int)ti.tok0);
+        bulk_commit();
+      }
     }
+    if (et == 0) bulk_wait0();  // every output write done before the CTA retires
   }
 
   tc_fence_before();
@@ -393,11 +425,15 @@ cudaError_t launch_readout_fp8_tc(const Problem& p, const void* Q8, const float*
   const uint64_t dims[3] = {(uint64_t)D, (uint64_t)p.H, (uint64_t)p.B * p.T * p.U};
   const uint64_t strides[2] = {(uint64_t)D, (uint64_t)p.Ht * D};
   const uint32_t box[3] = {(uint32_t)D, 1u, (uint32_t)kTileM};
-  CUtensorMap mQ;
+  CUtensorMap mQ, mO;
   if ((e = make_tmap_typed(&mQ, CU_TENSOR_MAP_DATA_TYPE_UINT8, Q8, 3, dims, strides, box,
                            CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
     return e;
-  readout_fp8_tc_kernel<<<(unsigned)ncta, kThreads, kSmemBytes, s>>>(mQ, a);
+  // O: bf16 [B*T*U tokens, H, D] from this problem's first head, 64-column boxes.
+  const uint64_t ostrides[2] = {(uint64_t)D * 2, (uint64_t)p.Ht * D * 2};
+  const uint32_t obox[3] = {64u, 1u, (uint32_t)kTileM};
+  if ((e = make_tmap_bf16(&mO, O, 3, dims, ostrides, obox)) != cudaSuccess) return e;
+  readout_fp8_tc_kernel<<<(unsigned)ncta, kThreads, kSmemBytes, s>>>(mQ, mO, a);
   return cudaGetLastError();
 }
 
