@@ -40,7 +40,8 @@ constexpr int kSBytes = D * D;          // one e4m3 image of S (16 KB)
 constexpr int kSHiOff = 0, kSLoOff = kSBytes, kQOff = 2 * kSBytes;
 constexpr int kOOff = kQOff + kStages * kTileBytes;  // bf16 output tile staged for the TMA store (32 KB)
 constexpr int kOBox = kTileM * 128;                      // one 64-column box of it
-constexpr int kBarOff = kOOff + 2 * kOBox;
+constexpr int kScOff = kOOff + 2 * kOBox;               // per stage, the tile's 128 query scales
+constexpr int kBarOff = kScOff + kStages * kTileM * 4;
 constexpr int kSmemBytes = kBarOff + 256 + 1024;
 // kind::f8f6f4: D f32, A and B e4m3, both K-major, M = 128, N = 128.
 constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(D >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
@@ -147,6 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sLo = smem + kSLoOff;
   uint8_t* sQ = smem + kQOff;
   uint8_t* sO = smem + kOOff;
+  float* sscale = reinterpret_cast<float*>(smem + kScOff);  // [kStages][kTileM]
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOff);
   uint64_t* empty = full + kStages;
   uint64_t* tfull = empty + kStages;
@@ -170,8 +172,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&full[s], 1 + 32);  // TMA bytes + the 32 lanes' scale copies
+      mbar_init(&empty[s], 1 + 8);  // MMA commit + the 8 epilogue warps (they read the scales)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
@@ -196,18 +198,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   int issued = 0;
 
   if (warp == 0) {
-    if (lane == 0) {
-      Iter it;
-      if (ntiles > 0) it.start(a, t_begin);
-      for (int n = 0; n < ntiles; ++n) {
-        if (n > 0) it.next(a);
-        const int s = n % kStages;
-        if (!mbar_wait(&empty[s], ((n / kStages) & 1) ^ 1, abort_flag, a.status, a.wait_ns)) break;
-        const Tile ti = it.tile(a, my_bh);
+    // Q tile by TMA (lane 0); the tile's query scales by 4-byte asynchronous
+    // copies (all lanes, zero past the tile's last valid row), on the same barrier.
+    Iter it;
+    if (ntiles > 0) it.start(a, t_begin);
+    for (int n = 0; n < ntiles; ++n) {
+      if (n > 0) it.next(a);
+      const int s = n % kStages;
+      int good = 1;
+      if (lane == 0) good = mbar_wait(&empty[s], ((n / kStages) & 1) ^ 1, abort_flag, a.status, a.wait_ns) ? 1 : 0;
+      good = __shfl_sync(0xffffffffu, good, 0);
+      if (!good) break;
+      const Tile ti = it.tile(a, my_bh);
+      if (lane == 0) {
         mbar_arrive_expect_tx(&full[s], kTileBytes);
         tma_load_3d(sQ + s * kTileBytes, &mQ, &full[s], 0, h, (int)ti.tok0);
-        issued = n + 1;
       }
+#pragma unroll
+      for (int j = 0; j < kTileM / 32; ++j) {
+        const int row = j * 32 + lane;
+        const bool in = row < ti.nvalid;
+        const float* src = a.q_scale + (ti.tok0 + (in ? row : 0)) * a.Ht + h;
+        cp_async_4(sscale + s * kTileM + row, src, in ? 4u : 0u);
+      }
+      cp_async_mbar_arrive_noinc(&full[s]);
+      if (lane == 0) issued = n + 1;
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -336,7 +351,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const bool live = r < ti.nvalid;
       const long long tok = ti.tok0 + (live ? r : 0);
-      const float scale = (live ? a.q_scale[tok * a.Ht + h] : 0.f) * inv_scale;
+      // The stage's scales have landed once its barrier completes; read this row's
+      // and give the stage back (with the MMA commit, the ninth arrival).
+      const int s = n % kStages;
+      const bool sgot = mbar_wait(&full[s], (n / kStages) & 1, abort_flag, a.status, a.wait_ns);
+      if (!__all_sync(0xffffffffu, sgot)) break;
+      const float scale = sscale[s * kTileM + r] * inv_scale;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
       // This warp's half row: 64 columns as eight 16-byte chunks of bf16.
       uint4 outs[8];
 #pragma unroll
