@@ -34,6 +34,12 @@ cudaError_t set_max_dynamic_smem(const void* func, int bytes) {
   std::lock_guard<std::mutex> lock(mu);
   if (done.count({func, dev})) return cudaSuccess;
   e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  // Every tensor-core kernel asks for the largest shared-memory carveout, so that
+  // CTAs of kernels that overlap (the statistics kernel and the compact solve
+  // CTAs beside it, the solve's last wave and the scan) find the SM in the same
+  // configuration and can be resident together.
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(func, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess) done.insert({func, dev});
   return e;
 }
