@@ -723,25 +723,38 @@ def run_backward_path(args, cfg, rank, world, local, dist, dev):
     ctx.profile_enable(False)
     if ctx.poll_device_status() != 0:
         raise RuntimeError("device status reported a timeout in the timed region")
-    launches = ctx.launch_count() - n0 + args.steps  # frame_bwd_simt is two launches per step
+    tc_tokens = "token_bwd_tc" in prof
+    # frame_bwd_simt is two launches per step when it also does the token part
+    launches = ctx.launch_count() - n0 + (0 if tc_tokens else args.steps)
     value = whole_job_rate(world, cfg, args.steps, ms_max)
     fl = backward_flops(cfg)
-    bn, bms = prof["frame_bwd_simt"]
-    b_s = bms / bn / 1e3
+    peaks, peak_src = load_peaks()
     sm_mhz = float(clocks.summary().get("sm_mhz") or 1965.0)
-    peak = alu_peak_tflops(sm_mhz)
-    achieved = (fl["frame"] + fl["token"]) / b_s / 1e12
+    dom = max(prof.items(), key=lambda kv: kv[1][1] / kv[1][0])[0]
+    dn, dms = prof[dom]
+    d_s = dms / dn / 1e3
+    B_, H_, d_, T_, U_ = cfg.B, cfg.H, cfg.d, cfg.T, cfg.U
+    esz = 4 if cfg.dtype == "f32" else 2
+    token_bytes = B_ * H_ * (T_ - 2) * U_ * (4 * d_ * esz + 8)  # K, V, beta in; dK, dV, dbeta out
+    if dom == "token_bwd_tc":
+        bound, unit, peak = "hbm", "GB/s", float(peaks["hbm_gbs"])
+        achieved = token_bytes / d_s / 1e9
+        peak_note = f"hbm_gbs of {peak_src}"
+    else:
+        bound, unit, peak = "alu", "TFLOP/s", alu_peak_tflops(sm_mhz)
+        achieved = (fl["frame"] + (0 if tc_tokens else fl["token"])) / d_s / 1e12
+        peak_note = f"fp32 FMA peak derived: 148 SMs x 128 lanes x 2 flop x {sm_mhz:.0f} MHz"
     if rank == 0:
         line = {"metric": "frame-step backward head-tokens/s (dK, dV, dbeta, dalpha, dS_prev)", "value": value,
                 "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic", "impl": "vda",
                 "config": {"workload": workload_desc(cfg), "path": "backward"},
-                "roofline": {"bound": "alu", "kernel": "frame_bwd_simt", "achieved": achieved, "peak": peak,
-                             "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
-                             "peak_source": f"fp32 FMA peak derived: 148 SMs x 128 lanes x 2 flop x {sm_mhz:.0f} MHz",
-                             "algorithmic_flops_per_launch": fl["frame"] + fl["token"],
-                             "algorithmic_bytes_per_launch": backward_bytes(cfg)},
+                "roofline": {"bound": bound, "kernel": dom, "achieved": achieved, "peak": peak,
+                             "unit": unit, "frac": achieved / peak, "traffic": None, "peak_source": peak_note,
+                             "algorithmic_flops_per_launch": fl["frame"] if dom != "token_bwd_tc" else fl["token"],
+                             "algorithmic_bytes_per_launch": token_bytes if dom == "token_bwd_tc"
+                             else backward_bytes(cfg)},
                 "kernels": {k: {"launches": n, "avg_us": tot / n * 1e3} for k, (n, tot) in prof.items()},
                 "gpu_launches": launches, "clocks": clocks.summary()}
         if world == 1 and args.cpu_budget > 0:

@@ -132,6 +132,7 @@ enum KernelId {
   K_SOLVE_TC_FRAMES,
   K_READOUT_FP8_TC,
   K_GRAM_FP8_TC,
+  K_TOKEN_BWD_TC,
   K_NUM_KERNELS
 };
 const char* kernel_name(int id);
@@ -150,7 +151,13 @@ cudaError_t launch_selftest_wait(uint32_t* status, unsigned long long spins, cud
 // written A_t, B_t): writes dS_prev, dalpha, dbeta, dK, dV (and Gx, Gsym into the
 // workspace's M and C slots). Two launches.
 cudaError_t launch_frame_bwd_simt(const Problem& p, const float* S_prev, const float* dS, float* dS_prev,
-                                  float* dalpha, float* dbeta, void* dK, void* dV, cudaStream_t s);
+                                  float* dalpha, float* dbeta, void* dK, void* dV, cudaStream_t s,
+                                  bool tokens = true);
+// The per-token part of that backward on tcgen05 (bf16, D = 128), after the
+// per-frame adjoints are in the workspace's M (Gx) and C (Gsym) slots.
+bool token_bwd_tc_supported(const Problem& p);
+cudaError_t launch_token_bwd_tc(const Problem& p, const void* K, const void* V, float* dbeta, void* dK, void* dV,
+                                cudaStream_t s);
 // The sweep solve's pivot reciprocal applied to x[0..n) (for an error bound test).
 cudaError_t launch_recip_selftest(const float* x, float* y, int n, cudaStream_t s);
 

@@ -800,7 +800,7 @@ cudaError_t launch_prep_text(const Problem& p, const void* Kt, const void* Vt, c
 }
 
 cudaError_t launch_frame_bwd_simt(const Problem& p, const float* S_prev, const float* dS, float* dS_prev,
-                                  float* dalpha, float* dbeta, void* dK, void* dV, cudaStream_t s) {
+                                  float* dalpha, float* dbeta, void* dK, void* dV, cudaStream_t s, bool tokens) {
   if (p.T < 3) return cudaSuccess;
   const BwdArgs g{S_prev, dS, dS_prev, dalpha, dbeta, dK, dV};
   return dispatch_d(p.D, [&](auto dc) {
@@ -810,6 +810,7 @@ cudaError_t launch_frame_bwd_simt(const Problem& p, const float* S_prev, const f
     if (e != cudaSuccess) return e;
     solve_bwd_simt_kernel<D><<<dim3(p.T - 2, p.H, p.B), SweepCfg<D>::kThreads, sm1, s>>>(p, g);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (!tokens) return cudaSuccess;  // the tensor-core token kernel follows
     const size_t sm2 = (size_t)(2 * D + 2 * 32) * (D + 1) * sizeof(float);
     e = set_max_dynamic_smem(reinterpret_cast<const void*>(token_bwd_simt_kernel<D>), (int)sm2);
     if (e != cudaSuccess) return e;

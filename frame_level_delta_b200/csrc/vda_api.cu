@@ -21,7 +21,7 @@ const char* kernel_name(int id) {
       "prep_video", "prep_text", "gram_simt", "gram_tc", "solve_simt",
       "scan_simt", "readout_simt", "readout_tc", "zero_anchors", "solve_tc", "scan_tc", "compose_tc",
       "solve_chol_tc", "window_attn_tc", "merge_tc", "frame_bwd_simt", "solve_tc_frames", "readout_fp8_tc",
-      "gram_fp8_tc"};
+      "gram_fp8_tc", "token_bwd_tc"};
   return (id >= 0 && id < K_NUM_KERNELS) ? names[id] : "?";
 }
 
@@ -692,9 +692,12 @@ vda_status vda_frame_solve_backward(vda_ctx* ctx, const void* K, const void* V, 
     st = run_kernel(ctx, K_GRAM_SIMT, s, [&] { return launch_gram_simt(p, s); });
   if (st != VDA_OK) return st;
   ctx->prepared = ctx->scanned = false;  // the workspace no longer holds a forward pass
-  return run_kernel(ctx, K_FRAME_BWD_SIMT, s, [&] {
-    return launch_frame_bwd_simt(p, S_prev, dS, dS_prev, dalpha, dbeta, dK, dV, s);
+  const bool tc = !use_simt_only(c) && token_bwd_tc_supported(p);
+  st = run_kernel(ctx, K_FRAME_BWD_SIMT, s, [&] {
+    return launch_frame_bwd_simt(p, S_prev, dS, dS_prev, dalpha, dbeta, dK, dV, s, !tc);
   });
+  if (st != VDA_OK || !tc) return st;
+  return run_kernel(ctx, K_TOKEN_BWD_TC, s, [&] { return launch_token_bwd_tc(p, K, V, dbeta, dK, dV, s); });
 }
 
 vda_status vda_hybrid_merge(const void* O_soft, const void* W_soft, const void* O_lin, const void* W_lin, void* Y,
