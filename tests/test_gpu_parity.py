@@ -164,13 +164,22 @@ CONV_EDGE = [
     ("conv_d64", dict(d=64, grid_h=4, grid_w=35)),
     ("conv_d128", dict(d=128, grid_h=7, grid_w=21)),
     ("conv_d128_single_row", dict(d=128, grid_h=1, grid_w=33)),
+    # d = 128 bf16 runs persistent CTAs over tiles of two grid rows and a frame
+    # loop unrolled by five: a single scanned frame, a loop that ends on each
+    # unrolled position, a second batch, and more tiles than SMs (each CTA
+    # walks several tiles across planes).
+    ("conv_d128_T3", dict(d=128, grid_h=3, grid_w=18, T=3, chunk=1)),
+    ("conv_d128_T6_batch_two", dict(d=128, B=2, grid_h=4, grid_w=16, T=6)),
+    ("conv_d128_T7", dict(d=128, grid_h=2, grid_w=47, T=7)),
+    ("conv_d128_T8", dict(d=128, grid_h=5, grid_w=3, T=8)),
+    ("conv_d128_many_tiles", dict(d=128, H=4, grid_h=15, grid_w=64, T=5)),
 ]
 
 
 @pytest.mark.parametrize("name,kw", CONV_EDGE, ids=[e[0] for e in CONV_EDGE])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_edge_conv_dims(name, kw, dtype):
-    cfg = CONFIGS["hires"].with_(name=name, H=2, T=9, L=5, chunk=2, dtype=dtype, **kw)
+    cfg = CONFIGS["hires"].with_(name=name, **{**dict(H=2, T=9, L=5, chunk=2, dtype=dtype), **kw})
     inp = make_inputs(cfg)
     check_config(cfg, inp=inp)
     _, regions, _ = run_gpu(cfg, inp)
