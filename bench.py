@@ -174,7 +174,7 @@ def kernel_bytes(name: str, cfg) -> float:
         return BH * F * 2 * dd4
     if name in ("solve_tc", "solve_chol_tc"):  # A, B, alpha read; C (fp32) and M's hi/lo operand images written
         return BH * (3 * NS * dd4 + F * dd4 + F * d * 4)
-    if name == "scan_tc":  # per step: a (chunk) map's hi/lo images + its C; S_T; readout states
+    if name in ("scan_tc", "scan_split_tc"):  # per step: a (chunk) map's hi/lo images + its C; S_T; readout states
         if composed_chunks(cfg):
             steps = 2 * (J - 2)
         else:
@@ -288,7 +288,7 @@ def source_digest(kernel: str):
     files = {"gram_tc": "gram_tc.cu", "readout_tc": "readout_tc.cu", "solve_tc": "solve_tc.cu",
              "gram_fp8_tc": "gram_fp8_tc.cu", "readout_fp8_tc": "readout_fp8_tc.cu",
              "solve_tc_frames": "solve_tc.cu", "window_attn_tc": "window_attn_tc.cu", "merge_tc": "merge_tc.cu",
-             "scan_tc": "scan_tc.cu", "compose_tc": "compose_tc.cu", "solve_chol_tc": "solve_chol_tc.cu",
+             "scan_tc": "scan_tc.cu", "scan_split_tc": "scan_split_tc.cu", "compose_tc": "compose_tc.cu", "solve_chol_tc": "solve_chol_tc.cu",
              "prep_video": "prep_video.cu"}
     fn = files.get(kernel, "kernels_simt.cu")
     p = os.path.join(ROOT, "frame_level_delta_b200", "csrc", fn)

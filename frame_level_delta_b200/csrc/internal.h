@@ -133,6 +133,7 @@ enum KernelId {
   K_READOUT_FP8_TC,
   K_GRAM_FP8_TC,
   K_TOKEN_BWD_TC,
+  K_SCAN_SPLIT_TC,
   K_NUM_KERNELS
 };
 const char* kernel_name(int id);
@@ -175,6 +176,10 @@ cudaError_t launch_solve_tc(const Problem& p, cudaStream_t s, int part);
 cudaError_t launch_solve_chol_tc(const Problem& p, cudaStream_t s);
 bool scan_tc_supported(const Problem& p);
 cudaError_t launch_scan_tc(const Problem& p, cudaStream_t s, bool chunked);
+// Frame scan with each state's 64-column halves on the two CTAs of a cluster
+// (after the sweep solve, injections formed in the scan).
+bool scan_split_tc_supported(const Problem& p);
+cudaError_t launch_scan_split_tc(const Problem& p, cudaStream_t s);
 cudaError_t launch_compose_tc(const Problem& p, cudaStream_t s);
 cudaError_t launch_readout_tc(const Problem& p, const void* gate, void* O, cudaStream_t s);
 

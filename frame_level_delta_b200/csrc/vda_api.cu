@@ -21,7 +21,7 @@ const char* kernel_name(int id) {
       "prep_video", "prep_text", "gram_simt", "gram_tc", "solve_simt",
       "scan_simt", "readout_simt", "readout_tc", "zero_anchors", "solve_tc", "scan_tc", "compose_tc",
       "solve_chol_tc", "window_attn_tc", "merge_tc", "frame_bwd_simt", "solve_tc_frames", "readout_fp8_tc",
-      "gram_fp8_tc", "token_bwd_tc"};
+      "gram_fp8_tc", "token_bwd_tc", "scan_split_tc"};
   return (id >= 0 && id < K_NUM_KERNELS) ? names[id] : "?";
 }
 
@@ -89,7 +89,8 @@ vda_status check_config(const vda_config* c, std::string* why) {
   if (c->chunk < 1) return bad("chunk must be >= 1");
   if (c->dtype != VDA_F32 && c->dtype != VDA_BF16) return bad("dtype must be VDA_F32 or VDA_BF16");
   if (!(c->l2_eps >= 0.f) || !(c->rms_eps >= 0.f)) return bad("eps must be >= 0");
-  if (c->flags & ~(VDA_PREP_CONV | VDA_READOUT_NORM_GATE | VDA_SOLVE_CHOLESKY | VDA_SCAN_CHUNKED | VDA_FORCE_SIMT))
+  if (c->flags &
+      ~(VDA_PREP_CONV | VDA_READOUT_NORM_GATE | VDA_SOLVE_CHOLESKY | VDA_SCAN_CHUNKED | VDA_SCAN_SPLIT | VDA_FORCE_SIMT))
     return bad("unknown flag bits");
   if (c->d_k != c->d_v) {
     if (why) *why = "d_k != d_v is not supported";
@@ -312,11 +313,13 @@ vda_status vda_describe(const vda_config* cfg, const char** text) {
   const bool v = !simt && solve_tc_supported(p), n = !simt && scan_tc_supported(p);
   const bool chol = v && (cfg->flags & VDA_SOLVE_CHOLESKY);
   const bool pf = pform_of(*cfg, p);
-  static char table[2][2][2][2][2][2][112];
-  char* t = table[g][v][chol][n][r][pf];
-  std::snprintf(t, 112, "gram=%s solve=%s scan=%s readout=%s%s", g ? "tcgen05" : "simt",
-                v ? (chol ? "tcgen05-cholesky" : "tcgen05") : "simt", n ? "tcgen05" : "simt", r ? "tcgen05" : "simt",
-                pf ? " inject=scan" : "");
+  p.pform = pf ? 1 : 0;
+  const bool split = n && (cfg->flags & VDA_SCAN_SPLIT) && scan_split_tc_supported(p);
+  static char table[2][2][2][2][2][2][2][120];
+  char* t = table[g][v][chol][n][split][r][pf];
+  std::snprintf(t, 120, "gram=%s solve=%s scan=%s readout=%s%s", g ? "tcgen05" : "simt",
+                v ? (chol ? "tcgen05-cholesky" : "tcgen05") : "simt",
+                n ? (split ? "tcgen05-split" : "tcgen05") : "simt", r ? "tcgen05" : "simt", pf ? " inject=scan" : "");
   *text = t;
   return VDA_OK;
 }
@@ -511,7 +514,16 @@ vda_status vda_scan_bidir(vda_ctx* ctx, void* stream) {
       st = run_kernel(ctx, K_COMPOSE_TC, s, [&] { return launch_compose_tc(ctx->p, s); });
       if (st != VDA_OK) return st;
     }
-    st = run_kernel(ctx, K_SCAN_TC, s, [&] { return launch_scan_tc(ctx->p, s, chunked); });
+    // On request, frame by frame on two-CTA clusters (each CTA half of every
+    // state's columns). One CTA per (b, h, direction) is the default: each step
+    // is bound by the MMA -> epilogue -> operand hand-offs, not by the MMAs or
+    // the epilogue's arithmetic that the split halves, and the split adds the
+    // exchange of the left factor's halves (measured at the H3-like clip:
+    // 93 us against 71 us).
+    if (!chunked && (ctx->cfg.flags & VDA_SCAN_SPLIT) && scan_split_tc_supported(ctx->p))
+      st = run_kernel(ctx, K_SCAN_SPLIT_TC, s, [&] { return launch_scan_split_tc(ctx->p, s); });
+    else
+      st = run_kernel(ctx, K_SCAN_TC, s, [&] { return launch_scan_tc(ctx->p, s, chunked); });
   } else
     st = run_kernel(ctx, K_SCAN_SIMT, s, [&] { return launch_scan_simt(ctx->p, s); });
   if (st != VDA_OK) return st;

@@ -24,6 +24,7 @@ VDA_PREP_CONV = 0x1
 VDA_READOUT_NORM_GATE = 0x2
 VDA_SOLVE_CHOLESKY = 0x4
 VDA_SCAN_CHUNKED = 0x8
+VDA_SCAN_SPLIT = 0x10
 VDA_FORCE_SIMT = 0x100
 REGIONS = {"status": 0, "A": 1, "B": 2, "M": 3, "C": 4, "S_fwd": 5, "S_rev": 6,
            "K_prep": 7, "V_prep": 8, "Kt_prep": 9, "Vt_prep": 10, "M_split": 11,
@@ -106,7 +107,7 @@ def lib() -> ctypes.CDLL:
 
 def make_config(cfg: VDAConfig, force_simt: bool = False, l2_eps: float = 1e-6,
                 rms_eps: float = 1e-6, cholesky: bool = False, chunked: bool = False,
-                heads: Optional[Tuple[int, int]] = None) -> vda_config:
+                heads: Optional[Tuple[int, int]] = None, split_scan: bool = False) -> vda_config:
     """The C config of a workload. ``heads = (h0, n)`` makes a context for heads
     h0 .. h0+n-1 of the workload's cfg.H heads (token tensors keep all cfg.H)."""
     flags = (VDA_PREP_CONV if cfg.prep_conv else 0) | (VDA_READOUT_NORM_GATE if cfg.norm_gate else 0)
@@ -116,6 +117,8 @@ def make_config(cfg: VDAConfig, force_simt: bool = False, l2_eps: float = 1e-6,
         flags |= VDA_SOLVE_CHOLESKY
     if chunked:
         flags |= VDA_SCAN_CHUNKED
+    if split_scan:
+        flags |= VDA_SCAN_SPLIT
     h0, n = heads if heads is not None else (0, cfg.H)
     return vda_config(B=cfg.B, H=n, T=cfg.T, U=cfg.U, grid_h=cfg.grid_h, grid_w=cfg.grid_w, L=cfg.L,
                       d_k=cfg.d, d_v=cfg.d, chunk=cfg.chunk,
@@ -166,10 +169,11 @@ class VDA:
     the context's heads here."""
 
     def __init__(self, cfg: VDAConfig, force_simt: bool = False, device="cuda", cholesky: bool = False,
-                 chunked: bool = False, heads: Optional[Tuple[int, int]] = None):
+                 chunked: bool = False, heads: Optional[Tuple[int, int]] = None, split_scan: bool = False):
         self.cfg = cfg
         self.heads = heads
-        self.c = make_config(cfg, force_simt=force_simt, cholesky=cholesky, chunked=chunked, heads=heads)
+        self.c = make_config(cfg, force_simt=force_simt, cholesky=cholesky, chunked=chunked, heads=heads,
+                             split_scan=split_scan)
         self._ctx = ctypes.c_void_p()
         st = lib().vda_create(ctypes.byref(self.c), ctypes.byref(self._ctx))
         if st != VDA_OK:

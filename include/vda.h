@@ -84,6 +84,11 @@ typedef enum vda_dtype {
                                       maps composed in parallel first) instead of the default scan
                                       frame by frame; the same readout states. Needs
                                       B * H <= 65535, else VDA_ERR_UNSUPPORTED from vda_create */
+#define VDA_SCAN_SPLIT 0x10u       /* tensor-core frame scan on a two-CTA cluster per (b, h,
+                                      direction), each CTA computing half of every state's columns
+                                      and sending its half of the next left factor to the other,
+                                      instead of the default one CTA per (b, h, direction) (the same
+                                      readout states; no effect with VDA_SCAN_CHUNKED) */
 #define VDA_FORCE_SIMT 0x100u      /* run the generic CUDA-core kernels even where a tensor-core
                                       kernel exists (diagnostics and cross-checks) */
 

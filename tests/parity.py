@@ -31,10 +31,11 @@ def rel_fro(a, b) -> float:
     return float(np.linalg.norm(a - b) / (nb if nb > 0 else 1.0))
 
 
-def run_gpu(cfg, inp_cpu, force_simt=False, cholesky=False, chunked=False):
+def run_gpu(cfg, inp_cpu, force_simt=False, cholesky=False, chunked=False, split_scan=False):
     dev = torch.device("cuda:0")
     inp = {k: v.to(dev) for k, v in inp_cpu.items()}
-    lib = V.VDA(cfg, force_simt=force_simt, device=dev, cholesky=cholesky, chunked=chunked)
+    lib = V.VDA(cfg, force_simt=force_simt, device=dev, cholesky=cholesky, chunked=chunked,
+                split_scan=split_scan)
     O = lib.run(inp)
     torch.cuda.synchronize()
     assert lib.poll_device_status() == 0
@@ -137,12 +138,16 @@ def local_output_errors(cfg, O_g, O_ref, pairs, pre_norms=None):
 
 
 def check_config(cfg, heads=None, force_simt=False, inp=None, stage_tol=None, cholesky=False, chunked=False,
-                 return_regions=False):
+                 return_regions=False, split_scan=False):
     """Run both sides and assert the bounds. Returns (O error, staged errors)
     (and the GPU's workspace regions with return_regions)."""
     if inp is None:
         inp = make_inputs(cfg)
-    O_gpu, regions, lib = run_gpu(cfg, inp, force_simt=force_simt, cholesky=cholesky, chunked=chunked)
+    O_gpu, regions, lib = run_gpu(cfg, inp, force_simt=force_simt, cholesky=cholesky, chunked=chunked,
+                                  split_scan=split_scan)
+    desc = V.describe(lib.c)
+    if not force_simt and cfg.dtype == "bf16" and cfg.d == 128 and "inject=scan" in desc:
+        assert ("scan=tcgen05-split" in desc) == split_scan, desc
     if cholesky and not force_simt and cfg.dtype == "bf16" and cfg.d == 128:
         assert "solve=tcgen05-cholesky" in V.describe(lib.c)
     ref = vo.vda_reference(inp, cfg, heads=heads)

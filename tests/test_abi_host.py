@@ -156,6 +156,10 @@ def test_status_strings_and_describe():
     assert "inject=scan" not in V.describe(V.make_config(CONFIGS["h3"], chunked=True))
     assert "inject=scan" not in V.describe(V.make_config(CONFIGS["h3"], cholesky=True))
     assert "inject=scan" not in V.describe(V.make_config(CONFIGS["small"]))  # d = 64: CUDA-core solve
+    # The two-CTA cluster scan only on request, and only where the scan forms the injections.
+    assert "scan=tcgen05 " in V.describe(V.make_config(CONFIGS["h3"]))
+    assert "scan=tcgen05-split" in V.describe(V.make_config(CONFIGS["h3"], split_scan=True))
+    assert "scan=tcgen05-split" not in V.describe(V.make_config(CONFIGS["h3"], split_scan=True, chunked=True))
 
 
 def test_region_view_undoes_column_quad_layout():

@@ -137,6 +137,9 @@ EDGE_CHUNKS = [
     ("d128_chunk_one", dict(T=9, chunk=1)),
     ("d128_wide_chunks", dict(T=20, chunk=8)),
     ("d128_batch_two", dict(B=2, T=11, chunk=3)),
+    # No scanned step in either direction, and one step in each.
+    ("d128_no_scan_step", dict(T=3, chunk=1)),
+    ("d128_one_scan_step", dict(T=4, chunk=1)),
 ]
 
 
@@ -144,6 +147,7 @@ EDGE_CHUNKS = [
 def test_edge_chunk_structures_tensor_core_scan(name, kw):
     cfg = CONFIGS["small"].with_(name=name, d=128, H=2, grid_h=4, grid_w=5, L=9, **kw)
     check_config(cfg)
+    check_config(cfg, split_scan=True)  # the frame scan on two-CTA clusters
     check_config(cfg, chunked=True)
     if name in ("d128_ragged_last_chunk", "d128_batch_two"):
         check_config(cfg, cholesky=True)
@@ -204,6 +208,20 @@ def test_degenerate_gates():
     inp["alpha"][:, 0].zero_()  # head 0 forgets everything each frame
     inp["beta"][:, 1, :, ::2] = 0  # head 1 skips every other token
     check_config(cfg, inp=inp)
+
+
+def test_split_scan_matches_one_cta_scan():
+    """The two-CTA cluster scan (each CTA half of every state's columns, the
+    halves of the next left factor exchanged between the CTAs' shared memories)
+    against the single-CTA scan on an H3-shaped clip: the same readout states up
+    to fp32 accumulation order over 29 steps."""
+    cfg = CONFIGS["h3"].with_(H=4)
+    inp = make_inputs(cfg)
+    _, r_split, lib = run_gpu(cfg, inp, split_scan=True)
+    assert "scan=tcgen05-split" in V.describe(lib.c)
+    _, r_one, _ = run_gpu(cfg, inp)
+    for k in ("S_fwd", "S_rev"):
+        assert rel_fro(r_split[k].numpy(), r_one[k].numpy()) <= 1e-5, k
 
 
 def test_repeated_runs_are_bitwise_identical():
