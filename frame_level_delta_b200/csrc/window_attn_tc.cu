@@ -371,12 +371,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sempty[i & 1]);  // S_i is in registers: the buffer may take S_{i+2}
-      float mb = -INFINITY;
+      // Columns past the block's keys are masked; the row maximum of the raw
+      // logits over eight independent chains, then taken to the log2 domain
+      // (sl > 0, and rounding is monotone: the same value as the maximum of the
+      // scaled logits).
+      if (valid < kTile) {
 #pragma unroll
-      for (int k = 0; k < kTile; ++k) {
-        s[k] = k < valid ? s[k] * a.sl : -INFINITY;
-        mb = fmaxf(mb, s[k]);
+        for (int k = 0; k < kTile; ++k)
+          if (k >= valid) s[k] = -INFINITY;
       }
+      float mx[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) mx[q] = s[q];
+#pragma unroll
+      for (int k = 8; k < kTile; ++k) mx[k & 7] = fmaxf(mx[k & 7], s[k]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) mx[q] = fmaxf(mx[q], mx[q + 4]);
+      const float mb = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * a.sl;
       // Rescale when the maximum grows by more than 2^8 over the reference the
       // earlier P entries used (the whole warp takes part in the TMEM access).
       const bool grow = i > 0 && mb > m_run + 8.f;
@@ -410,21 +421,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P_i goes where P_{i-2} was: that product must be complete.
       if (i >= 2 && !warp_wait(&pvdone[i & 1], ((i - 2) >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
-      float ls = 0.f;
+      // p = 2^(s sl - m): one packed FMA per pair of logits; the row sum over
+      // four independent packed chains.
       const uint32_t pa = tmem + lane_off + ((i & 1) ? C::kP1 : C::kP0);
+      const float2 sl2 = make_float2(a.sl, a.sl), nm2 = make_float2(-m_run, -m_run);
+      float2 ls2[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) ls2[q] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
         uint32_t w[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-          const float p0 = ex2_approx(s[c4 * 32 + 2 * k] - m_run);
-          const float p1 = ex2_approx(s[c4 * 32 + 2 * k + 1] - m_run);
-          ls += p0 + p1;
+          const float2 x = __ffma2_rn(make_float2(s[c4 * 32 + 2 * k], s[c4 * 32 + 2 * k + 1]), sl2, nm2);
+          const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+          ls2[k & 3] = __fadd2_rn(ls2[k & 3], make_float2(p0, p1));
           w[k] = pack_bf16(p0, p1);
         }
         tmem_st16(pa + c4 * 16, w);
       }
-      l_run += ls;
+      l_run += ((ls2[0].x + ls2[0].y) + (ls2[1].x + ls2[1].y)) + ((ls2[2].x + ls2[2].y) + (ls2[3].x + ls2[3].y));
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
