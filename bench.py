@@ -860,8 +860,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work (0: skip)")
     ap.add_argument("--solve", default="sweep", choices=["sweep", "cholesky"],
                     help="tensor-core frame solve: symmetric sweep (default) or blocked Cholesky")
-    ap.add_argument("--scan", default="frames", choices=["frames", "chunked"],
-                    help="tensor-core scan frame by frame (default) or over composed chunk maps")
+    ap.add_argument("--scan", default="frames", choices=["frames", "chunked", "split"],
+                    help="tensor-core scan frame by frame (default), over composed chunk maps, or frame "
+                         "by frame on two-CTA clusters (each CTA half of every state's columns)")
     ap.add_argument("--heads", type=int, default=0,
                     help="override H (a smaller case of the same workload, e.g. for profiler captures)")
     ap.add_argument("--path", default="linear", choices=["linear", "softmax", "hybrid", "backward"],
@@ -916,7 +917,8 @@ def main():
     global SCAN_CHUNKED, SOLVE_CHOLESKY
     SCAN_CHUNKED = args.scan == "chunked"
     SOLVE_CHOLESKY = args.solve == "cholesky"
-    lib = V.VDA(cfg, device=dev, cholesky=args.solve == "cholesky", chunked=SCAN_CHUNKED, heads=heads)
+    lib = V.VDA(cfg, device=dev, cholesky=args.solve == "cholesky", chunked=SCAN_CHUNKED, heads=heads,
+                split_scan=args.scan == "split")
     # Per-kernel accounting below is for the heads this rank serves.
     kcfg = cfg if heads is None else cfg.with_(H=heads[1])
     O = lib.new_output()
