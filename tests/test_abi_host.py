@@ -128,6 +128,22 @@ def test_calls_out_of_order_and_bad_pointers_are_rejected_before_launch():
         assert L.vda_destroy(ctx) == 0
 
 
+def test_fp8_prepare_rejects_conv_and_non_tensor_core_configs():
+    """vda_prepare_fp8 needs d = 128, bf16 outputs and no conv prep; it refuses
+    the others with VDA_ERR_UNSUPPORTED before touching any pointer."""
+    L = V.lib()
+    fake = [ctypes.c_void_p(0x100000 * (i + 1)) for i in range(9)]  # K8 .. beta_txt
+    for cfg in (CONFIGS["hires"], CONFIGS["small"], CONFIGS["tiny"]):
+        c = V.make_config(cfg)
+        st, ctx = _create(c)
+        assert st == 0
+        try:
+            got = L.vda_prepare_fp8(ctx, *fake, ctypes.c_void_p(0x7000000), ctypes.c_size_t(V.workspace_size(c)), None)
+            assert V.STATUS_NAMES[got] == "VDA_ERR_UNSUPPORTED", (cfg.name, got)
+        finally:
+            L.vda_destroy(ctx)
+
+
 def test_conv_and_gate_requirements():
     c = V.make_config(CONFIGS["hires"])
     st, ctx = _create(c)

@@ -116,6 +116,18 @@ def test_fp8_path_matches_oracle_on_stored_values(name, cfg):
             assert rel_fro(regions["B"][b, h, s], it["B"][s]) <= 4e-3, ("B", b, h, s)
 
 
+def test_fp8_path_long_clip_three_heads():
+    """The long clip's per-head workload at full size (120 frames of 30 x 52
+    tokens, chunks of 5, L = 512) with three heads: heads are independent, so
+    this is config 4's per-head computation, with the host-side float64 copies
+    of the inputs kept to a few GB."""
+    cfg = CONFIGS["long"].with_(H=3)
+    got, ref, _ = _run_fp8_path(cfg)
+    assert rel_fro(got, ref["O"]) <= TOL_O["bf16"]
+    loc = local_output_errors(cfg, got, ref["O"], ref["heads"])
+    assert loc["frame"] <= TOL_O["bf16"] and loc["token_ratio"] <= 1.0, loc
+
+
 def test_fp8_path_h3_full_size_spread_heads():
     cfg = CONFIGS["h3"]
     heads = [(0, 0), (0, 11), (0, 23)]
