@@ -319,27 +319,46 @@ __global__ void __launch_bounds__(kThreads, 1)
         const long long off = ((long long)ti.bh * a.J + ti.j) * (long long)D * D;
         const float4* pf = reinterpret_cast<const float4*>(a.Sf + off);
         const float4* pr = reinterpret_cast<const float4*>(a.Sr + off);
-        for (int e = et; e < D * (D / 8); e += kEpiThreads) {
-          const int c8 = e / D, i = e % D;  // row i, 8 consecutive k (column quads 2 c8, 2 c8 + 1)
-          float x[8];
-          const float4 f0 = pf[(2 * c8) * D + i], f1 = pf[(2 * c8 + 1) * D + i];
-          const float4 r0 = pr[(2 * c8) * D + i], r1 = pr[(2 * c8 + 1) * D + i];
-          x[0] = f0.x + r0.x; x[1] = f0.y + r0.y; x[2] = f0.z + r0.z; x[3] = f0.w + r0.w;
-          x[4] = f1.x + r1.x; x[5] = f1.y + r1.y; x[6] = f1.z + r1.z; x[7] = f1.w + r1.w;
-          uint32_t hp[4], lp[4];
+        // Each thread takes kItems (row, 8-column) items; the loads of a batch of
+        // them are issued before any is used, so a batch costs one L2 round trip.
+        constexpr int kItems = D * (D / 8) / kEpiThreads;
+        constexpr int kBatch = kItems < 4 ? kItems : 4;
+        static_assert(kItems % kBatch == 0 && D * (D / 8) % kEpiThreads == 0, "prologue items");
 #pragma unroll
-          for (int k2 = 0; k2 < 4; ++k2) {
-            const __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * k2], x[2 * k2 + 1]);
-            const float2 hf = __bfloat1622float2(hh);
-            hp[k2] = bf162_bits(hh);
-            lp[k2] = bf162_bits(__floats2bfloat162_rn(x[2 * k2] - hf.x, x[2 * k2 + 1] - hf.y));
+        for (int b0 = 0; b0 < kItems; b0 += kBatch) {
+          float4 f[kBatch][2], rv[kBatch][2];
+#pragma unroll
+          for (int bi = 0; bi < kBatch; ++bi) {
+            const int e = et + (b0 + bi) * kEpiThreads;
+            const int c8 = e / D, i = e % D;  // row i, 8 consecutive k (column quads 2 c8, 2 c8 + 1)
+            f[bi][0] = pf[(2 * c8) * D + i];
+            f[bi][1] = pf[(2 * c8 + 1) * D + i];
+            rv[bi][0] = pr[(2 * c8) * D + i];
+            rv[bi][1] = pr[(2 * c8 + 1) * D + i];
           }
-          const uint4 hv = make_uint4(hp[0], hp[1], hp[2], hp[3]);
-          const uint4 lv = make_uint4(lp[0], lp[1], lp[2], lp[3]);
-          const int atom = c8 / 8, chunk = c8 % 8;
-          const int boff = atom * C::kSAtomBytes + i * 128 + ((chunk ^ (i & 7)) * 16);
-          *reinterpret_cast<uint4*>(sShi + boff) = hv;
-          *reinterpret_cast<uint4*>(sSlo + boff) = lv;
+#pragma unroll
+          for (int bi = 0; bi < kBatch; ++bi) {
+            const int e = et + (b0 + bi) * kEpiThreads;
+            const int c8 = e / D, i = e % D;
+            const float4 f0 = f[bi][0], f1 = f[bi][1], r0 = rv[bi][0], r1 = rv[bi][1];
+            float x[8];
+            x[0] = f0.x + r0.x; x[1] = f0.y + r0.y; x[2] = f0.z + r0.z; x[3] = f0.w + r0.w;
+            x[4] = f1.x + r1.x; x[5] = f1.y + r1.y; x[6] = f1.z + r1.z; x[7] = f1.w + r1.w;
+            uint32_t hp[4], lp[4];
+#pragma unroll
+            for (int k2 = 0; k2 < 4; ++k2) {
+              const __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * k2], x[2 * k2 + 1]);
+              const float2 hf = __bfloat1622float2(hh);
+              hp[k2] = bf162_bits(hh);
+              lp[k2] = bf162_bits(__floats2bfloat162_rn(x[2 * k2] - hf.x, x[2 * k2 + 1] - hf.y));
+            }
+            const uint4 hv = make_uint4(hp[0], hp[1], hp[2], hp[3]);
+            const uint4 lv = make_uint4(lp[0], lp[1], lp[2], lp[3]);
+            const int atom = c8 / 8, chunk = c8 % 8;
+            const int boff = atom * C::kSAtomBytes + i * 128 + ((chunk ^ (i & 7)) * 16);
+            *reinterpret_cast<uint4*>(sShi + boff) = hv;
+            *reinterpret_cast<uint4*>(sSlo + boff) = lv;
+          }
         }
         fence_proxy_async_smem();
         if (!epi_sync()) { ok = false; break; }
