@@ -292,10 +292,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         const long long off = ((long long)my_bh * a.J + ti.j) * (long long)D * D;
         const float4* pf = reinterpret_cast<const float4*>(a.Sf + off);
         const float4* pr = reinterpret_cast<const float4*>(a.Sr + off);
+        // Loads issued in batches before they are used: one L2 round trip per
+        // batch instead of per item.
         float mx = 0.f;
-        for (int e = et; e < D * D / 4; e += kEpi) {
-          const float4 f = pf[e], g = pr[e];
-          mx = fmaxf(mx, fmaxf(fmaxf(fabsf(f.x + g.x), fabsf(f.y + g.y)), fmaxf(fabsf(f.z + g.z), fabsf(f.w + g.w))));
+        constexpr int kMaxItems = D * D / 4 / kEpi, kMaxBatch = 4;
+        static_assert(D * D / 4 % kEpi == 0 && kMaxItems % kMaxBatch == 0, "prologue items");
+#pragma unroll
+        for (int b0 = 0; b0 < kMaxItems; b0 += kMaxBatch) {
+          float4 f[kMaxBatch], g[kMaxBatch];
+#pragma unroll
+          for (int bi = 0; bi < kMaxBatch; ++bi) {
+            f[bi] = pf[et + (b0 + bi) * kEpi];
+            g[bi] = pr[et + (b0 + bi) * kEpi];
+          }
+#pragma unroll
+          for (int bi = 0; bi < kMaxBatch; ++bi)
+            mx = fmaxf(mx, fmaxf(fmaxf(fabsf(f[bi].x + g[bi].x), fabsf(f[bi].y + g[bi].y)),
+                                 fmaxf(fabsf(f[bi].z + g[bi].z), fabsf(f[bi].w + g[bi].w))));
         }
 #pragma unroll
         for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -307,38 +320,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int E = mx > 0.f ? max(-100, min(100, (int)floorf(log2f(240.f / mx)))) : 0;
         const float sc = ldexpf(1.f, E);
         inv_scale = ldexpf(1.f, -E);
-        // Row i, 16 consecutive k (column quads 4 c .. 4 c + 3) per work item.
-        for (int e = et; e < D * (D / 16); e += kEpi) {
-          const int c16 = e / D, i = e % D;
-          float x[16];
+        // Row i, 16 consecutive k (column quads 4 c .. 4 c + 3) per work item,
+        // the loads of two items issued before either is used.
+        constexpr int kItems = D * (D / 16) / kEpi, kBatch = kItems < 2 ? kItems : 2;
+        static_assert(D * (D / 16) % kEpi == 0 && kItems % kBatch == 0, "prologue items");
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float4 f = pf[(4 * c16 + q) * D + i], g = pr[(4 * c16 + q) * D + i];
-            x[4 * q] = (f.x + g.x) * sc;
-            x[4 * q + 1] = (f.y + g.y) * sc;
-            x[4 * q + 2] = (f.z + g.z) * sc;
-            x[4 * q + 3] = (f.w + g.w) * sc;
-          }
-          // Pairs packed into 32-bit words by shifts (no type-punned stores).
-          uint32_t hw[4], lw[4];
+        for (int b0 = 0; b0 < kItems; b0 += kBatch) {
+          float4 fb[kBatch][4], gb[kBatch][4];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const uint16_t hh = to_e4m3x2(x[2 * q], x[2 * q + 1]);
-            const float2 hf = from_e4m3x2(hh);
-            const uint16_t ll = to_e4m3x2(x[2 * q] - hf.x, x[2 * q + 1] - hf.y);
-            if (q & 1) {
-              hw[q >> 1] |= (uint32_t)hh << 16;
-              lw[q >> 1] |= (uint32_t)ll << 16;
-            } else {
-              hw[q >> 1] = hh;
-              lw[q >> 1] = ll;
+          for (int bi = 0; bi < kBatch; ++bi) {
+            const int e = et + (b0 + bi) * kEpi, c16 = e / D, i = e % D;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              fb[bi][q] = pf[(4 * c16 + q) * D + i];
+              gb[bi][q] = pr[(4 * c16 + q) * D + i];
             }
           }
-          const uint4 hv = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          const uint4 lv = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-          const int boff = i * 128 + ((c16 ^ (i & 7)) << 4);
-          *reinterpret_cast<uint4*>(sHi + boff) = hv;
-          *reinterpret_cast<uint4*>(sLo + boff) = lv;
+#pragma unroll
+          for (int bi = 0; bi < kBatch; ++bi) {
+            const int e = et + (b0 + bi) * kEpi, c16 = e / D, i = e % D;
+            float x[16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float4 f = fb[bi][q], g = gb[bi][q];
+              x[4 * q] = (f.x + g.x) * sc;
+              x[4 * q + 1] = (f.y + g.y) * sc;
+              x[4 * q + 2] = (f.z + g.z) * sc;
+              x[4 * q + 3] = (f.w + g.w) * sc;
+            }
+            // Pairs packed into 32-bit words by shifts (no type-punned stores).
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const uint16_t hh = to_e4m3x2(x[2 * q], x[2 * q + 1]);
+              const float2 hf = from_e4m3x2(hh);
+              const uint16_t ll = to_e4m3x2(x[2 * q] - hf.x, x[2 * q + 1] - hf.y);
+              if (q & 1) {
+                hw[q >> 1] |= (uint32_t)hh << 16;
+                lw[q >> 1] |= (uint32_t)ll << 16;
+              } else {
+                hw[q >> 1] = hh;
+                lw[q >> 1] = ll;
+              }
+            }
+            const uint4 hv = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            const uint4 lv = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            const int boff = i * 128 + ((c16 ^ (i & 7)) << 4);
+            *reinterpret_cast<uint4*>(sHi + boff) = hv;
+            *reinterpret_cast<uint4*>(sLo + boff) = lv;
+          }
         }
         fence_proxy_async_smem();
         if (!epi_sync()) break;
