@@ -80,6 +80,8 @@ def test_fp8_readout_h3_full_size_spread_heads():
 FP8_PATH = [
     ("h3_shaped", CONFIGS["h3"].with_(H=2, T=10, grid_h=8, grid_w=8, L=16)),
     ("ragged", CONFIGS["h3"].with_(H=3, T=11, grid_h=7, grid_w=9, L=70, chunk=3)),
+    # More heads than the exponent pre-pass takes in one pass over a slot's tokens.
+    ("many_heads", CONFIGS["h3"].with_(H=34, T=6, grid_h=4, grid_w=5, L=9, chunk=2)),
 ]
 
 
