@@ -76,8 +76,24 @@ struct PrepIO<float> {
   static __device__ __forceinline__ void store4(float* dst, float4 v) { *reinterpret_cast<float4*>(dst) = v; }
 };
 
-// Fast division intrinsic: a few ulp, far below the bf16 rounding of the output.
-__device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.f + __expf(-x)); }
+// SiLU. fp32 storage: x / (1 + e^-x) with the fast division intrinsic (a few
+// ulp). bf16 storage: x sigmoid(x) = h + h tanh(h) with h = x / 2 and the
+// hardware's approximate tanh (about 2^-11 error), one special-function
+// operation instead of two, under the bf16 rounding of the output.
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+template <typename TIn>
+__device__ __forceinline__ float silu(float x) {
+  if constexpr (sizeof(TIn) == 2) {
+    const float h = 0.5f * x;
+    return fmaf(h, tanh_approx(h), h);
+  } else {
+    return __fdividef(x, 1.f + __expf(-x));
+  }
+}
 
 template <typename TIn, int D>
 __global__ void __launch_bounds__(PrepCfg<TIn, D>::kThreads, PrepCfg<TIn, D>::kMinBlocks)
@@ -210,9 +226,9 @@ __global__ void __launch_bounds__(PrepCfg<TIn, D>::kThreads, PrepCfg<TIn, D>::kM
         const float4 f = *reinterpret_cast<const float4*>(swt + s * D + ch);
         ft[s][0] = f.x; ft[s][1] = f.y; ft[s][2] = f.z; ft[s][3] = f.w;
       }
+      float o[kTPT][4];
 #pragma unroll
       for (int k = 0; k < kTPT; ++k) {
-        float o[4];
 #pragma unroll
         for (int cp = 0; cp < 2; ++cp) {  // channel pairs: packed fp32x2 FMAs, each lane as fmaf
           float2 v = make_float2(0.f, 0.f);
@@ -220,20 +236,50 @@ __global__ void __launch_bounds__(PrepCfg<TIn, D>::kThreads, PrepCfg<TIn, D>::kM
           for (int s = 0; s < 5; ++s)
             v = __ffma2_rn(make_float2(ft[s][2 * cp], ft[s][2 * cp + 1]),
                            make_float2(ring[s][k][2 * cp], ring[s][k][2 * cp + 1]), v);
-          o[2 * cp] = silu(v.x);
-          o[2 * cp + 1] = silu(v.y);
+          o[k][2 * cp] = silu<TIn>(v.x);
+          o[k][2 * cp + 1] = silu<TIn>(v.y);
         }
-        float sc = 1.f;
-        if (which == 0) {
-          float ss = o[0] * o[0] + o[1] * o[1] + o[2] * o[2] + o[3] * o[3];
+      }
+      // Key norm: each token's sum of squares over the lanes of its channel group.
+      float sc[kTPT];
 #pragma unroll
-          for (int off = C::kLanesPerGroup / 2; off; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-          sc = rsqrtf(ss + p.l2_eps);
+      for (int k = 0; k < kTPT; ++k) sc[k] = 1.f;
+      if (which == 0) {
+        float ss[kTPT];
+#pragma unroll
+        for (int k = 0; k < kTPT; ++k)
+          ss[k] = o[k][0] * o[k][0] + o[k][1] * o[k][1] + o[k][2] * o[k][2] + o[k][3] * o[k][3];
+        if constexpr (C::kLanesPerGroup == 32 && kTPT == 4) {
+          // The four tokens' sums at once over the whole warp (ten shuffles, not
+          // twenty): after the halving steps lane l holds token (l >> 3) & 3's.
+          const bool b4 = lane & 16, b3 = lane & 8;
+          float a2[2];
+#pragma unroll
+          for (int i = 0; i < 2; ++i)
+            a2[i] = (b4 ? ss[i + 2] : ss[i]) + __shfl_xor_sync(0xffffffffu, b4 ? ss[i] : ss[i + 2], 16);
+          float e = (b3 ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, b3 ? a2[0] : a2[1], 8);
+#pragma unroll
+          for (int off = 4; off; off >>= 1) e += __shfl_xor_sync(0xffffffffu, e, off);
+          const float mine = rsqrtf(e + p.l2_eps);
+#pragma unroll
+          for (int k = 0; k < kTPT; ++k) sc[k] = __shfl_sync(0xffffffffu, mine, k << 3);
+        } else {
+#pragma unroll
+          for (int k = 0; k < kTPT; ++k) {
+            float v = ss[k];
+#pragma unroll
+            for (int off = C::kLanesPerGroup / 2; off; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+            sc[k] = rsqrtf(v + p.l2_eps);
+          }
         }
+      }
+#pragma unroll
+      for (int k = 0; k < kTPT; ++k) {
         const int x = x0 + kTPT * xg + k;
         if (x < gw) {
           const long long ot = (((long long)b * H + h) * T + to) * U + (long long)y * gw + x;
-          PrepIO<TIn>::store4(out + ot * D + ch, make_float4(o[0] * sc, o[1] * sc, o[2] * sc, o[3] * sc));
+          PrepIO<TIn>::store4(out + ot * D + ch,
+                              make_float4(o[k][0] * sc[k], o[k][1] * sc[k], o[k][2] * sc[k], o[k][3] * sc[k]));
         }
       }
     }
