@@ -61,3 +61,14 @@ def test_attention_pair_count_matches_the_oracles_visible_sets():
         want = sum(len(visible_frames(t, cfg.chunk, cfg.T)) for t in range(cfg.T)) * cfg.U * cfg.U
         assert bench.attention_pairs(cfg) == want
         assert bench.attention_flops(cfg) == 4 * cfg.d * want * cfg.B * cfg.H
+
+
+def test_split_scan_counts_as_the_frame_scan():
+    """The two-CTA scan does the frame scan's work: the same algorithmic bytes
+    (one read of each P_t image pair, B_t and alpha_t, the readout states out)
+    and flops, and its source is hashed for the traffic table."""
+    for name in ("h3", "long", "hires"):
+        cfg = CONFIGS[name]
+        assert bench.kernel_bytes("scan_split_tc", cfg) == bench.kernel_bytes("scan_tc", cfg) > 0
+        assert bench.kernel_flops("scan_split_tc", cfg) == bench.kernel_flops("scan_tc", cfg) > 0
+    assert bench.source_digest("scan_split_tc") != bench.source_digest("scan_tc")
